@@ -1,0 +1,548 @@
+"""CPU oracle for decode attention over an asymmetrically quantized KV cache.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this file:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference arm use it.  It shares no code with the CUDA library; it is a plain,
+slow restatement of what the method computes, in numpy.
+
+What it follows
+---------------
+* "[Framework] The Asymmetric Key-Value Cache Compression", §III (Pillar I,
+  KIVI partitioning): keys are quantized per channel, values per token, and
+  the most recent tokens stay in an FP16 window.
+* "Asymmetric Key-Value Quantization: 2-Bit Values and 4-Bit Keys under
+  Long-Context Drift", §1: attn(Q, K, V) = softmax(Q K^T / sqrt(d)) V;
+  §2.1: the output is sum_j alpha_j v_j; §3.1: keys at 4 bits, values at
+  2 bits (K2/V2 is the 2-bit KIVI setting of the first page, §III).
+* InnerQ abstract (page "WUSH-KV: KV Cache Quantization with Data-Adaptive
+  Transforms", third abstract): per-group asymmetric quantization.
+
+Readings where the pages are silent (each is listed in the design notes):
+* quantizer: uniform asymmetric min/scale with Q = 2^b - 1 levels;
+  s = fp16(fp32(max - min) / Q), z = fp16(min),
+  code = clamp(rne(fp32(fp32(x - z) / s)), 0, Q), computed with the STORED
+  fp16 s and z widened to fp32; s == 0 gives code 0 everywhere.
+* every K/V value entering the cache is first rounded to fp16 (the cache's
+  precision, the FP16 window of §III); quantization acts on those values, so
+  a token quantized at prefill and one that passed through the fp16 tail give
+  the same bytes.
+* key groups: G consecutive tokens from position 0 of each sequence; value
+  groups: G consecutive channels of one token; the tail holds the n mod G
+  newest tokens of both K and V.
+* GQA: query head h reads kv head floor(h / (Hq / Hkv)).
+* attention is evaluated in float64 on the dequantized cache
+  x_hat = code * s + z (tail tokens exactly as stored in fp16).
+
+The byte layout (``LAYOUT v1``) is a fixed per-group permutation of the codes
+and metadata; ``key_code_position``/``value_code_position`` and the
+``*_meta_index`` functions state it element by element.
+
+Parity is pinned for every function here (see tests/test_oracle_*.py); no
+function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+LAYOUT_VERSION = 1
+
+
+# ---------------------------------------------------------------------------
+# configuration and byte accounting
+# ---------------------------------------------------------------------------
+@dataclass(frozen=True)
+class Config:
+    k_bits: int
+    v_bits: int
+    group: int
+    head_dim: int
+    n_q_heads: int
+    n_kv_heads: int
+    max_seqs: int = 1
+    max_tokens: int = 0
+
+    @property
+    def gqa(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def value_groups(self) -> int:  # J: value channel groups per token
+        return self.head_dim // self.group
+
+
+def block_sections(cfg: Config) -> dict:
+    """Byte offsets and sizes of the sections of one group block (LAYOUT v1).
+
+    Order: key codes, key scales, key mins, value codes, value scales,
+    value mins.  All scales/mins are IEEE binary16.
+    """
+    G, d = cfg.group, cfg.head_dim
+    J = cfg.value_groups
+    sizes = [
+        ("kcodes", G * d * cfg.k_bits // 8),
+        ("kscale", 2 * d),
+        ("kmin", 2 * d),
+        ("vcodes", G * d * cfg.v_bits // 8),
+        ("vscale", 2 * G * J),
+        ("vmin", 2 * G * J),
+    ]
+    out, off = {}, 0
+    for name, sz in sizes:
+        out[name] = (off, sz)
+        off += sz
+    out["total"] = (0, off)
+    return out
+
+
+def block_bytes(cfg: Config) -> int:
+    return block_sections(cfg)["total"][1]
+
+
+def bytes_per_token_head(cfg: Config) -> float:
+    """Packed bytes per (token, kv-head) in a full group: codes + fp16 pairs."""
+    return block_bytes(cfg) / cfg.group
+
+
+def fp16_bytes_per_token_head(d: int) -> int:
+    """Unquantized fp16 K and V: 2 tensors x d x 2 bytes."""
+    return 2 * d * 2
+
+
+def bits_per_coordinate(k_bits: int, v_bits: int, group: int = 0,
+                        with_metadata: bool = False) -> float:
+    """Average stored bits per K/V coordinate.
+
+    Without metadata this is the pages' (b_K + b_V) / 2 (second page §3.1:
+    (4 + 2) / 2 = 3).  With metadata, each group of ``group`` elements carries
+    one fp16 (scale, min) pair = 32 bits, for keys and for values.
+    """
+    avg = (k_bits + v_bits) / 2.0
+    if with_metadata:
+        avg += 32.0 / group
+    return avg
+
+
+def compression_vs_fp16(k_bits, v_bits, group=0, with_metadata=False) -> float:
+    return 16.0 / bits_per_coordinate(k_bits, v_bits, group, with_metadata)
+
+
+def kv_cache_bytes_fp16(layers: int, heads: int, head_dim: int, tokens: int) -> int:
+    """Bytes of an unquantized fp16 KV cache: K and V, 2 bytes per element."""
+    return 2 * layers * heads * head_dim * 2 * tokens
+
+
+# ---------------------------------------------------------------------------
+# quantizer (uniform asymmetric min/scale), fp32 arithmetic
+# ---------------------------------------------------------------------------
+def to_fp16(x) -> np.ndarray:
+    """Round to IEEE binary16, nearest-even (the cache's storage precision)."""
+    return np.asarray(x).astype(np.float16)
+
+
+def quantize_along(x16: np.ndarray, bits: int, axis: int):
+    """Quantize fp16 values with one (scale, min) per slice along ``axis``.
+
+    Returns (codes uint8 same shape as x16, scale fp16, min fp16) where scale
+    and min have ``axis`` removed.  Steps, all in IEEE fp32 with
+    round-to-nearest-even and no fused multiply-add:
+      mn, mx = exact min / max over the group
+      s32 = (mx - mn) / Q          ; Q = 2^bits - 1 levels
+      s = fp16(s32), z = fp16(mn)  ; the stored pair
+      code = clamp(rne((x - z) / s), 0, Q) using fp32(s), fp32(z);
+      code = 0 for every element when s == 0.
+    """
+    Q = np.float32(2 ** bits - 1)
+    x32 = np.asarray(x16, dtype=np.float16).astype(np.float32)
+    mn = x32.min(axis=axis)
+    mx = x32.max(axis=axis)
+    s32 = (mx - mn) / Q                      # fp32 subtract, fp32 IEEE divide
+    s16 = s32.astype(np.float16)
+    z16 = mn.astype(np.float16)
+    s_w = np.expand_dims(s16.astype(np.float32), axis)
+    z_w = np.expand_dims(z16.astype(np.float32), axis)
+    diff = x32 - z_w                         # fp32
+    safe = np.where(s_w == 0, np.float32(1), s_w)
+    t = diff / safe                          # fp32 IEEE divide
+    codes = np.clip(np.rint(t), 0, Q)        # rint: ties to even
+    codes = np.where(s_w == 0, np.float32(0), codes)
+    return codes.astype(np.uint8), s16, z16
+
+
+def quantize_keys(k16: np.ndarray, bits: int):
+    """Per-channel key quantization of key groups.
+
+    k16: [..., G, d] fp16 (G tokens of one kv-head per group).  One
+    (scale, min) per channel, shared by the G tokens ("[Framework] The
+    Asymmetric Key-Value Cache Compression", §III: quantize K per channel).
+    Returns codes [..., G, d], scale [..., d], min [..., d].
+    """
+    return quantize_along(k16, bits, axis=-2)
+
+
+def quantize_values(v16: np.ndarray, bits: int, group: int):
+    """Per-token value quantization.
+
+    v16: [..., T, d] fp16.  Each token's channels are cut into d / group
+    groups of ``group`` consecutive channels, one (scale, min) per
+    (token, channel group) (same page, §III: quantize V per token).
+    Returns codes [..., T, d], scale [..., T, d/group], min [..., T, d/group].
+    """
+    d = v16.shape[-1]
+    J = d // group
+    shp = v16.shape[:-1] + (J, group)
+    codes, s, z = quantize_along(np.asarray(v16).reshape(shp), bits, axis=-1)
+    return codes.reshape(v16.shape), s, z
+
+
+def dequantize(codes, scale, mn) -> np.ndarray:
+    """x_hat = code * s + z in float64 (scale/min broadcast by the caller)."""
+    return codes.astype(np.float64) * np.asarray(scale, np.float64) + np.asarray(mn, np.float64)
+
+
+def dequantize_keys(codes, s16, z16) -> np.ndarray:
+    """codes [..., G, d], s16/z16 [..., d] -> [..., G, d] float64."""
+    return dequantize(codes, np.asarray(s16)[..., None, :], np.asarray(z16)[..., None, :])
+
+
+def dequantize_values(codes, s16, z16, group) -> np.ndarray:
+    """codes [..., T, d], s16/z16 [..., T, d/group] -> [..., T, d] float64."""
+    d = codes.shape[-1]
+    J = d // group
+    c = codes.reshape(codes.shape[:-1] + (J, group))
+    x = dequantize(c, np.asarray(s16)[..., None], np.asarray(z16)[..., None])
+    return x.reshape(codes.shape)
+
+
+# ---------------------------------------------------------------------------
+# LAYOUT v1: element positions inside a group block
+# ---------------------------------------------------------------------------
+def key_code_position(t: int, c: int, d: int, bits: int):
+    """(byte, bit) of key code (token t, channel c) inside the key-code section.
+
+    Tokens are cut into tiles of 8 (nt = t // 8, r = t % 8) and channels into
+    tiles of 16 (kt = c // 16, cc = c % 16 -> v = cc // 8, i = (cc % 8) // 2,
+    e = cc % 2).  Lane = 4 r + i; operand p = 2 kt + v; each lane owns
+    d * bits / 32 bytes per token tile, read as 32-bit words holding
+    F = 16 / bits code pairs: word p // F, field (p % F) + F e, i.e. bit
+    bits * field of that little-endian word.
+    """
+    nt, r = divmod(t, 8)
+    kt, cc = divmod(c, 16)
+    v, rem = divmod(cc, 8)
+    i, e = divmod(rem, 2)
+    lane = 4 * r + i
+    p = 2 * kt + v
+    F = 16 // bits
+    w, f = divmod(p, F)
+    bit = bits * (f + F * e)
+    lane_bytes = d * bits // 32
+    byte = nt * 32 * lane_bytes + lane * lane_bytes + 4 * w + bit // 8
+    return byte, bit % 8
+
+
+def value_code_position(t: int, c: int, d: int, bits: int):
+    """(byte, bit) of value code (token t, channel c) inside the value-code section.
+
+    Tokens are cut into tiles of 16 (kv = t // 16, tk = t % 16 ->
+    kh = tk // 8, i = (tk % 8) // 2, e = tk % 2) and channels into tiles of
+    16 (mt = c // 16, cm = c % 16 -> hr = cm // 8, g = cm % 8).
+    Lane = 4 g + i; each lane owns d * bits / 16 bytes per token tile, read
+    as 32-bit words holding F = 16 / bits code pairs; a word covers
+    F / 4 channel tiles: word mt // (F/4), u = mt % (F/4),
+    field 2 u + hr + (F/2) kh + F e, i.e. bit bits * field.
+    """
+    kv, tk = divmod(t, 16)
+    kh, rem = divmod(tk, 8)
+    i, e = divmod(rem, 2)
+    mt, cm = divmod(c, 16)
+    hr, g = divmod(cm, 8)
+    lane = 4 * g + i
+    F = 16 // bits
+    w, u = divmod(mt, F // 4)
+    bit = bits * (2 * u + hr + (F // 2) * kh + F * e)
+    lane_bytes = d * bits // 16
+    byte = kv * 32 * lane_bytes + lane * lane_bytes + 4 * w + bit // 8
+    return byte, bit % 8
+
+
+def key_meta_index(c: int, d: int) -> int:
+    """Slot of channel c in the key scale (and key min) arrays of a block:
+    i (d/4) + 4 kt + 2 v + e with kt = c // 16, v = (c % 16) // 8,
+    i = (c % 8) // 2, e = c % 2."""
+    kt, cc = divmod(c, 16)
+    v, rem = divmod(cc, 8)
+    i, e = divmod(rem, 2)
+    return i * (d // 4) + 4 * kt + 2 * v + e
+
+
+def value_meta_index(t: int, j: int, J: int) -> int:
+    """Slot of (token t, channel group j) in the value scale (and min) arrays:
+    ((4 kv + i) J + j) 4 + 2 kh + e with kv = t // 16, kh = (t % 16) // 8,
+    i = (t % 8) // 2, e = t % 2."""
+    kv, tk = divmod(t, 16)
+    kh, rem = divmod(tk, 8)
+    i, e = divmod(rem, 2)
+    return ((4 * kv + i) * J + j) * 4 + 2 * kh + e
+
+
+def tail_key_index(t: int, c: int, d: int) -> int:
+    """Element index of the fp16 key-tail slot (t, c): token-major."""
+    return t * d + c
+
+
+def tail_value_index(t: int, c: int, d: int) -> int:
+    """Element index of the fp16 value-tail slot (t, c): token pairs
+    interleaved, ((t // 2) d + c) 2 + t % 2."""
+    return ((t // 2) * d + c) * 2 + (t % 2)
+
+
+def _code_slot_table(T: int, d: int, bits: int, pos_fn) -> np.ndarray:
+    """Invert a code-position function: for every (byte, slot) of a packed
+    code section, the flat index t * d + c of the code stored there.
+
+    Slot s of a byte holds bits [s * bits, (s + 1) * bits).  Asserts that the
+    position function is a bijection onto the section.
+    """
+    per = 8 // bits
+    nbytes = T * d * bits // 8
+    table = np.full((nbytes, per), -1, dtype=np.int64)
+    for t in range(T):
+        for c in range(d):
+            byte, bit = pos_fn(t, c, d, bits)
+            assert bit % bits == 0 and table[byte, bit // bits] == -1
+            table[byte, bit // bits] = t * d + c
+    assert (table >= 0).all()
+    return table
+
+
+_TABLES: dict = {}
+
+
+def _slot_table(kind: str, T: int, d: int, bits: int) -> np.ndarray:
+    key = (kind, T, d, bits)
+    if key not in _TABLES:
+        fn = key_code_position if kind == "k" else value_code_position
+        _TABLES[key] = _code_slot_table(T, d, bits, fn)
+    return _TABLES[key]
+
+
+def pack_codes(codes: np.ndarray, bits: int, kind: str) -> np.ndarray:
+    """Pack codes [..., T, d] (kind "k" or "v") into [..., T*d*bits/8] bytes."""
+    T, d = codes.shape[-2:]
+    table = _slot_table(kind, T, d, bits)
+    flat = codes.reshape(codes.shape[:-2] + (T * d,)).astype(np.uint32)
+    gathered = flat[..., table]                      # [..., nbytes, per]
+    shifts = (np.arange(table.shape[1], dtype=np.uint32) * bits)
+    return (gathered << shifts).sum(axis=-1).astype(np.uint8)
+
+
+def unpack_codes(buf: np.ndarray, T: int, d: int, bits: int, kind: str) -> np.ndarray:
+    """Inverse of ``pack_codes``: bytes [..., nbytes] -> codes [..., T, d]."""
+    table = _slot_table(kind, T, d, bits)
+    per = table.shape[1]
+    buf = np.asarray(buf, np.uint8).astype(np.uint32)
+    shifts = np.arange(per, dtype=np.uint32) * bits
+    vals = (buf[..., :, None] >> shifts) & ((1 << bits) - 1)     # [..., nbytes, per]
+    out = np.zeros(buf.shape[:-1] + (T * d,), dtype=np.uint8)
+    out[..., table.reshape(-1)] = vals.reshape(buf.shape[:-1] + (-1,))
+    return out.reshape(buf.shape[:-1] + (T, d))
+
+
+def _key_meta_perm(d: int) -> np.ndarray:
+    """perm[slot] = channel stored at that slot of the key scale/min arrays."""
+    perm = np.full(d, -1, np.int64)
+    for c in range(d):
+        perm[key_meta_index(c, d)] = c
+    assert (perm >= 0).all()
+    return perm
+
+
+def _value_meta_perm(G: int, J: int) -> np.ndarray:
+    """perm[slot] = t * J + j stored at that slot of the value scale/min arrays."""
+    perm = np.full(G * J, -1, np.int64)
+    for t in range(G):
+        for j in range(J):
+            perm[value_meta_index(t, j, J)] = t * J + j
+    assert (perm >= 0).all()
+    return perm
+
+
+def pack_blocks(cfg: Config, kc, ks, kz, vc, vs, vz) -> np.ndarray:
+    """Assemble group blocks (uint8 [..., block_bytes]) from codes and fp16
+    metadata: kc [..., G, d] key codes, ks/kz [..., d] fp16,
+    vc [..., G, d] value codes, vs/vz [..., G, J] fp16."""
+    sec = block_sections(cfg)
+    G, d, J = cfg.group, cfg.head_dim, cfg.value_groups
+    lead = kc.shape[:-2]
+    blk = np.zeros(lead + (block_bytes(cfg),), dtype=np.uint8)
+    o, n = sec["kcodes"]
+    blk[..., o:o + n] = pack_codes(kc, cfg.k_bits, "k")
+    o, n = sec["vcodes"]
+    blk[..., o:o + n] = pack_codes(vc, cfg.v_bits, "v")
+    kp, vp = _key_meta_perm(d), _value_meta_perm(G, J)
+    metas = (("kscale", np.asarray(ks, np.float16)[..., kp]),
+             ("kmin", np.asarray(kz, np.float16)[..., kp]),
+             ("vscale", np.asarray(vs, np.float16).reshape(lead + (G * J,))[..., vp]),
+             ("vmin", np.asarray(vz, np.float16).reshape(lead + (G * J,))[..., vp]))
+    for name, arr in metas:
+        o, n = sec[name]
+        blk[..., o:o + n] = np.ascontiguousarray(arr).view(np.uint8)
+    return blk
+
+
+def pack_block(cfg: Config, kc, ks, kz, vc, vs, vz) -> np.ndarray:
+    """One group block (see ``pack_blocks``)."""
+    return pack_blocks(cfg, kc, ks, kz, vc, vs, vz)
+
+
+def unpack_blocks(cfg: Config, blk: np.ndarray):
+    """Inverse of ``pack_blocks``: returns (kc, ks, kz, vc, vs, vz)."""
+    sec = block_sections(cfg)
+    G, d, J = cfg.group, cfg.head_dim, cfg.value_groups
+    blk = np.asarray(blk, dtype=np.uint8)
+    lead = blk.shape[:-1]
+    o, n = sec["kcodes"]
+    kc = unpack_codes(blk[..., o:o + n], G, d, cfg.k_bits, "k")
+    o, n = sec["vcodes"]
+    vc = unpack_codes(blk[..., o:o + n], G, d, cfg.v_bits, "v")
+
+    def half(name):
+        o, n = sec[name]
+        return np.ascontiguousarray(blk[..., o:o + n]).view(np.float16)
+
+    kp, vp = _key_meta_perm(d), _value_meta_perm(G, J)
+    ks = np.zeros(lead + (d,), np.float16)
+    kz = np.zeros(lead + (d,), np.float16)
+    ks[..., kp] = half("kscale")
+    kz[..., kp] = half("kmin")
+    vs = np.zeros(lead + (G * J,), np.float16)
+    vz = np.zeros(lead + (G * J,), np.float16)
+    vs[..., vp] = half("vscale")
+    vz[..., vp] = half("vmin")
+    return kc, ks, kz, vc, vs.reshape(lead + (G, J)), vz.reshape(lead + (G, J))
+
+
+def unpack_block(cfg: Config, blk: np.ndarray):
+    return unpack_blocks(cfg, blk)
+
+
+# ---------------------------------------------------------------------------
+# the cache: groups + fp16 tail, as a function of the token history
+# ---------------------------------------------------------------------------
+def split_tokens(n: int, group: int):
+    """(N, T): tokens in full key groups, tokens in the fp16 tail (n mod G)."""
+    T = n % group
+    return n - T, T
+
+
+def quantize_group(cfg: Config, k16: np.ndarray, v16: np.ndarray):
+    """Quantize key groups and their values: k16, v16 [..., G, d] fp16.
+    Returns (kc, ks, kz, vc, vs, vz)."""
+    kc, ks, kz = quantize_keys(k16, cfg.k_bits)
+    vc, vs, vz = quantize_values(v16, cfg.v_bits, cfg.group)
+    return kc, ks, kz, vc, vs, vz
+
+
+def grouped(cfg: Config, x16: np.ndarray) -> np.ndarray:
+    """[n, Hkv, d] token history -> [Hkv, N/G, G, d] full groups."""
+    G = cfg.group
+    N, _ = split_tokens(x16.shape[0], G)
+    x = np.asarray(x16[:N], np.float16).reshape(N // G, G, x16.shape[1], x16.shape[2])
+    return x.transpose(2, 0, 1, 3)
+
+
+def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True):
+    """Expected cache contents for one sequence.
+
+    k16, v16: [n, Hkv, d] fp16 token history.  Returns a dict with
+    ``groups``: (kc, ks, kz, vc, vs, vz) with a leading [Hkv, n_groups] shape,
+    ``blocks``: [Hkv, n_groups, block_bytes] uint8 (if ``pack``),
+    ``tail_k``/``tail_v``: [Hkv, T, d] fp16 tail tokens, and N, T.
+    """
+    n = k16.shape[0]
+    N, T = split_tokens(n, cfg.group)
+    q = quantize_group(cfg, grouped(cfg, k16), grouped(cfg, v16))
+    out = {"N": N, "T": T, "groups": q}
+    if pack:
+        out["blocks"] = pack_blocks(cfg, *q)
+    out["tail_k"] = np.ascontiguousarray(np.asarray(k16[N:], np.float16).transpose(1, 0, 2))
+    out["tail_v"] = np.ascontiguousarray(np.asarray(v16[N:], np.float16).transpose(1, 0, 2))
+    return out
+
+
+def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray):
+    """Place T tail tokens [T, d] into the G-slot tail arrays (flat fp16,
+    LAYOUT v1); slots >= T are zero here (their device contents are
+    unspecified)."""
+    G, d = cfg.group, cfg.head_dim
+    tk = np.zeros(G * d, np.float16)
+    tv = np.zeros(G * d, np.float16)
+    for t in range(tail_k.shape[0]):
+        for c in range(d):
+            tk[tail_key_index(t, c, d)] = tail_k[t, c]
+            tv[tail_value_index(t, c, d)] = tail_v[t, c]
+    return tk, tv
+
+
+def dequantized_cache(cfg: Config, k16: np.ndarray, v16: np.ndarray):
+    """K_hat, V_hat [n, Hkv, d] float64: quantized groups dequantized, the
+    tail exactly as stored (fp16)."""
+    n, hkv, d = k16.shape
+    img = cache_image(cfg, k16, v16, pack=False)
+    N = img["N"]
+    kc, ks, kz, vc, vs, vz = img["groups"]
+    kh = np.zeros((n, hkv, d))
+    vh = np.zeros((n, hkv, d))
+    # [Hkv, ng, G, d] -> [N, Hkv, d]
+    kh[:N] = dequantize_keys(kc, ks, kz).transpose(1, 2, 0, 3).reshape(N, hkv, d)
+    vh[:N] = dequantize_values(vc, vs, vz, cfg.group).transpose(1, 2, 0, 3).reshape(N, hkv, d)
+    kh[N:] = np.asarray(k16[N:], np.float64)
+    vh[N:] = np.asarray(v16[N:], np.float64)
+    return kh, vh
+
+
+# ---------------------------------------------------------------------------
+# attention (fp64), the quantity the cache approximates
+# ---------------------------------------------------------------------------
+def softmax(x: np.ndarray, axis: int = -1) -> np.ndarray:
+    m = np.max(x, axis=axis, keepdims=True)
+    e = np.exp(x - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, gqa: int = 1) -> np.ndarray:
+    """Decode attention for one sequence, float64.
+
+    q [Hq, d]; k, v [n, Hkv, d].  Query head h attends with kv head
+    h // gqa: out_h = sum_t alpha_t v_t, alpha = softmax(q_h . k_t / sqrt(d))
+    ("Asymmetric Key-Value Quantization ...", §1 and §2.1).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    n = k.shape[0]
+    if n == 0:
+        raise ValueError("attention over an empty context is undefined")
+    hq, d = q.shape
+    out = np.zeros((hq, d))
+    for h in range(hq):
+        kv = h // gqa
+        logits = (k[:, kv, :] @ q[h]) / math.sqrt(d)
+        alpha = softmax(logits)
+        out[h] = alpha @ v[:, kv, :]
+    return out
+
+
+def attention_weights(q_h: np.ndarray, k_kv: np.ndarray) -> np.ndarray:
+    """alpha for one query head against [n, d] keys (float64)."""
+    d = q_h.shape[-1]
+    return softmax((np.asarray(k_kv, np.float64) @ np.asarray(q_h, np.float64)) / math.sqrt(d))
+
+
+def decode(cfg: Config, k16: np.ndarray, v16: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """Decode output for one sequence on the quantized cache, float64 [Hq, d]."""
+    kh, vh = dequantized_cache(cfg, k16, v16)
+    return attention(q, kh, vh, cfg.gqa)
