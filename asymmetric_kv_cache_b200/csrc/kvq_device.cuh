@@ -1,0 +1,160 @@
+// Device helpers for the libkvq kernels (sm_100a): bulk (TMA) copies into
+// shared memory with mbarrier completion, bounded waits, the fp16 tensor-core
+// tile, and exact unpacking of 2/4-bit codes into fp16 pairs.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace kvq {
+
+// Iteration cap of every spin on an mbarrier.  A wait that runs out sets the
+// workspace error word and the kernel abandons its remaining work instead of
+// hanging; no correct launch ever gets near the cap.
+constexpr uint32_t kWaitSpinLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Make barrier initialisation visible to the asynchronous (TMA) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's earlier shared-memory accesses before later bulk-copy
+// writes into the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared (this CTA), completion counted on bar.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of bar.  Returns false if the cap ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitSpinLimit; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  return false;
+}
+
+// D += A * B on one m16n8k16 tile, fp16 inputs, fp32 accumulate.
+// A row-major 16x16 (4 regs of half2), B column-major 16x8 (2 regs).
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
+  return *reinterpret_cast<__half2*>(&u);
+}
+
+// Pack two fp32 values into an fp16 pair (round to nearest even); lo -> bits 0..15.
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  return h2_as_u32(__floats2half2_rn(lo, hi));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Exact fp16 pair of the code pair in field f of a packed word.
+// BITS-bit codes, F = 16/BITS pairs per 32-bit word: the low element of
+// pair f sits at bits [BITS*f, BITS*f + BITS), the high element 16 bits
+// higher.  OR-ing a field into the mantissa of 1024.0 (0x6400) gives
+// 1024 + m*code with m = 2^(BITS*(f mod 8/BITS)); one fused multiply-add
+// by 1/m and -1024/m then yields the code exactly (all values are small
+// integers times powers of two).
+template <int BITS, int F_IDX>
+__device__ __forceinline__ uint32_t unpack_pair(uint32_t w) {
+  static_assert(BITS == 2 || BITS == 4, "2- or 4-bit codes");
+  constexpr int kPerByte = 8 / BITS;               // fields per byte half-word part
+  constexpr int kShift = (F_IDX >= kPerByte) ? 8 : 0;
+  constexpr int kF = F_IDX % kPerByte;
+  constexpr uint32_t kLowMask = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
+  constexpr uint32_t kMask = kLowMask << (BITS * kF);
+  constexpr float kMul = float(1u << (BITS * kF));
+  const uint32_t x = ((w >> kShift) & kMask) | 0x64006400u;
+  const __half2 inv = __float2half2_rn(1.0f / kMul);
+  const __half2 off = __float2half2_rn(-1024.0f / kMul);
+  return h2_as_u32(__hfma2(u32_as_h2(x), inv, off));
+}
+
+// Runtime-field variant for loops that the compiler unrolls.
+template <int BITS>
+__device__ __forceinline__ uint32_t unpack_pair_rt(uint32_t w, int f) {
+  if (BITS == 4) {
+    switch (f) {
+      case 0: return unpack_pair<4, 0>(w);
+      case 1: return unpack_pair<4, 1>(w);
+      case 2: return unpack_pair<4, 2>(w);
+      default: return unpack_pair<4, 3>(w);
+    }
+  } else {
+    switch (f) {
+      case 0: return unpack_pair<2, 0>(w);
+      case 1: return unpack_pair<2, 1>(w);
+      case 2: return unpack_pair<2, 2>(w);
+      case 3: return unpack_pair<2, 3>(w);
+      case 4: return unpack_pair<2, 4>(w);
+      case 5: return unpack_pair<2, 5>(w);
+      case 6: return unpack_pair<2, 6>(w);
+      default: return unpack_pair<2, 7>(w);
+    }
+  }
+}
+
+__device__ __forceinline__ float load_as_float(const void* base, int64_t idx, int dtype) {
+  // dtype: 0 fp16, 1 bf16, 2 fp32 (kvq_dtype)
+  if (dtype == 0) return __half2float(reinterpret_cast<const __half*>(base)[idx]);
+  if (dtype == 1) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
+  return reinterpret_cast<const float*>(base)[idx];
+}
+
+}  // namespace kvq

@@ -1,0 +1,120 @@
+// Internal declarations shared by the host side of libkvq (kvq_abi.cpp) and
+// its CUDA kernels.  Geometry only: the offsets of LAYOUT v1 (documented in
+// include/kvq.h) and the launch entry points of each kernel family.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// Upper bound on decode CTAs; sizes the split-partial region of the
+// workspace (two partial slots per CTA: its first and its last piece).
+constexpr int kMaxDecodeCtas = 1024;
+// At most this many query heads share one pass over a kv head (the M = 16
+// rows of the tensor-core tile hold up to 8 heads plus their low halves).
+constexpr int kHeadsPerSlice = 8;
+// Sequences per append launch (per-sequence arguments travel as kernel
+// parameters); longer batches are split into several launches.
+constexpr int kAppendMaxSeqs = 512;
+// Sequences per decode call (the CTA-local slot prefix lives in shared memory).
+constexpr int kMaxSeqsDecode = 8192;
+
+struct Geom {
+  int32_t kb, vb, G, d, hq, hkv, gqa, J, slices;
+  int32_t max_seqs, max_tokens, max_groups;
+  int32_t block_bytes;
+  int32_t sec_kcodes, sec_kscale, sec_kmin, sec_vcodes, sec_vscale, sec_vmin;
+  int64_t lens_off, counters_off, blocks_off, tails_off, tail_bytes, total_bytes;
+};
+
+// Workspace of kvq_decode: [error word | tickets | partials].
+struct WsLayout {
+  int64_t err_off, tickets_off, partials_off, total;
+  int32_t units;      // tickets
+  int32_t slot_floats; // floats per partial slot: heads * (d + 2)
+};
+
+inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Fill g from a validated configuration (no checks here).
+inline void make_geom(const kvq_config& c, Geom* g) {
+  g->kb = c.k_bits;
+  g->vb = c.v_bits;
+  g->G = c.group;
+  g->d = c.head_dim;
+  g->hq = c.n_q_heads;
+  g->hkv = c.n_kv_heads;
+  g->gqa = c.n_q_heads / c.n_kv_heads;
+  g->J = c.head_dim / c.group;
+  g->slices = (g->gqa + kHeadsPerSlice - 1) / kHeadsPerSlice;
+  g->max_seqs = c.max_seqs;
+  g->max_tokens = c.max_tokens;
+  g->max_groups = c.max_tokens / c.group;
+  const int G = g->G, d = g->d, J = g->J;
+  int off = 0;
+  g->sec_kcodes = off; off += G * d * g->kb / 8;
+  g->sec_kscale = off; off += 2 * d;
+  g->sec_kmin = off;   off += 2 * d;
+  g->sec_vcodes = off; off += G * d * g->vb / 8;
+  g->sec_vscale = off; off += 2 * G * J;
+  g->sec_vmin = off;   off += 2 * G * J;
+  g->block_bytes = off;
+  int64_t pos = 0;
+  g->lens_off = pos;
+  pos = align_up(pos + 4LL * c.max_seqs, 256);
+  g->counters_off = pos;   // append completion tickets, one per sequence
+  pos = align_up(pos + 4LL * c.max_seqs, 256);
+  g->blocks_off = pos;
+  pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->max_groups * g->block_bytes, 256);
+  g->tails_off = pos;
+  g->tail_bytes = 4LL * G * d;  // K tail + V tail, fp16
+  pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->tail_bytes, 256);
+  g->total_bytes = pos;
+}
+
+inline void make_ws_layout(const Geom& g, WsLayout* w) {
+  w->units = g.max_seqs * g.hkv * g.slices;
+  w->slot_floats = kHeadsPerSlice * (g.d + 2);
+  w->err_off = 0;
+  w->tickets_off = 256;
+  w->partials_off = align_up(w->tickets_off + 4LL * w->units, 256);
+  w->total = align_up(w->partials_off + 2LL * kMaxDecodeCtas * w->slot_floats * 4, 256);
+}
+
+// ---- append / quantize ----------------------------------------------------
+// Per-sequence arguments of one append launch.  The current lengths are
+// not among them: the kernel reads them from the device copy, so a captured
+// append stays correct when replayed (as long as its task counts do not
+// depend on the lengths, i.e. every n_new < G).
+struct AppendSeqs {
+  int32_t n;                           // sequences in this launch
+  int32_t seq0;                        // index of the first one in the cache
+  int32_t task_prefix[kAppendMaxSeqs + 1];
+  int32_t row_off[kAppendMaxSeqs];     // first input row of each sequence
+  int32_t n_new[kAppendMaxSeqs];
+};
+
+cudaError_t launch_append(const Geom& g, unsigned char* cache, const void* k, const void* v,
+                          int dtype, const AppendSeqs& seqs, int n_tasks, cudaStream_t stream);
+
+// ---- decode ---------------------------------------------------------------
+struct DecodeArgs {
+  const unsigned char* cache;
+  const void* q;
+  int32_t q_dtype;
+  void* out;             // fp16 [n_seq][hq][d]
+  unsigned char* ws;
+  int32_t n_seq;
+};
+
+// Resident-CTA cap of the decode kernel for this geometry on the current device.
+cudaError_t decode_max_ctas(const Geom& g, int* max_ctas);
+cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
+                          cudaStream_t stream);
+
+}  // namespace kvq

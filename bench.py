@@ -1,0 +1,528 @@
+"""Benchmark of the quantized-KV decode step on B200.
+
+One step = one decode step of one attention layer over a batch: append the
+new token of every sequence to the cache (quantizing and flushing a key
+group whenever a tail fills) and run split-K decode attention over the
+whole cache (groups + fp16 tail), on inputs already resident in HBM.
+
+Default workload: the Llama-3-8B-shaped layer (8 sequences, 32 query / 8 kv
+heads, head_dim 128, K4/V2, G = 32), contexts centred on 4096 + 17 tokens.
+The step rotates over C copies of the cache (each its own buffer, > 4x L2 in
+total) so every decode reads its cache from HBM; each copy's contexts start
+below 4113 so that over the timed steps their mean is 4113.
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA
+graphs (one graph = one round over the copies; two instances alternate so
+that CUDA events around every decode can be read while the next round
+runs), bracketed by barrier + synchronize, CUDA events on the launch
+stream, max over ranks.  Under torchrun every rank runs its own replica
+(weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (test infrastructure) on the same
+workload and metric, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV tokens/s on K4/V2 cache; achieved HBM GB/s vs B200 peak"
+UNIT = "KV tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+class Workload:
+    def __init__(self, args, rank: int):
+        from asymmetric_kv_cache_b200 import inputs
+        self.name = args.workload
+        if self.name != "llama3_8b":
+            raise SystemExit(f"unknown workload {self.name}")
+        self.batch, self.hq, self.hkv, self.d = 8, 32, 8, 128
+        self.kb, self.vb, self.G = 4, 2, 32
+        self.center = 4096 + 17
+        self.K, self.W = args.steps, args.warmup
+        per = L2_BYTES * 4 / (self.batch * self.hkv * self.center * 128) + 1
+        self.C = args.copies or int(max(16, math.ceil(per), math.ceil(self.K / 64)))
+        self.C = min(self.C, 1024)
+        self.seed = inputs.SEED_BASE + 1 + 1000 * rank
+        # appends per copy: step s uses copy s % C
+        total = self.W + self.K
+        self.n_warm = [sum(1 for s in range(self.W) if s % self.C == c) for c in range(self.C)]
+        self.n_time = [sum(1 for s in range(self.W, total) if s % self.C == c) for c in range(self.C)]
+        self.prefill = [self.center - self.n_warm[c] - self.n_time[c] // 2 for c in range(self.C)]
+        # headroom for the end-to-end pass that follows the timed steps
+        self.e2e_steps = min(args.e2e_steps, 4 * self.C)
+        self.max_tokens = max(p + w + t for p, w, t in zip(self.prefill, self.n_warm, self.n_time))
+        self.max_tokens += -(-self.e2e_steps // self.C) + 1
+
+    def make_inputs(self):
+        from asymmetric_kv_cache_b200 import inputs
+        rng = np.random.default_rng(self.seed)
+        n = max(self.prefill)
+        ks = np.stack([inputs.keys_channel_outliers(rng, n, self.hkv, self.d) for _ in range(self.batch)])
+        vs = np.stack([inputs.values_token_norms(rng, n, self.hkv, self.d) for _ in range(self.batch)])
+        pool = 64
+        nk, nv = inputs.append_stream(self.seed + 7, self.batch, pool, self.hkv, self.d)
+        q = rng.standard_normal((pool, self.batch, self.hq, self.d)).astype(np.float16)
+        return ks.astype(np.float16), vs.astype(np.float16), nk, nv, q
+
+    def algorithmic_bytes(self, lens) -> int:
+        """codes + fp16 (scale, min) pairs + fp16 tail + queries of one decode."""
+        blk = self.G * self.d * (self.kb + self.vb) // 8 + 4 * self.d + 4 * self.d
+        tot = 0
+        for n in lens:
+            ng, T = n // self.G, n % self.G
+            tot += self.hkv * (ng * blk + T * 2 * self.d * 2)
+        return tot + self.batch * self.hq * self.d * 2
+
+
+def run_ours(args, rank, world, device):
+    import torch
+    from asymmetric_kv_cache_b200 import kvq
+
+    wl = Workload(args, rank)
+    ks, vs, nk, nv, q = wl.make_inputs()
+    spec = kvq.CacheSpec(wl.kb, wl.vb, wl.G, wl.d, wl.hq, wl.hkv, wl.batch, wl.max_tokens)
+    caches = []
+    k_dev = torch.from_numpy(ks).to(device)   # [B, n, hkv, d]
+    v_dev = torch.from_numpy(vs).to(device)
+    for c in range(wl.C):
+        cache = kvq.KVQCache(spec, device=device)
+        P = wl.prefill[c]
+        kk = k_dev[:, :P].reshape(-1, wl.hkv, wl.d).contiguous()
+        vv = v_dev[:, :P].reshape(-1, wl.hkv, wl.d).contiguous()
+        cache.append(kk, vv, [P] * wl.batch)
+        caches.append(cache)
+        if c:
+            cache.workspace = caches[0].workspace   # calls never overlap: share one workspace
+    del k_dev, v_dev
+    pool = q.shape[0]
+    nk_dev = [torch.from_numpy(x).to(device) for x in nk]
+    nv_dev = [torch.from_numpy(x).to(device) for x in nv]
+    q_dev = [torch.from_numpy(x).to(device) for x in q]
+    out = torch.empty((wl.batch, wl.hq, wl.d), dtype=torch.float16, device=device)
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.synchronize(device)
+
+    def step(s, strm):
+        c = s % wl.C
+        caches[c].append(nk_dev[s % pool], nv_dev[s % pool], [1] * wl.batch, stream=strm)
+        caches[c].decode(q_dev[s % pool], out=out, stream=strm)
+
+    # ---- warm-up (eager: also sets launch attributes before capture)
+    with torch.cuda.stream(stream):
+        for s in range(wl.W):
+            step(s, stream)
+    stream.synchronize()
+
+    # ---- capture: a round covers steps W + r*C ... of every copy once
+    C = wl.C
+    steps_in_round = min(C, wl.K)
+
+    def capture(n_steps, first_step):
+        evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_steps)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_steps):
+                s = first_step + i
+                c = s % C
+                caches[c].append(nk_dev[s % pool], nv_dev[s % pool], [1] * wl.batch, stream=stream)
+                evs[i][0].record(stream)
+                caches[c].decode(q_dev[s % pool], out=out, stream=stream)
+                evs[i][1].record(stream)
+        return g, evs
+
+    # the copy of step s is s % C, so every round starts at a multiple of C
+    # relative to the first timed step W; record the round in that order
+    rounds = wl.K // C
+    rem = wl.K - rounds * C
+    gA = capture(steps_in_round, wl.W) if rounds else None
+    gB = capture(steps_in_round, wl.W) if rounds > 1 else None
+    gR = capture(rem, wl.W + rounds * C) if rem else None
+    for cache in caches:          # capture advanced the host mirrors only
+        cache.sync_lengths(stream)
+
+    # host view of every copy's length at each timed step (for the metric)
+    lens_at = []
+    cur = [wl.prefill[c] + wl.n_warm[c] for c in range(C)]
+    for s in range(wl.W, wl.W + wl.K):
+        c = s % C
+        cur[c] += 1
+        lens_at.append(cur[c])
+    kv_tokens = sum(L * wl.batch for L in lens_at)
+    alg_bytes = sum(wl.algorithmic_bytes([L] * wl.batch) for L in lens_at)
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        tdist.barrier()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    decode_ms = []
+    elapsed_ok = True
+
+    def collect(evs):
+        nonlocal elapsed_ok
+        for a, b in evs:
+            try:
+                decode_ms.append(a.elapsed_time(b))
+            except Exception:
+                elapsed_ok = False
+
+    insts = [x for x in (gA, gB) if x is not None]
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        pending = None
+        for r in range(rounds):
+            g, evs = insts[r % len(insts)]
+            g.replay()
+            if len(insts) == 1:
+                # one instance: its events must be read before it is replayed again
+                evs[-1][1].synchronize()
+                collect(evs)
+            else:
+                # two instances: read the previous round while this one runs
+                if pending is not None:
+                    pending[-1][1].synchronize()
+                    collect(pending)
+                pending = evs
+        if gR is not None:
+            gR[0].replay()
+        t1.record(stream)
+    t1.synchronize()
+    if pending is not None and len(insts) > 1:
+        collect(pending)
+    if gR is not None:
+        collect(gR[1])
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    if dist:
+        import torch.distributed as tdist
+        tt = torch.tensor([total_ms], device=device)
+        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+        tdist.barrier()
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, wl, caches, nk, nv, q, stream, device)
+
+    for cache in caches:
+        if cache.workspace_status(stream) != 0:
+            raise RuntimeError("decode kernel reported a failed wait")
+
+    value = kv_tokens * world / (total_ms / 1e3)
+    dec_avg_ms = statistics.fmean(decode_ms) if decode_ms and elapsed_ok else None
+    peak, peak_kind = _peaks()
+    roof = None
+    if dec_avg_ms:
+        achieved = (alg_bytes / wl.K) / (dec_avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": _traffic(),
+                "kernel": "kvq decode_kernel<128,4,2,32>", "peak_kind": peak_kind,
+                "bytes_per_launch": int(alg_bytes / wl.K),
+                "avg_launch_us": round(dec_avg_ms * 1e3, 3)}
+    return {
+        "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
+        "clocks": clocks, "gpu_launches": 2 * wl.K, "wl": wl,
+        "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K,
+    }
+
+
+def run_e2e(args, wl, caches, nk, nv, q, stream, device):
+    """Same metric through the C ABI with host buffers: per step, pinned host
+    -> device copies of the new token and the query, append, decode, and the
+    output back to pinned host memory, all inside the timed region."""
+    import torch
+    steps = wl.e2e_steps
+    pool = q.shape[0]
+    hk = [torch.from_numpy(x).pin_memory() for x in nk]
+    hv = [torch.from_numpy(x).pin_memory() for x in nv]
+    hq = [torch.from_numpy(x).pin_memory() for x in q]
+    dk = torch.empty_like(hk[0], device=device)
+    dv = torch.empty_like(hv[0], device=device)
+    dq = torch.empty_like(hq[0], device=device)
+    dout = torch.empty((wl.batch, wl.hq, wl.d), dtype=torch.float16, device=device)
+    hout = torch.empty((wl.batch, wl.hq, wl.d), dtype=torch.float16).pin_memory()
+    for cache in caches:
+        cache.sync_lengths(stream)
+    lens0 = [cache.lengths(wl.batch)[0] for cache in caches]
+    kv = 0
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(steps):
+            c = s % wl.C
+            dk.copy_(hk[s % pool], non_blocking=True)
+            dv.copy_(hv[s % pool], non_blocking=True)
+            dq.copy_(hq[s % pool], non_blocking=True)
+            caches[c].append(dk, dv, [1] * wl.batch, stream=stream)
+            caches[c].decode(dq, out=dout, stream=stream)
+            hout.copy_(dout, non_blocking=True)
+            lens0[c] += 1
+            kv += lens0[c] * wl.batch
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    h2d = hk[0].numel() * 2 + hv[0].numel() * 2 + hq[0].numel() * 2
+    return {"value": kv / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": hout.numel() * 2, "steps": steps}
+
+
+def _traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "asymmetric_kv_cache_b200", "csrc", "kvq_decode.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if rec.get("kernel_sha256_16") != h:
+        return None
+    return rec.get("dram_bytes_per_launch_full_workload")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+def _oracle_unit_inputs():
+    """One (sequence, kv head) unit of the llama3_8b layer at its mean context:
+    4113 tokens of one kv head and the 4 query heads that read it."""
+    from asymmetric_kv_cache_b200 import inputs
+    rng = np.random.default_rng(inputs.SEED_BASE + 1)
+    n = 4096 + 17
+    k = inputs.keys_channel_outliers(rng, n, 1, 128).astype(np.float16)
+    v = inputs.values_token_norms(rng, n, 1, 128).astype(np.float16)
+    q = rng.standard_normal((4, 128)).astype(np.float16).astype(np.float32)
+    return k, v, q
+
+
+def oracle_unit(k, v, q, tokens):
+    """The oracle as it stands on the first `tokens` tokens of one unit:
+    quantize, dequantize and fp64 attention (returns KV tokens processed)."""
+    from oracle import kvq_oracle as o
+    cfg = o.Config(4, 2, 32, 128, 4, 1)
+    o.decode(cfg, k[:tokens], v[:tokens], q)
+    return tokens
+
+
+def cpu_oracle(budget_s: float):
+    """cpu_baseline: the oracle on whole units of the workload, one thread,
+    until budget_s seconds have passed.  A unit is 1/8 of a sequence (one kv
+    head, all its query heads), so one KV token of the unit is 1/8 of a
+    layer KV token; the rate is reported in layer KV tokens/s."""
+    from threadpoolctl import threadpool_limits
+    k, v, q = _oracle_unit_inputs()
+    n = k.shape[0]
+    done = 0
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        while True:
+            oracle_unit(k, v, q, n)
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+    return {"value": done * n / 8 / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, kv-head) units of the llama3_8b layer at context {n} "
+                      f"(quantize + dequantize + fp64 attention of 4 query heads), "
+                      f"1 thread, {el:.1f} s"}
+
+
+def reference_arm(args):
+    """--impl reference: W warm-up and K timed steps of the oracle; each step
+    is a bounded sample of the workload (one unit, its context cut to fit the
+    whole run into about two minutes)."""
+    from threadpoolctl import threadpool_limits
+    k, v, q = _oracle_unit_inputs()
+    n = k.shape[0]
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        oracle_unit(k, v, q, n)
+        t_unit = time.perf_counter() - t0
+        budget = 120.0
+        tokens = n
+        if (args.steps + args.warmup) * t_unit > budget:
+            frac = budget / ((args.steps + args.warmup) * t_unit)
+            tokens = max(32, int(n * frac) // 32 * 32)
+        for _ in range(args.warmup):
+            oracle_unit(k, v, q, tokens)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_unit(k, v, q, tokens)
+        el = time.perf_counter() - t0
+    value = args.steps * tokens / 8 / el
+    sample = (f"each step: one (sequence, kv-head) unit of the llama3_8b layer, first {tokens} "
+              f"of {n} tokens (quantize + dequantize + fp64 attention of 4 query heads), 1 thread")
+    return value, el * 1e3 / args.steps, sample
+
+
+def config_dict(wl, extra=None):
+    d = {"workload": "llama3_8b_layer_decode", "batch": wl.batch, "n_q_heads": wl.hq,
+         "n_kv_heads": wl.hkv, "head_dim": wl.d, "k_bits": wl.kb, "v_bits": wl.vb,
+         "group": wl.G, "context_mean": wl.center,
+         "step": "append 1 token per sequence (flush when a tail fills) + decode",
+         "copies": wl.C,
+         "l2": f"inputs larger than L2: {wl.C} cache copies rotated "
+               f"({wl.C * wl.algorithmic_bytes([wl.center] * wl.batch) / 1e9:.2f} GB)",
+         "parallelism": "replicas per GPU (weak scaling)"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--copies", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=512)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = Workload(args, 0)
+        value, ms, sample = reference_arm(args)
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": config_dict(wl, {"l2": "n/a (CPU oracle)"}),
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device(device))
+    res = run_ours(args, rank, world, device)
+    wl = res["wl"]
+    cb = cpu_oracle(args.cpu_budget) if (rank == 0 and world == 1) else None
+    if rank == 0:
+        line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "fp16", "data": "synthetic", "config": config_dict(wl),
+                "e2e": res["e2e"], "roofline": res["roofline"], "cpu_baseline": cb,
+                "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
+                "kv_tokens_per_step": res["kv_tokens_per_step"]}
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

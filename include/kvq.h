@@ -1,0 +1,226 @@
+/*
+ * kvq.h — C ABI of libkvq: decode-step attention over an asymmetrically
+ * quantized KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * Keys are quantized per channel and values per token, with uniform
+ * asymmetric (min + scale) codes, and the newest tokens stay in fp16:
+ *   "[Framework] The Asymmetric Key-Value Cache Compression", §III (Pillar I,
+ *   KIVI partitioning): K per channel, V per token, an FP16 window of recent
+ *   tokens; "Asymmetric Key-Value Quantization: 2-Bit Values and 4-Bit Keys
+ *   under Long-Context Drift", §3.1: keys at 4 bits, values at 2 bits.
+ * Decode attention is out_h = sum_t alpha_t v_t,
+ * alpha = softmax(q_h . k_t / sqrt(d))  (same report, §1 and §2.1), evaluated
+ * over the dequantized groups and the fp16 tail.
+ *
+ * Quantizer (bit-exact contract).  Every K/V element entering the cache is
+ * first rounded to IEEE binary16 (round to nearest even).  For each group,
+ * in IEEE fp32 with round-to-nearest-even and no fused multiply-add:
+ *     mn, mx = min / max over the group
+ *     s      = fp16( (mx - mn) / Q )            Q = 2^bits - 1
+ *     z      = fp16( mn )
+ *     code   = clamp( rne( (x - z) / s ), 0, Q )   with fp32(s), fp32(z);
+ *              code = 0 when s == 0.
+ * Key group: G consecutive tokens x one channel (G tokens from position 0 of
+ * each sequence).  Value group: G consecutive channels of one token.
+ * The n mod G newest tokens of each sequence (keys and values) sit in an
+ * fp16 tail; when the tail reaches G tokens it is quantized as the next group
+ * ("flush").  Query head h reads kv head h / (n_q_heads / n_kv_heads).
+ *
+ * Conventions
+ * -----------
+ *  - Every function returns kvq_status (0 = KVQ_OK); nothing throws.
+ *  - All device memory is owned by the caller.  The handle owns host state
+ *    only (configuration and a host mirror of the sequence lengths).
+ *  - Calls taking a stream (cudaStream_t passed as void*; NULL = legacy
+ *    default stream) are asynchronous on that stream; pointers must stay
+ *    valid until the stream has passed the call.  Argument errors are
+ *    detected on the host, before anything is launched, and leave the
+ *    cache unchanged.
+ *  - A handle is not thread-safe; distinct handles are independent.
+ *
+ * LAYOUT v1 of the cache buffer (all region offsets 256-byte aligned; see
+ * kvq_layout for the numbers):
+ *   lens   : int32 [max_seqs]                 device copy of the lengths
+ *   tickets: int32 [max_seqs]                 append completion counters (0 at rest)
+ *   blocks : [max_seqs][n_kv_heads][max_groups] group blocks of block_bytes
+ *   tails  : [max_seqs][n_kv_heads] { K tail fp16 [G][d] token-major,
+ *                                     V tail fp16 [G/2][d][2] token pairs }
+ *            K tail slot (t, c) is element t*d + c; V tail slot (t, c) is
+ *            element ((t/2)*d + c)*2 + t%2.
+ * A group block holds, in this order (byte offsets in kvq_layout):
+ *   key codes   G*d*kbits/8 bytes
+ *   key scales  d fp16, key mins d fp16
+ *   value codes G*d*vbits/8 bytes
+ *   value scales G*(d/G) fp16, value mins G*(d/G) fp16
+ * Code packing (little-endian 32-bit words, F = 16/bits code pairs per
+ * word, field f occupies bits [f*bits, (f+1)*bits)):
+ *   key (token t, channel c): nt = t/8, r = t%8, kt = c/16, v = (c%16)/8,
+ *     i = (c%8)/2, e = c%2; lane = 4r+i; p = 2kt+v;
+ *     byte offset = nt*32*LB + lane*LB + 4*(p/F) with LB = d*kbits/32,
+ *     field = p%F + F*e.
+ *   value (token t, channel c): kv = t/16, kh = (t%16)/8, i = (t%8)/2,
+ *     e = t%2, mt = c/16, hr = (c%16)/8, g = c%8; lane = 4g+i;
+ *     word = mt/(F/4), u = mt%(F/4); byte offset = kv*32*LB + lane*LB +
+ *     4*word with LB = d*vbits/16; field = 2u + hr + (F/2)*kh + F*e.
+ *   key scale/min of channel c sit at slot i*(d/4) + 4kt + 2v + e;
+ *   value scale/min of (token t, channel group j), J = d/G groups, sit at
+ *   slot ((4kv + i)*J + j)*4 + 2kh + e.
+ * (These are the tensor-core fragment orders the decode kernel reads with
+ * 128-bit loads; the packing is a fixed permutation, so every token still
+ * costs a fixed number of bits.)
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_LAYOUT_VERSION 1
+
+/* Exported entry points (the library is built with hidden visibility). */
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+typedef int32_t kvq_status;
+enum {
+  KVQ_OK = 0,
+  KVQ_ERR_NULL = 1,              /* a required pointer is NULL */
+  KVQ_ERR_CONFIG = 2,            /* unsupported bits / group / head_dim / heads */
+  KVQ_ERR_BUFFER_TOO_SMALL = 3,  /* cache or workspace buffer too small */
+  KVQ_ERR_CAPACITY = 4,          /* append past max_tokens or n_seq > max_seqs */
+  KVQ_ERR_EMPTY = 5,             /* decode over a sequence of length 0 */
+  KVQ_ERR_DTYPE = 6,             /* unsupported element type */
+  KVQ_ERR_CUDA = 7,              /* a CUDA call failed (see kvq_last_error) */
+  KVQ_ERR_ALIGN = 8,             /* a pointer is not suitably aligned */
+  KVQ_ERR_ARG = 9,               /* other invalid argument (negative count ...) */
+  KVQ_ERR_DEVICE = 10            /* a kernel reported a failed internal wait */
+};
+
+typedef enum { KVQ_FP16 = 0, KVQ_BF16 = 1, KVQ_FP32 = 2 } kvq_dtype;
+
+typedef struct {
+  int32_t k_bits;          /* 2 or 4 */
+  int32_t v_bits;          /* 2 or 4 */
+  int32_t group;           /* G: 32 or 64 */
+  int32_t head_dim;        /* d: 64 or 128 (d % G == 0) */
+  int32_t n_q_heads;       /* Hq, a multiple of n_kv_heads */
+  int32_t n_kv_heads;      /* Hkv >= 1 */
+  int32_t max_seqs;        /* sequences the buffer holds, >= 1 */
+  int32_t max_tokens;      /* capacity per sequence, >= 1 */
+  int32_t layout_version;  /* must be KVQ_LAYOUT_VERSION (or 0 = current) */
+} kvq_config;
+
+typedef struct {
+  uint64_t total_bytes;    /* cache buffer size */
+  uint64_t lens_offset;    /* int32[max_seqs] */
+  uint64_t counters_offset;/* int32[max_seqs], zero between calls */
+  uint64_t blocks_offset;  /* first group block */
+  uint64_t block_bytes;    /* one group block */
+  uint64_t max_groups;     /* floor(max_tokens / G) blocks per (seq, kv head) */
+  uint64_t tails_offset;   /* first tail */
+  uint64_t tail_bytes;     /* K tail + V tail of one (seq, kv head) = 4*G*d */
+  uint64_t kcodes_offset, kscale_offset, kmin_offset; /* within a block */
+  uint64_t vcodes_offset, vscale_offset, vmin_offset; /* within a block */
+} kvq_layout;
+
+typedef struct kvq_cache kvq_cache;
+
+/* Human-readable name of a status code (static string). */
+KVQ_API const char* kvq_status_string(kvq_status s);
+
+/* Detail of the last failure on the calling thread ("" if none).  The
+ * string stays valid until the next call on that thread. */
+KVQ_API const char* kvq_last_error(void);
+
+/* LAYOUT v1 offsets for a configuration (host only, no device work).
+ * Errors: KVQ_ERR_NULL, KVQ_ERR_CONFIG. */
+KVQ_API kvq_status kvq_layout_for(const kvq_config* cfg, kvq_layout* out);
+
+/* Bytes the caller must provide: the cache buffer and the decode workspace
+ * (split partials, per-unit tickets and an error word).  Either output
+ * pointer may be NULL.  Host only.  Errors: KVQ_ERR_NULL, KVQ_ERR_CONFIG. */
+KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* cache_bytes,
+                                    size_t* workspace_bytes);
+
+/* Bind a handle to a caller-owned device buffer of at least cache_bytes
+ * (256-byte aligned).  Validates the configuration on the host first
+ * (KVQ_ERR_NULL, KVQ_ERR_CONFIG, KVQ_ERR_BUFFER_TOO_SMALL, KVQ_ERR_ALIGN),
+ * then zeroes the device length and counter arrays synchronously on the
+ * current device (KVQ_ERR_CUDA if that fails).  The buffer is not otherwise
+ * touched. */
+KVQ_API kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_buf, size_t bytes,
+                            kvq_cache** out);
+
+/* Free the host handle (never the device buffer).  NULL is accepted. */
+KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
+
+/* Set every sequence length to 0 (host mirror and device copy, on stream). */
+KVQ_API kvq_status kvq_reset(kvq_cache* cache, void* stream);
+
+/* Append n_new[b] tokens to sequence b, for b in [0, n_seq).
+ * k, v: device arrays [sum_b n_new[b], n_kv_heads, head_dim] of dtype
+ * (fp16, bf16 or fp32), token-major, sequences concatenated in order b;
+ * 16-byte aligned.  n_new: host array of n_seq non-negative counts.
+ * Performs prefill quantization (whole groups straight from the input),
+ * per-step appends into the fp16 tail and the flush of a tail that reaches
+ * G tokens, all in one launch.  The kernel takes the current lengths from
+ * the device copy and advances it, so an append captured in a CUDA graph
+ * may be replayed provided every n_new[b] < G (the launch shape then does
+ * not depend on the lengths); after replays, kvq_sync_lengths refreshes the
+ * host mirror.  Values outside the fp16 range are not representable by the
+ * cache (their codes are unspecified).
+ * Errors (host side, cache unchanged): KVQ_ERR_NULL, KVQ_ERR_ARG,
+ * KVQ_ERR_CAPACITY (n_seq > max_seqs or a length would pass max_tokens),
+ * KVQ_ERR_DTYPE, KVQ_ERR_ALIGN; KVQ_ERR_CUDA if the launch fails. */
+KVQ_API kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype dtype,
+                      const int32_t* n_new, int32_t n_seq, void* stream);
+
+/* Decode attention for sequences [0, n_seq): q device [n_seq, n_q_heads, d]
+ * (fp16, bf16 or fp32, 16-byte aligned); out device [n_seq, n_q_heads, d]
+ * fp16.  workspace: device buffer of at least the workspace_bytes reported
+ * by kvq_cache_required_bytes, 256-byte aligned, zero-filled before its
+ * first use (kvq_workspace_init); every completed call leaves it ready for
+ * the next.  Calls that share a workspace must not overlap on the GPU.
+ * Errors (host side): KVQ_ERR_NULL, KVQ_ERR_ARG, KVQ_ERR_CAPACITY,
+ * KVQ_ERR_EMPTY (some sequence has length 0), KVQ_ERR_DTYPE,
+ * KVQ_ERR_ALIGN, KVQ_ERR_BUFFER_TOO_SMALL; KVQ_ERR_CUDA on launch failure.
+ * The kernel reads the lengths from the device copy, so a captured decode
+ * may be replayed while appends advance them (the launch shape, fixed at
+ * capture, stays valid as lengths grow).  A failed internal wait inside the
+ * kernel (never expected) is recorded in the workspace and reported by
+ * kvq_workspace_status.  The environment variable KVQ_DECODE_MAX_CTAS, if
+ * set to a positive integer, caps the number of CTAs (split granularity;
+ * results stay within rounding of each other). */
+KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* out,
+                      int32_t n_seq, void* workspace, size_t ws_bytes, void* stream);
+
+/* Zero-fill a decode workspace on stream (cudaMemsetAsync). */
+KVQ_API kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Read the workspace error word (synchronous copy on stream): KVQ_OK, or
+ * KVQ_ERR_DEVICE if some decode kernel gave up a bounded wait. */
+KVQ_API kvq_status kvq_workspace_status(const void* workspace, void* stream);
+
+/* Refresh the host length mirror from the device copy (synchronizes
+ * stream).  Needed after replaying captured appends. */
+KVQ_API kvq_status kvq_sync_lengths(kvq_cache* cache, void* stream);
+
+/* The configuration, layout and host length mirror of a handle. */
+KVQ_API kvq_status kvq_cache_config(const kvq_cache* cache, kvq_config* out);
+KVQ_API kvq_status kvq_cache_layout(const kvq_cache* cache, kvq_layout* out);
+KVQ_API kvq_status kvq_get_lengths(const kvq_cache* cache, int32_t* host_lens, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */
