@@ -84,24 +84,39 @@ struct WarpState {
   float m;              // running max of head (lane / 4), log2 domain
 };
 
-// Load this lane's query fragments for head `hd` (or zeros): rows g of the
-// A tile, channels 16kt + 2i + {0,1} and + 8 + {0,1}; q is pre-scaled by
+// Load this lane's query fragments (or zeros for a padding head): rows g of
+// the A tile, channels 16kt + 2i + {0,1} and + 8 + {0,1}; q is scaled by
 // log2(e)/sqrt(d) and split into fp16 high and low parts.
 template <int D>
 __device__ __forceinline__ void load_query(const void* q, int dtype, int64_t row, bool valid,
                                            int i4, uint32_t (&qh)[D / 16][2],
                                            uint32_t (&ql)[D / 16][2]) {
   const float sc = kLog2e * rsqrtf((float)D);
+  float2 x[D / 16][2];
 #pragma unroll
   for (int kt = 0; kt < D / 16; ++kt) {
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
-      const int c = 16 * kt + 8 * v + 2 * i4;
-      float x0 = 0.f, x1 = 0.f;
+      const int64_t idx = row * D + 16 * kt + 8 * v + 2 * i4;
+      float2 f = make_float2(0.f, 0.f);
       if (valid) {
-        x0 = load_as_float(q, row * D + c, dtype) * sc;
-        x1 = load_as_float(q, row * D + c + 1, dtype) * sc;
+        if (dtype == KVQ_FP16) {
+          f = __half22float2(*reinterpret_cast<const __half2*>(reinterpret_cast<const __half*>(q) + idx));
+        } else if (dtype == KVQ_BF16) {
+          f = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(reinterpret_cast<const __nv_bfloat16*>(q) + idx));
+        } else {
+          f = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(q) + idx);
+        }
       }
+      x[kt][v] = f;
+    }
+  }
+#pragma unroll
+  for (int kt = 0; kt < D / 16; ++kt) {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const float x0 = x[kt][v].x * sc, x1 = x[kt][v].y * sc;
       const __half2 h = __floats2half2_rn(x0, x1);
       const float2 hf = __half22float2(h);
       qh[kt][v] = h2_as_u32(h);
@@ -157,17 +172,17 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   uint32_t qs[C::KT][2];
   float bias[4] = {0.f, 0.f, 0.f, 0.f};
   {
-    const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
-    const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
+    uint32_t ksw[D / 8], kzw[D / 8];
+    lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8), ksw);
+    lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8), kzw);
 #pragma unroll
     for (int kt = 0; kt < C::KT; ++kt) {
       const uint32_t s0 = ksw[2 * kt], s1 = ksw[2 * kt + 1];
-      const uint32_t z0 = kzw[2 * kt], z1 = kzw[2 * kt + 1];
       qs[kt][0] = h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s0),
                                     __hmul2(u32_as_h2(ql[kt][0]), u32_as_h2(s0))));
       qs[kt][1] = h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s1),
                                     __hmul2(u32_as_h2(ql[kt][1]), u32_as_h2(s1))));
-      mma16816(bias, qh[kt][0], ql[kt][0], qh[kt][1], ql[kt][1], z0, z1);
+      mma16816(bias, qh[kt][0], ql[kt][0], qh[kt][1], ql[kt][1], kzw[2 * kt], kzw[2 * kt + 1]);
     }
   }
   const float b = bias[0] + bias[2];   // head g8: high-part rows + low-part rows
@@ -175,23 +190,21 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   // S = q' K^T over the G tokens
   float s[C::NT][2];
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
-#pragma unroll
-  for (int nt = 0; nt < C::NT; ++nt) {
+  static_for<C::NT>([&](auto nt_) {
+    constexpr int nt = decltype(nt_)::value;
     uint32_t kw[C::LWK];
-    const uint32_t* src = kcw + (nt * 32 + lane) * C::LWK;
-#pragma unroll
-    for (int w = 0; w < C::LWK; ++w) kw[w] = src[w];
+    lds_words<C::LWK>(kcw + (nt * 32 + lane) * C::LWK, kw);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int kt = 0; kt < C::KT; ++kt) {
-      const int p0 = 2 * kt, p1 = 2 * kt + 1;
-      const uint32_t b0 = unpack_pair_rt<KB>(kw[p0 / C::FK], p0 % C::FK);
-      const uint32_t b1 = unpack_pair_rt<KB>(kw[p1 / C::FK], p1 % C::FK);
+    static_for<C::KT>([&](auto kt_) {
+      constexpr int kt = decltype(kt_)::value;
+      constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
+      const uint32_t b0 = unpack_pair<KB, p0 % C::FK>(kw[p0 / C::FK]);
+      const uint32_t b1 = unpack_pair<KB, p1 % C::FK>(kw[p1 / C::FK]);
       mma16816(acc, qs[kt][0], 0u, qs[kt][1], 0u, b0, b1);
-    }
+    });
     s[nt][0] = acc[0] + b;
     s[nt][1] = acc[1] + b;
-  }
+  });
 
   uint32_t p[C::NT];
   softmax_update<D, C::NT, KB, VB, G>(st, s, p, lane);
@@ -200,8 +213,8 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
   const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
   const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
-#pragma unroll
-  for (int kv = 0; kv < C::KV; ++kv) {
+  static_for<C::KV>([&](auto kv_) {
+    constexpr int kv = decltype(kv_)::value;
     const uint32_t bp0 = p[2 * kv], bp1 = p[2 * kv + 1];
     uint32_t za0 = 0u, za2 = 0u;
     if (g8 < C::J) {
@@ -213,53 +226,77 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
     }
     mma16816(st.z, za0, 0u, za2, 0u, bp0, bp1);
 
+    uint32_t sw[2 * C::J];
+    lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
     uint32_t bs[C::J][2];
-    const uint32_t* ss = vsw + (4 * kv + i4) * C::J * 2;
 #pragma unroll
     for (int j = 0; j < C::J; ++j) {
-      bs[j][0] = h2_as_u32(__hmul2(u32_as_h2(bp0), u32_as_h2(ss[2 * j])));
-      bs[j][1] = h2_as_u32(__hmul2(u32_as_h2(bp1), u32_as_h2(ss[2 * j + 1])));
+      bs[j][0] = h2_as_u32(__hmul2(u32_as_h2(bp0), u32_as_h2(sw[2 * j])));
+      bs[j][1] = h2_as_u32(__hmul2(u32_as_h2(bp1), u32_as_h2(sw[2 * j + 1])));
     }
     uint32_t vw[C::LWV];
-    const uint32_t* src = vcw + (kv * 32 + lane) * C::LWV;
-#pragma unroll
-    for (int w = 0; w < C::LWV; ++w) vw[w] = src[w];
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) {
+    lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
+    static_for<C::MT>([&](auto mt_) {
+      constexpr int mt = decltype(mt_)::value;
       constexpr int TPW = C::FV / 4;     // channel tiles per word
-      const int wd = mt / TPW, u = mt % TPW;
-      const int j = (16 * mt) / G;
-      const uint32_t a0 = unpack_pair_rt<VB>(vw[wd], 2 * u);
-      const uint32_t a1 = unpack_pair_rt<VB>(vw[wd], 2 * u + 1);
-      const uint32_t a2 = unpack_pair_rt<VB>(vw[wd], 2 * u + C::FV / 2);
-      const uint32_t a3 = unpack_pair_rt<VB>(vw[wd], 2 * u + 1 + C::FV / 2);
+      constexpr int wd = mt / TPW, u = mt % TPW;
+      constexpr int j = (16 * mt) / G;
+      const uint32_t a0 = unpack_pair<VB, 2 * u>(vw[wd]);
+      const uint32_t a1 = unpack_pair<VB, 2 * u + 1>(vw[wd]);
+      const uint32_t a2 = unpack_pair<VB, 2 * u + C::FV / 2>(vw[wd]);
+      const uint32_t a3 = unpack_pair<VB, 2 * u + 1 + C::FV / 2>(vw[wd]);
       mma16816(st.o[mt], a0, a1, a2, a3, bs[j][0], bs[j][1]);
-    }
-  }
+    });
+  });
 }
 
-// The fp16 tail (T tokens, 0 < T < G) of one (sequence, kv head).
+// The fp16 tail (T tokens, 0 < T < G) of one (sequence, kv head), staged
+// 16 tokens at a time through the warp's (idle) ring with cp.async: key rows
+// and value token-pair rows, padded so that the fragment reads below are
+// free of bank conflicts; rows past T are zero-filled.
+template <int D>
+struct TailStage {
+  static constexpr int KROW = 2 * D + 16;       // bytes per padded key row
+  static constexpr int VROW = 4 * D + 16;       // bytes per padded value pair-row
+  static constexpr int VOFF = 16 * KROW;
+  static constexpr int BYTES = VOFF + 8 * VROW;
+};
+
 template <int D, int KB, int VB, int G>
 __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
                                              const __half* __restrict__ tk,
                                              const __half* __restrict__ tv, int T,
                                              const uint32_t (&qh)[D / 16][2],
-                                             const uint32_t (&ql)[D / 16][2], int lane) {
+                                             const uint32_t (&ql)[D / 16][2], int lane,
+                                             unsigned char* __restrict__ buf) {
   using C = DecCfg<D, KB, VB, G>;
+  using TS = TailStage<D>;
+  static_assert(TS::BYTES <= C::NST * C::BLK, "tail chunk must fit in a warp's ring");
   const int g8 = lane >> 2, i4 = lane & 3;
-  const uint32_t* tkw = reinterpret_cast<const uint32_t*>(tk);
-  const uint32_t* tvw = reinterpret_cast<const uint32_t*>(tv);
   for (int kv = 0; kv * 16 < T; ++kv) {
+    // stage 16 key rows and 8 value pair-rows (16-byte pieces)
+    for (int seg = lane; seg < 16 * (D / 8); seg += 32) {
+      const int r = seg / (D / 8), cs = seg % (D / 8), t = 16 * kv + r;
+      cp_async16(buf + r * TS::KROW + cs * 16, tk + (t < T ? (int64_t)t * D + cs * 8 : 0),
+                 t < T ? 16u : 0u);
+    }
+    for (int seg = lane; seg < 8 * (D / 4); seg += 32) {
+      const int pr = seg / (D / 4), cs = seg % (D / 4), pp = 8 * kv + pr;
+      cp_async16(buf + TS::VOFF + pr * TS::VROW + cs * 16,
+                 tv + (2 * pp < T ? (int64_t)pp * 2 * D + cs * 8 : 0), 2 * pp < T ? 16u : 0u);
+    }
+    cp_async_wait_all();
+    __syncwarp();
+
     float s[2][2];
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
-      const int tb = 16 * kv + 8 * n + g8;          // token of this lane's B column
-      const bool vb = tb < T;
+      const unsigned char* krow = buf + (8 * n + g8) * TS::KROW + 4 * i4;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kt = 0; kt < C::KT; ++kt) {
-        const uint32_t b0 = vb ? __ldg(tkw + (tb * D + 16 * kt + 2 * i4) / 2) : 0u;
-        const uint32_t b1 = vb ? __ldg(tkw + (tb * D + 16 * kt + 8 + 2 * i4) / 2) : 0u;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(krow + 32 * kt);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(krow + 32 * kt + 16);
         mma16816(acc, qh[kt][0], ql[kt][0], qh[kt][1], ql[kt][1], b0, b1);
       }
       const int t0 = 16 * kv + 8 * n + 2 * i4;      // tokens of this lane's C columns
@@ -270,21 +307,21 @@ __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
     softmax_update<D, 2, KB, VB, G>(st, s, p, lane);
     const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
     mma16816(st.z, ones, 0u, ones, 0u, p[0], p[1]);
-    // V^T fragments straight from the pair-interleaved tail; tokens >= T are
-    // zeroed (their slots hold stale data)
+    // V^T fragments; the second token of the last pair may be stale: mask it
     const int ta = 16 * kv + 2 * i4, tb = ta + 8;
-    const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : (ta < T ? 0x0000FFFFu : 0u);
-    const uint32_t mb = (tb + 1 < T) ? 0xFFFFFFFFu : (tb < T ? 0x0000FFFFu : 0u);
-    const int pa = (ta >> 1) * D, pb = (tb >> 1) * D;
+    const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+    const uint32_t mb = (tb + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+    const unsigned char* va = buf + TS::VOFF + i4 * TS::VROW + 4 * g8;
+    const unsigned char* vb = va + 4 * TS::VROW;
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) {
-      const int c = 16 * mt + g8;
-      const uint32_t a0 = ma ? (__ldg(tvw + pa + c) & ma) : 0u;
-      const uint32_t a1 = ma ? (__ldg(tvw + pa + c + 8) & ma) : 0u;
-      const uint32_t a2 = mb ? (__ldg(tvw + pb + c) & mb) : 0u;
-      const uint32_t a3 = mb ? (__ldg(tvw + pb + c + 8) & mb) : 0u;
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(va + 64 * mt) & ma;
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
       mma16816(st.o[mt], a0, a1, a2, a3, p[0], p[1]);
     }
+    __syncwarp();   // every lane is done with this chunk before the next copy
   }
 }
 
@@ -430,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (ok && Tb > 0 && slot1 == wb && slot0 <= ng && ((ng - slot0) % kWarps) == warp) {
       const __half* tk = reinterpret_cast<const __half*>(
           a.cache + g.tails_off + ((int64_t)b * g.hkv + kvh) * g.tail_bytes);
-      process_tail<D, KB, VB, G>(st, tk, tk + G * D, Tb, qh, ql, lane);
+      process_tail<D, KB, VB, G>(st, tk, tk + G * D, Tb, qh, ql, lane, wring);
     }
 
     // ---- merge the 4 warps (the ring is idle: every issued copy was waited on)
@@ -525,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 3)
         if (tid == 0) tickets[unit] = 0;
       }
     }
-    __syncthreads();   // merge area and ctl are reused by the next piece
+    fence_proxy_async_smem();   // generic accesses before the next bulk copies
+    __syncthreads();            // merge area and ctl are reused by the next piece
     pos += slot1 - slot0;
   }
 }

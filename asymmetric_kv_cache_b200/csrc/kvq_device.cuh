@@ -4,6 +4,8 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
+#include <utility>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -126,28 +128,46 @@ __device__ __forceinline__ uint32_t unpack_pair(uint32_t w) {
   return h2_as_u32(__hfma2(u32_as_h2(x), inv, off));
 }
 
-// Runtime-field variant for loops that the compiler unrolls.
-template <int BITS>
-__device__ __forceinline__ uint32_t unpack_pair_rt(uint32_t w, int f) {
-  if (BITS == 4) {
-    switch (f) {
-      case 0: return unpack_pair<4, 0>(w);
-      case 1: return unpack_pair<4, 1>(w);
-      case 2: return unpack_pair<4, 2>(w);
-      default: return unpack_pair<4, 3>(w);
+// Compile-time loop: f(std::integral_constant<int, i>) for i = 0 .. N-1.
+template <class F, int... I>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// N consecutive 32-bit words from shared memory with the widest aligned loads.
+template <int N>
+__device__ __forceinline__ void lds_words(const uint32_t* p, uint32_t (&w)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+      w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+    }
+  } else if constexpr (N % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p + i);
+      w[i] = v.x; w[i + 1] = v.y;
     }
   } else {
-    switch (f) {
-      case 0: return unpack_pair<2, 0>(w);
-      case 1: return unpack_pair<2, 1>(w);
-      case 2: return unpack_pair<2, 2>(w);
-      case 3: return unpack_pair<2, 3>(w);
-      case 4: return unpack_pair<2, 4>(w);
-      case 5: return unpack_pair<2, 5>(w);
-      case 6: return unpack_pair<2, 6>(w);
-      default: return unpack_pair<2, 7>(w);
-    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) w[i] = p[i];
   }
+}
+
+// 16-byte asynchronous global -> shared copy; src_bytes < 16 zero-fills the
+// rest (0 reads nothing).  dst, src 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ float load_as_float(const void* base, int64_t idx, int dtype) {
