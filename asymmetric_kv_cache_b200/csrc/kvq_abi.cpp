@@ -296,6 +296,64 @@ kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* 
   return ok();
 }
 
+kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* out,
+                              int32_t n_seq, void* stream) {
+  if (!cache) return fail(KVQ_ERR_NULL, "cache is NULL");
+  if (!q || !out) return fail(KVQ_ERR_NULL, "q or out is NULL");
+  if (n_seq < 1) return fail(KVQ_ERR_ARG, "n_seq %d < 1", n_seq);
+  if (n_seq > cache->cfg.max_seqs)
+    return fail(KVQ_ERR_CAPACITY, "n_seq %d > max_seqs %d", n_seq, cache->cfg.max_seqs);
+  if (n_seq > kvq::kMaxSeqsDecode)
+    return fail(KVQ_ERR_CAPACITY, "n_seq %d > %d sequences per decode call", n_seq,
+                kvq::kMaxSeqsDecode);
+  kvq_status s = dtype_ok(q_dtype);
+  if (s != KVQ_OK) return s;
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_ERR_ALIGN, "q and out must be 16-byte aligned");
+  const kvq::Geom& g = cache->geom;
+  int64_t slots = 0;
+  for (int b = 0; b < n_seq; ++b) {
+    const int L = cache->lens[b];
+    if (L <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
+    slots += (int64_t)g.hkv * g.slices * (L / g.G + (L % g.G ? 1 : 0));
+  }
+  // The fixed scratch holds [error word | tickets | two partial slots per
+  // CTA]; the CTA count is lowered until the partials fit.
+  kvq::WsLayout w = cache->ws;
+  const int64_t slot_bytes = 2LL * w.slot_floats * 4;
+  const int64_t room = kvq::kNoAllocScratchBytes - w.partials_off;
+  if (room < slot_bytes)
+    return fail(KVQ_ERR_CAPACITY,
+                "kvq_decode_noalloc: %d (sequence, kv head, head slice) units need more than the "
+                "%lld-byte fixed scratch; use kvq_decode with a workspace",
+                w.units, (long long)kvq::kNoAllocScratchBytes);
+  if (cache->max_ctas == 0) {
+    cudaError_t e = kvq::decode_max_ctas(g, &cache->max_ctas);
+    if (e != cudaSuccess) return cuda_fail(e, "decode occupancy query");
+  }
+  int64_t grid = std::min<int64_t>(slots, cache->max_ctas);
+  grid = std::min<int64_t>(grid, room / slot_bytes);
+  void* scratch = nullptr;
+  cudaError_t e = kvq::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed decode scratch");
+  // the error word and the tickets must start at zero; the array keeps
+  // whatever the previous call left
+  e = cudaMemsetAsync(scratch, 0, (size_t)w.partials_off, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed decode scratch");
+  w.total = w.partials_off + grid * slot_bytes;
+  kvq::DecodeArgs a;
+  a.cache = cache->buf;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.out = out;
+  a.ws = static_cast<unsigned char*>(scratch);
+  a.n_seq = n_seq;
+  e = kvq::launch_decode(g, w, a, (int)grid, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+size_t kvq_noalloc_scratch_bytes(void) { return (size_t)kvq::kNoAllocScratchBytes; }
+
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace) return fail(KVQ_ERR_NULL, "workspace is NULL");
   cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, (cudaStream_t)stream);

@@ -646,4 +646,40 @@ cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a,
 
 #undef KVQ_DECODE_DISPATCH
 
+// ---------------------------------------------------------------------------
+// Decode without a caller workspace.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// code running while a CUDA graph is being captured (an allocation there
+// breaks or pollutes the capture), plugins whose host framework owns every
+// device allocation and offers no workspace hook, and deployments that forbid
+// allocation after start-up.  For them the scratch the decode kernel needs
+// (error word, per-unit tickets, split partials) lives in this fixed
+// file-scope device array instead of a caller buffer.  Every GPU that loads
+// the library holds it until the process exits.  All such calls share it:
+// calls that overlap on the GPU race on it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};   // device address of the array, per device
+}  // namespace
+
+// Set-up, once per device, with that device current: the address the
+// kernels must be given (the array's name is only a host-side stand-in).
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace kvq

@@ -117,4 +117,9 @@ cudaError_t decode_max_ctas(const Geom& g, int* max_ctas);
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
                           cudaStream_t stream);
 
+// Size of the fixed device scratch used by kvq_decode_noalloc, and the device
+// address of that array on the current device (looked up on first use).
+constexpr int64_t kNoAllocScratchBytes = 8LL << 20;
+cudaError_t noalloc_scratch(void** ptr);
+
 }  // namespace kvq

@@ -74,11 +74,14 @@ kvq_cache_config = _sig("kvq_cache_config", [_vp, _P(KvqConfig)])
 kvq_cache_layout = _sig("kvq_cache_layout", [_vp, _P(KvqLayout)])
 kvq_get_lengths = _sig("kvq_get_lengths", [_vp, _P(ctypes.c_int32), ctypes.c_int32])
 kvq_sync_lengths = _sig("kvq_sync_lengths", [_vp, _vp])
+kvq_decode_noalloc = _sig("kvq_decode_noalloc", [_vp, _vp, ctypes.c_int32, _vp, ctypes.c_int32, _vp])
+kvq_noalloc_scratch_bytes = _sig("kvq_noalloc_scratch_bytes", [], ctypes.c_size_t)
 
 EXPORTED = ["kvq_status_string", "kvq_last_error", "kvq_layout_for", "kvq_cache_required_bytes",
             "kvq_cache_create", "kvq_cache_destroy", "kvq_reset", "kvq_append", "kvq_decode",
             "kvq_workspace_init", "kvq_workspace_status", "kvq_cache_config",
-            "kvq_cache_layout", "kvq_get_lengths", "kvq_sync_lengths"]
+            "kvq_cache_layout", "kvq_get_lengths", "kvq_sync_lengths", "kvq_decode_noalloc",
+            "kvq_noalloc_scratch_bytes"]
 
 
 class KvqError(RuntimeError):
@@ -217,6 +220,20 @@ class KVQCache:
         check(kvq_decode(self._h, _dev_ptr(q, "q"), DTYPE_CODES[q.dtype], _dev_ptr(out, "out"),
                          n_seq, self.workspace.data_ptr(), self.workspace.numel(),
                          _stream(stream)), "kvq_decode")
+        return out
+
+    def decode_noalloc(self, q: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        """kvq_decode_noalloc: decode into a caller-given ``out`` using the
+        library's fixed device scratch (no allocation, no workspace)."""
+        if q.dtype not in DTYPE_CODES:
+            raise ValueError("q must be fp16, bf16 or fp32")
+        if q.dim() != 3 or tuple(q.shape[1:]) != (self.spec.n_q_heads, self.spec.head_dim):
+            raise ValueError(f"q must be [n_seq, {self.spec.n_q_heads}, {self.spec.head_dim}]")
+        if out.dtype != torch.float16 or out.shape != q.shape:
+            raise ValueError("out must be an fp16 tensor shaped like q")
+        check(kvq_decode_noalloc(self._h, _dev_ptr(q, "q"), DTYPE_CODES[q.dtype],
+                                 _dev_ptr(out, "out"), q.shape[0], _stream(stream)),
+              "kvq_decode_noalloc")
         return out
 
     def workspace_status(self, stream=None) -> int:

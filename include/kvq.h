@@ -203,6 +203,35 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kv
 KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* out,
                       int32_t n_seq, void* workspace, size_t ws_bytes, void* stream);
 
+/* kvq_decode for callers that cannot allocate device memory when they
+ * decode: code running while a CUDA graph is being captured (an allocation
+ * there is not allowed in the capture), plugins whose host framework owns
+ * every device allocation and has no workspace hook, and deployments that
+ * forbid allocation after start-up.  The pages have no counterpart of this
+ * call: it only changes where the decode scratch lives.
+ * Instead of a caller workspace, the scratch (error word, per-unit tickets,
+ * split partials) is a fixed 8 MiB device array inside the library
+ * (kvq_noalloc_scratch_bytes()); every GPU that loads the library holds it
+ * until exit.  The call allocates nothing: it clears the error word and
+ * tickets with cudaMemsetAsync, lowers the number of CTAs until the
+ * partials fit, and launches the same decode kernel.  All calls share the
+ * array, which keeps the last call's contents, so calls that overlap on the
+ * GPU (other streams, other threads) race: serialize them.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  Arguments and errors as
+ * kvq_decode; KVQ_ERR_CAPACITY if the cache has so many (sequence, kv head,
+ * head slice) units that even one CTA's partials do not fit.  A failed
+ * internal wait (never expected) is recorded only in the array's error
+ * word, which the next call clears; use kvq_decode with a workspace where
+ * that report matters.  Bit-for-bit
+ * results may differ from kvq_decode's when the CTA count differs (split
+ * order); both are within the same tolerance of exact attention. */
+KVQ_API kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype,
+                                      void* out, int32_t n_seq, void* stream);
+
+/* Size in bytes of the fixed scratch array used by kvq_decode_noalloc. */
+KVQ_API size_t kvq_noalloc_scratch_bytes(void);
+
 /* Zero-fill a decode workspace on stream (cudaMemsetAsync). */
 KVQ_API kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
