@@ -316,8 +316,8 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
     if (L <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
     slots += (int64_t)g.hkv * g.slices * (L / g.G + (L % g.G ? 1 : 0));
   }
-  // The fixed scratch holds [error word | tickets | two partial slots per
-  // CTA]; the CTA count is lowered until the partials fit.
+  // The fixed scratch holds [error word | per-unit split records | two
+  // partial slots per CTA]; the CTA count is lowered until the partials fit.
   kvq::WsLayout w = cache->ws;
   const int64_t slot_bytes = 2LL * w.slot_floats * 4;
   const int64_t room = kvq::kNoAllocScratchBytes - w.partials_off;
@@ -335,8 +335,8 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
   void* scratch = nullptr;
   cudaError_t e = kvq::noalloc_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed decode scratch");
-  // the error word and the tickets must start at zero; the array keeps
-  // whatever the previous call left
+  // the error word must start at zero; the array keeps whatever the previous
+  // call left (the split records are rewritten by every call)
   e = cudaMemsetAsync(scratch, 0, (size_t)w.partials_off, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed decode scratch");
   w.total = w.partials_off + grid * slot_bytes;

@@ -50,13 +50,53 @@ struct AppCfg {
   static constexpr int SM_TOTAL = SM_VZ + 2 * G * J;
 };
 
-// Element (input row r, kv head h, channel c) of a [rows, hkv, d] input,
-// rounded to fp16 (round to nearest even).
-__device__ __forceinline__ __half input_fp16(const void* base, int64_t idx, int dtype) {
-  if (dtype == KVQ_FP16) return reinterpret_cast<const __half*>(base)[idx];
-  if (dtype == KVQ_BF16)
-    return __float2half_rn(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]));
-  return __float2half_rn(reinterpret_cast<const float*>(base)[idx]);
+// Eight consecutive input elements (16-byte aligned) rounded to fp16
+// (nearest even), packed in a uint4.
+__device__ __forceinline__ uint4 load8_fp16(const void* base, int64_t idx, int dtype) {
+  if (dtype == KVQ_FP16) return *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(base) + idx);
+  uint32_t h[4];
+  if (dtype == KVQ_BF16) {
+    const uint4 r = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      const __half2 hh = __floats2half2_rn(f.x, f.y);
+      h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+    const __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
+    const __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
+    h[0] = *reinterpret_cast<const uint32_t*>(&h0);
+    h[1] = *reinterpret_cast<const uint32_t*>(&h1);
+    h[2] = *reinterpret_cast<const uint32_t*>(&h2);
+    h[3] = *reinterpret_cast<const uint32_t*>(&h3);
+  }
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// Channels 8cc .. 8cc+7 of tail token u from the value tail, whose token
+// pairs are interleaved ([u/2][c][u%2]).
+__device__ __forceinline__ uint4 tail_v8(const __half* tailv, int u, int cc, int D) {
+  const uint4* src = reinterpret_cast<const uint4*>(tailv + ((u >> 1) * D + 8 * cc) * 2);
+  const uint4 a = src[0], b = src[1];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)   // halves (2i, u&1) and (2i+1, u&1)
+    o[i] = (u & 1) ? __byte_perm(w[2 * i], w[2 * i + 1], 0x7632) : __byte_perm(w[2 * i], w[2 * i + 1], 0x5410);
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Write eight fp16 values (one 16-byte chunk of token t) into the tails.
+__device__ __forceinline__ void store_tail8(__half* tailk, __half* tailv, int t, int cc, int D,
+                                            uint4 k8, uint4 v8) {
+  *reinterpret_cast<uint4*>(tailk + t * D + 8 * cc) = k8;
+  const __half* hv = reinterpret_cast<const __half*>(&v8);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tailv[((t >> 1) * D + 8 * cc + i) * 2 + (t & 1)] = hv[i];
 }
 
 // Quantize one value: clamp(rne((x - z) / s), 0, Q) in fp32 with the stored
@@ -117,13 +157,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   // the last CTA of this sequence to finish publishes the new length
   auto finish = [&]() {
     __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      if (atomicAdd(tickets + seq, 1) == seq_ctas - 1) {
-        if (fits) lens[seq] = len0 + nn;
-        tickets[seq] = 0;
-        __threadfence();
-      }
+    if (tid == 0 && atomic_add_acq_rel_gpu(tickets + seq, 1) == seq_ctas - 1) {
+      if (fits) lens[seq] = len0 + nn;
+      tickets[seq] = 0;
     }
   };
   if (!fits) {
@@ -131,12 +167,13 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     return;
   }
 
+  constexpr int CPR = D / 8;   // 16-byte fp16 chunks per token row
   if (F == 0) {
     // no group completes: new tokens go to tail slots T0 .. T0 + nn - 1
-    for (int idx = tid; idx < nn * D; idx += blockDim.x) {
-      const int j = idx / D, c = idx % D, t = T0 + j;
-      tailk[t * D + c] = input_fp16(kin, in_idx(j, c), dtype);
-      tailv[((t >> 1) * D + c) * 2 + (t & 1)] = input_fp16(vin, in_idx(j, c), dtype);
+    for (int ci = tid; ci < nn * CPR; ci += blockDim.x) {
+      const int j = ci / CPR, cc = ci % CPR;
+      store_tail8(tailk, tailv, T0 + j, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
+                  load8_fp16(vin, in_idx(j, 8 * cc), dtype));
     }
     finish();
     return;
@@ -146,20 +183,29 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     return;
   }
 
-  // ---- load the group: virtual token u = tau*G + r of [old tail ++ input]
-  for (int idx = tid; idx < G * D; idx += blockDim.x) {
-    const int r = idx / D, c = idx % D;
-    const int u = tau * G + r;
-    __half xk, xv;
-    if (u < T0) {
-      xk = tailk[u * D + c];
-      xv = tailv[((u >> 1) * D + c) * 2 + (u & 1)];
-    } else {
-      xk = input_fp16(kin, in_idx(u - T0, c), dtype);
-      xv = input_fp16(vin, in_idx(u - T0, c), dtype);
+  // ---- load the group: virtual token u = tau*G + r of [old tail ++ input],
+  // 16-byte chunks, every load of a thread issued before its stores
+  {
+    constexpr int NCH = G * CPR / 128;   // chunks per thread (K and V each)
+    uint4 kx[NCH], vx[NCH];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int ci = tid + 128 * j, r = ci / CPR, cc = ci % CPR;
+      const int u = tau * G + r;
+      if (u < T0) {
+        kx[j] = *reinterpret_cast<const uint4*>(tailk + u * D + 8 * cc);
+        vx[j] = tail_v8(tailv, u, cc, D);
+      } else {
+        kx[j] = load8_fp16(kin, in_idx(u - T0, 8 * cc), dtype);
+        vx[j] = load8_fp16(vin, in_idx(u - T0, 8 * cc), dtype);
+      }
     }
-    sk[idx] = xk;
-    sv[idx] = xv;
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int ci = tid + 128 * j;
+      reinterpret_cast<uint4*>(sk)[ci] = kx[j];
+      reinterpret_cast<uint4*>(sv)[ci] = vx[j];
+    }
   }
   __syncthreads();
 
@@ -266,11 +312,11 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   if (tau == 0) {
     // the new tail: virtual tokens F*G .. F*G + T1 - 1, all from the input
     // (the old tail was fully read above, before the barrier)
-    for (int idx = tid; idx < T1 * D; idx += blockDim.x) {
-      const int t = idx / D, c = idx % D;
+    for (int ci = tid; ci < T1 * CPR; ci += blockDim.x) {
+      const int t = ci / CPR, cc = ci % CPR;
       const int64_t r = (int64_t)F * G + t - T0;
-      tailk[t * D + c] = input_fp16(kin, in_idx(r, c), dtype);
-      tailv[((t >> 1) * D + c) * 2 + (t & 1)] = input_fp16(vin, in_idx(r, c), dtype);
+      store_tail8(tailk, tailv, t, cc, D, load8_fp16(kin, in_idx(r, 8 * cc), dtype),
+                  load8_fp16(vin, in_idx(r, 8 * cc), dtype));
     }
   }
   finish();

@@ -24,15 +24,16 @@
 //   * folds the per-channel key scales into the query: q'_c = q_c s_c, so
 //     q . k_hat = sum_c q'_c code_c + sum_c q_c z_c; the second sum (one per
 //     group and head) runs on the tensor core with q split into fp16 high and
-//     low halves (rows 8-15 of the tile) against the key mins;
-//   * unpacks key codes to exact fp16 pairs and runs S = q' K^T on m16n8k16
-//     tiles (rows = query heads, columns = tokens);
-//   * updates the running max / rescales, exponentiates (exp2 domain);
+//     low halves (rows 0-7 and 8-15 of the tile) against the key mins;
+//   * unpacks key codes to exact fp16 pairs and runs S^T = codes q'^T on
+//     m16n8k16 tiles (rows = 16 tokens, columns = the 8 query heads of the
+//     GQA group), so each lane's softmax state covers two heads;
+//   * updates the running max / rescales, exponentiates (exp2 domain) and
+//     transposes the fp16 P tile in registers (movmatrix);
 //   * runs O^T += V_code^T (p s_v) on tiles whose rows are channels and whose
-//     columns are heads (the P fragment of S is already the B fragment), with
-//     the per-token value scale folded into p for each channel group, and
-//     sum_t p_t z_t (value mins) and sum_t p_t (the softmax denominator) on
-//     one more tile.
+//     columns are heads, with the per-token value scale folded into p for
+//     each channel group, and sum_t p_t z_t (value mins) and sum_t p_t (the
+//     softmax denominator) on one more tile.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -66,31 +67,42 @@ struct DecCfg {
   static constexpr int SEC_VSCALE = SEC_VCODES + G * D * VB / 8;
   static constexpr int SEC_VMIN = SEC_VSCALE + 2 * G * J;
   static constexpr int BLK = SEC_VMIN + 2 * G * J;
-  static constexpr int NST = (BLK <= 4096) ? 4 : 2;   // ring stages per warp
+  static constexpr int NST = (BLK <= 4096) ? 3 : 2;   // ring stages per warp
+  // resident CTAs per SM the register budget aims at (shared memory allows
+  // four CTAs with 3-stage rings of blocks up to 4 KB, three otherwise)
+  static constexpr int MIN_BLOCKS = (BLK <= 4096) ? 4 : 3;
   static constexpr int RING = kWarps * NST * BLK;
+  // query fragments of the current unit, shared by the CTA's warps:
+  // [kt][lane][4 words] = {hi v0, lo v0, hi v1, lo v1}
+  static constexpr int QA_OFF = RING;
+  static constexpr int QA_BYTES = KT * 32 * 16;
+  // both parts divided by the key code multiplier m of their register,
+  // [kt][lane][4 words] (the B operand of q.k is (q_hi/m + q_lo/m) * s_k)
+  static constexpr int QM_OFF = QA_OFF + QA_BYTES;
+  static constexpr int QM_BYTES = KT * 32 * 16;
   static constexpr int MERGE_FLOATS = kWarps * kHeadsPerSlice * (D + 2);
   static_assert(MERGE_FLOATS * 4 <= RING, "merge area must fit in the ring");
-  static constexpr int SMEM_FIXED = RING + kWarps * NST * 8 + 64;
-};
-
-struct SharedCtl {
-  int last;   // this CTA completes the current unit
+  static constexpr int BAR_OFF = QM_OFF + QM_BYTES;
+  static constexpr int SMEM_FIXED = BAR_OFF + kWarps * NST * 8 + 64;
 };
 
 template <int D, int KB, int VB, int G>
 struct WarpState {
-  float o[D / 16][4];   // O^T: rows channels, cols heads (unnormalized)
-  float z[4];           // rows: value-min terms (j < J) and sum p (row J)
-  float m;              // running max of head (lane / 4), log2 domain
+  float o[D / 16][4];   // O^T: (channel 16mt + g, heads 2i, 2i+1), then channel + 8
+  float z[4];           // rows: value-min terms (j < J) and sum p (row J); cols heads
+  float m[2];           // running max of heads 2i, 2i+1 (i = lane & 3), log2 domain
 };
 
-// Load this lane's query fragments (or zeros for a padding head): rows g of
-// the A tile, channels 16kt + 2i + {0,1} and + 8 + {0,1}; q is scaled by
-// log2(e)/sqrt(d) and split into fp16 high and low parts.
-template <int D>
+// Query fragments of head g = lane/4 (zeros for a padding head), channels
+// 16kt + 2i + {0,1} (v = 0) and + 8 (v = 1), i = lane & 3: q is scaled by
+// log2(e)/sqrt(d), split into fp16 high and low parts and stored per lane
+// as qs[kt * 32 + lane] = {hi v0, lo v0, hi v1, lo v1} - the A quad of the
+// key-min tile (rows g: high part, rows g + 8: low part).
+template <int D, int KB>
 __device__ __forceinline__ void load_query(const void* q, int dtype, int64_t row, bool valid,
-                                           int i4, uint32_t (&qh)[D / 16][2],
-                                           uint32_t (&ql)[D / 16][2]) {
+                                           int lane, uint4* __restrict__ qs,
+                                           uint4* __restrict__ qm) {
+  const int i4 = lane & 3;
   const float sc = kLog2e * rsqrtf((float)D);
   float2 x[D / 16][2];
 #pragma unroll
@@ -112,127 +124,170 @@ __device__ __forceinline__ void load_query(const void* q, int dtype, int64_t row
       x[kt][v] = f;
     }
   }
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
+  static_for<D / 16>([&](auto kt_) {
+    constexpr int kt = decltype(kt_)::value;
+    uint32_t w[4];
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
       const float x0 = x[kt][v].x * sc, x1 = x[kt][v].y * sc;
       const __half2 h = __floats2half2_rn(x0, x1);
       const float2 hf = __half22float2(h);
-      qh[kt][v] = h2_as_u32(h);
-      ql[kt][v] = pack_h2(x0 - hf.x, x1 - hf.y);
+      w[2 * v] = h2_as_u32(h);
+      w[2 * v + 1] = pack_h2(x0 - hf.x, x1 - hf.y);
     }
-  }
+    qs[kt * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
+    constexpr int FK = 16 / KB;
+    constexpr int e0 = code_log2_mul<KB, (2 * kt) % FK>();
+    constexpr int e1 = code_log2_mul<KB, (2 * kt + 1) % FK>();
+    qm[kt * 32 + lane] = make_uint4(hmul2_b(w[0], h2_pow2_neg(e0)), hmul2_b(w[1], h2_pow2_neg(e0)),
+                                    hmul2_b(w[2], h2_pow2_neg(e1)), hmul2_b(w[3], h2_pow2_neg(e1)));
+  });
 }
 
-// Online-softmax update of a warp for new logits s[n][0..1] (head = lane/4,
-// tokens in the C layout) and conversion to fp16 probabilities p[n].
-template <int D, int N, int KB, int VB, int G>
-__device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, float (&s)[N][2],
-                                               uint32_t (&p)[N], int lane) {
-  float mx = -INFINITY;
+// Online-softmax update for new logits in the transposed tile layout:
+// s[mt] = {(token g, head 2i), (token g, head 2i+1), (token g+8, head 2i),
+// (token g+8, head 2i+1)} of a 16-token tile mt (g = lane/4, i = lane&3).
+// Produces the fp16 probabilities as B fragments of the p.v tile
+// (pt[mt] = {tokens 0-7, tokens 8-15} of head g, 2 tokens per lane).
+template <int D, int NM, int KB, int VB, int G>
+__device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, float (&s)[NM][4],
+                                               uint32_t (&pt)[NM][2]) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int n = 0; n < N; ++n) mx = fmaxf(mx, fmaxf(s[n][0], s[n][1]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const float mnew = fmaxf(st.m, mx);
-  if (__any_sync(0xffffffffu, mnew > st.m)) {
-    const float alpha = fast_exp2(st.m - mnew);   // 0 when st.m = -inf
-    const int i4 = lane & 3;
-    const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * i4);
-    const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * i4 + 4);
-#pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      st.o[mt][0] *= a0;
-      st.o[mt][1] *= a1;
-      st.o[mt][2] *= a0;
-      st.o[mt][3] *= a1;
-    }
-    st.z[0] *= a0;
-    st.z[1] *= a1;
-    st.z[2] *= a0;
-    st.z[3] *= a1;
-    st.m = mnew;
+  for (int mt = 0; mt < NM; ++mt) {
+    mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+    mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
   }
 #pragma unroll
-  for (int n = 0; n < N; ++n)
-    p[n] = pack_h2(fast_exp2(s[n][0] - st.m), fast_exp2(s[n][1] - st.m));
+  for (int o = 4; o <= 16; o <<= 1) {   // across the 8 token rows (lane bits 2-4)
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float n0 = fmaxf(st.m[0], mx0), n1 = fmaxf(st.m[1], mx1);
+  if (__any_sync(0xffffffffu, n0 > st.m[0] || n1 > st.m[1])) {
+    if (st.m[0] != -INFINITY) {   // accumulators hold data: rescale them
+      const float a0 = fast_exp2(st.m[0] - n0), a1 = fast_exp2(st.m[1] - n1);
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        st.o[mt][0] *= a0;
+        st.o[mt][1] *= a1;
+        st.o[mt][2] *= a0;
+        st.o[mt][3] *= a1;
+      }
+      st.z[0] *= a0;
+      st.z[1] *= a1;
+      st.z[2] *= a0;
+      st.z[3] *= a1;
+    }
+    st.m[0] = n0;
+    st.m[1] = n1;
+  }
+#pragma unroll
+  for (int mt = 0; mt < NM; ++mt) {
+    pt[mt][0] = movmatrix_trans(
+        pack_h2(fast_exp2(s[mt][0] - st.m[0]), fast_exp2(s[mt][1] - st.m[1])));
+    pt[mt][1] = movmatrix_trans(
+        pack_h2(fast_exp2(s[mt][2] - st.m[0]), fast_exp2(s[mt][3] - st.m[1])));
+  }
 }
 
 // One quantized group from the shared-memory stage `sp`.
+//
+// Key codes enter the tensor core as x = 1024 + m*code (code_offset) against
+// B = (q/m) * s_k, carried as an fp16 high + low pair (one fp16 rounding of
+// the product would cost ~2^-12 of each logit term, which matters for
+// channels with large scales); the offset is removed with tiles against a
+// constant 1024 operand, which sum exactly the fp16 B values the tensor core
+// saw.  Value
+// codes are unpacked to exact fp16 integers (unpack_pair).
 template <int D, int KB, int VB, int G>
 __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
                                               const unsigned char* __restrict__ sp,
-                                              const uint32_t (&qh)[D / 16][2],
-                                              const uint32_t (&ql)[D / 16][2], int lane) {
+                                              const uint4* __restrict__ qsm,
+                                              const uint4* __restrict__ qmsm, int lane) {
   using C = DecCfg<D, KB, VB, G>;
+  constexpr int NM = G / 16;
   const int g8 = lane >> 2, i4 = lane & 3;
 
-  // q' = q * s_key (fp16, one rounding) and the min term sum_c q_c z_c
-  uint32_t qs[C::KT][2];
+  // B = (q s_k) / m as an fp16 high + low pair, the key-min term and the
+  // offset correction
+  uint32_t qs[C::KT][2], ql[C::KT][2];
   float bias[4] = {0.f, 0.f, 0.f, 0.f};
+  float kcor[4] = {0.f, 0.f, 0.f, 0.f};
   {
     uint32_t ksw[D / 8], kzw[D / 8];
     lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8), ksw);
     lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8), kzw);
-#pragma unroll
-    for (int kt = 0; kt < C::KT; ++kt) {
+    static_for<C::KT>([&](auto kt_) {
+      constexpr int kt = decltype(kt_)::value;
+      const uint4 q4 = qsm[kt * 32 + lane];
+      const uint4 qm = qmsm[kt * 32 + lane];
+      // high part: one rounding of hi*s + lo*s; low part: the rest of it,
+      // (hi*s - high) exact in one fused step, plus lo*s
       const uint32_t s0 = ksw[2 * kt], s1 = ksw[2 * kt + 1];
-      qs[kt][0] = h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s0),
-                                    __hmul2(u32_as_h2(ql[kt][0]), u32_as_h2(s0))));
-      qs[kt][1] = h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s1),
-                                    __hmul2(u32_as_h2(ql[kt][1]), u32_as_h2(s1))));
-      mma16816(bias, qh[kt][0], ql[kt][0], qh[kt][1], ql[kt][1], kzw[2 * kt], kzw[2 * kt + 1]);
-    }
+      qs[kt][0] = hfma2_b(qm.x, s0, hmul2_b(qm.y, s0));
+      qs[kt][1] = hfma2_b(qm.z, s1, hmul2_b(qm.w, s1));
+      ql[kt][0] = hfma2_b(qm.y, s0, hfma2_b(qm.x, s0, qs[kt][0] ^ 0x80008000u));
+      ql[kt][1] = hfma2_b(qm.w, s1, hfma2_b(qm.z, s1, qs[kt][1] ^ 0x80008000u));
+      mma16816(bias, q4.x, q4.y, q4.z, q4.w, kzw[2 * kt], kzw[2 * kt + 1]);
+      mma16816(kcor, kH2One024, kH2One024, kH2One024, kH2One024, qs[kt][0], qs[kt][1]);
+      mma16816(kcor, kH2One024, kH2One024, kH2One024, kH2One024, ql[kt][0], ql[kt][1]);
+    });
   }
-  const float b = bias[0] + bias[2];   // head g8: high-part rows + low-part rows
+  // bias of head g8 is in every lane of quad g8; fetch heads 2*i4 and 2*i4+1
+  const float bg = bias[0] + bias[2];
+  const float b0 = __shfl_sync(0xffffffffu, bg, 8 * i4) - kcor[0];
+  const float b1 = __shfl_sync(0xffffffffu, bg, 8 * i4 + 4) - kcor[1];
 
-  // S = q' K^T over the G tokens
-  float s[C::NT][2];
+  // S^T = codes q'^T: rows = tokens (two 8-token code tiles), cols = heads
+  float s[NM][4];
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
-  static_for<C::NT>([&](auto nt_) {
-    constexpr int nt = decltype(nt_)::value;
-    uint32_t kw[C::LWK];
-    lds_words<C::LWK>(kcw + (nt * 32 + lane) * C::LWK, kw);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  static_for<NM>([&](auto mt_) {
+    constexpr int mt = decltype(mt_)::value;
+    uint32_t kw0[C::LWK], kw1[C::LWK];
+    lds_words<C::LWK>(kcw + ((2 * mt) * 32 + lane) * C::LWK, kw0);
+    lds_words<C::LWK>(kcw + ((2 * mt + 1) * 32 + lane) * C::LWK, kw1);
+    float acc[4] = {b0, b1, b0, b1};
     static_for<C::KT>([&](auto kt_) {
       constexpr int kt = decltype(kt_)::value;
       constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
-      const uint32_t b0 = unpack_pair<KB, p0 % C::FK>(kw[p0 / C::FK]);
-      const uint32_t b1 = unpack_pair<KB, p1 % C::FK>(kw[p1 / C::FK]);
-      mma16816(acc, qs[kt][0], 0u, qs[kt][1], 0u, b0, b1);
+      const uint32_t a0 = code_offset<KB, p0 % C::FK>(kw0[p0 / C::FK]);   // token g
+      const uint32_t a1 = code_offset<KB, p0 % C::FK>(kw1[p0 / C::FK]);   // token g + 8
+      const uint32_t a2 = code_offset<KB, p1 % C::FK>(kw0[p1 / C::FK]);   // channels + 8
+      const uint32_t a3 = code_offset<KB, p1 % C::FK>(kw1[p1 / C::FK]);
+      mma16816(acc, a0, a1, a2, a3, qs[kt][0], qs[kt][1]);
+      mma16816(acc, a0, a1, a2, a3, ql[kt][0], ql[kt][1]);
     });
-    s[nt][0] = acc[0] + b;
-    s[nt][1] = acc[1] + b;
+    s[mt][0] = acc[0];
+    s[mt][1] = acc[1];
+    s[mt][2] = acc[2];
+    s[mt][3] = acc[3];
   });
 
-  uint32_t p[C::NT];
-  softmax_update<D, C::NT, KB, VB, G>(st, s, p, lane);
+  uint32_t pt[NM][2];
+  softmax_update<D, NM, KB, VB, G>(st, s, pt);
 
   // O^T += V^T (p * s_v); Z += [z_v; 1]^T p
   const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
   const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
   const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
+  // rows of the Z tile: row g8 < J takes its group's value mins, row J is (1, 1)
+  const int zrow = g8 < C::J ? g8 : 0;
+  const uint32_t zsel = g8 < C::J ? 0xFFFFFFFFu : 0u;
+  const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
   static_for<C::KV>([&](auto kv_) {
     constexpr int kv = decltype(kv_)::value;
-    const uint32_t bp0 = p[2 * kv], bp1 = p[2 * kv + 1];
-    uint32_t za0 = 0u, za2 = 0u;
-    if (g8 < C::J) {
-      const uint32_t* zz = vzw + ((4 * kv + i4) * C::J + g8) * 2;
-      za0 = zz[0];
-      za2 = zz[1];
-    } else if (g8 == C::J) {
-      za0 = za2 = 0x3C003C00u;   // fp16 pair (1, 1)
-    }
-    mma16816(st.z, za0, 0u, za2, 0u, bp0, bp1);
+    const uint32_t bp0 = pt[kv][0], bp1 = pt[kv][1];
+    const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
+    mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
 
     uint32_t sw[2 * C::J];
     lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
     uint32_t bs[C::J][2];
 #pragma unroll
     for (int j = 0; j < C::J; ++j) {
-      bs[j][0] = h2_as_u32(__hmul2(u32_as_h2(bp0), u32_as_h2(sw[2 * j])));
-      bs[j][1] = h2_as_u32(__hmul2(u32_as_h2(bp1), u32_as_h2(sw[2 * j + 1])));
+      bs[j][0] = hmul2_b(bp0, sw[2 * j]);
+      bs[j][1] = hmul2_b(bp1, sw[2 * j + 1]);
     }
     uint32_t vw[C::LWV];
     lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
@@ -266,8 +321,7 @@ template <int D, int KB, int VB, int G>
 __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
                                              const __half* __restrict__ tk,
                                              const __half* __restrict__ tv, int T,
-                                             const uint32_t (&qh)[D / 16][2],
-                                             const uint32_t (&ql)[D / 16][2], int lane,
+                                             const uint4* __restrict__ qsm, int lane,
                                              unsigned char* __restrict__ buf) {
   using C = DecCfg<D, KB, VB, G>;
   using TS = TailStage<D>;
@@ -288,25 +342,30 @@ __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
     cp_async_wait_all();
     __syncwarp();
 
-    float s[2][2];
+    // S^T = K q^T with q = high + low parts (two products per tile)
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
+    const unsigned char* k1 = k0 + 8 * TS::KROW;
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const unsigned char* krow = buf + (8 * n + g8) * TS::KROW + 4 * i4;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kt = 0; kt < C::KT; ++kt) {
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(krow + 32 * kt);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(krow + 32 * kt + 16);
-        mma16816(acc, qh[kt][0], ql[kt][0], qh[kt][1], ql[kt][1], b0, b1);
-      }
-      const int t0 = 16 * kv + 8 * n + 2 * i4;      // tokens of this lane's C columns
-      s[n][0] = (t0 < T) ? acc[0] + acc[2] : -INFINITY;
-      s[n][1] = (t0 + 1 < T) ? acc[1] + acc[3] : -INFINITY;
+    for (int kt = 0; kt < C::KT; ++kt) {
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(k0 + 32 * kt);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(k1 + 32 * kt);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16);
+      const uint4 q4 = qsm[kt * 32 + lane];
+      mma16816(acc, a0, a1, a2, a3, q4.x, q4.z);
+      mma16816(acc, a0, a1, a2, a3, q4.y, q4.w);
     }
-    uint32_t p[2];
-    softmax_update<D, 2, KB, VB, G>(st, s, p, lane);
+    const int t0 = 16 * kv + g8, t1 = t0 + 8;
+    float s[1][4];
+    s[0][0] = (t0 < T) ? acc[0] : -INFINITY;
+    s[0][1] = (t0 < T) ? acc[1] : -INFINITY;
+    s[0][2] = (t1 < T) ? acc[2] : -INFINITY;
+    s[0][3] = (t1 < T) ? acc[3] : -INFINITY;
+    uint32_t pt[1][2];
+    softmax_update<D, 1, KB, VB, G>(st, s, pt);
     const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
-    mma16816(st.z, ones, 0u, ones, 0u, p[0], p[1]);
+    mma16816(st.z, ones, 0u, ones, 0u, pt[0][0], pt[0][1]);
     // V^T fragments; the second token of the last pair may be stale: mask it
     const int ta = 16 * kv + 2 * i4, tb = ta + 8;
     const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
@@ -319,14 +378,14 @@ __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
       const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
       const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
       const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
-      mma16816(st.o[mt], a0, a1, a2, a3, p[0], p[1]);
+      mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
     }
     __syncwarp();   // every lane is done with this chunk before the next copy
   }
 }
 
 // Largest b in [0, n) with prefix[b] <= pos (prefix[0] = 0, increasing).
-__device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int64_t pos) {
+__device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int pos) {
   int lo = 0, hi = n;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
@@ -336,13 +395,14 @@ __device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int64_t po
 }
 
 template <int D, int KB, int VB, int G>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
   using C = DecCfg<D, KB, VB, G>;
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING);
-  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + kWarps * C::NST);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint4* qsm = reinterpret_cast<uint4*>(smem + C::QA_OFF);
+  uint4* qmsm = reinterpret_cast<uint4*>(smem + C::QM_OFF);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::SMEM_FIXED);
   float* merge = reinterpret_cast<float*>(smem);   // reuses the ring between pieces
 
@@ -352,9 +412,11 @@ __global__ void __launch_bounds__(kThreads, 3)
   const int per_seq_units = g.hkv * g.slices;
   const int32_t* lens = reinterpret_cast<const int32_t*>(a.cache + g.lens_off);
   int32_t* err = reinterpret_cast<int32_t*>(a.ws + w.err_off);
-  int32_t* tickets = reinterpret_cast<int32_t*>(a.ws + w.tickets_off);
   float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
 
+  // the combine kernel (a programmatic dependent of this grid) may be
+  // scheduled now; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) mbar_init(&bars[warp * C::NST + s], 1);
@@ -391,12 +453,11 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
   __syncthreads();
 
-  const int64_t T = prefix[n_seq];
-  const int64_t grid = gridDim.x;
-  const int64_t k = blockIdx.x;
-  const int64_t start = k * T / grid, end = (k + 1) * T / grid;
-  auto cta_of = [&](int64_t p) { return ((p + 1) * grid - 1) / T; };
-  auto cta_start = [&](int64_t kk) { return kk * T / grid; };
+  // this CTA's slot range (the only 64-bit divisions of the kernel, once)
+  const int T = prefix[n_seq];
+  const int grid = gridDim.x;
+  const int k = blockIdx.x;
+  const int start = (int)((int64_t)k * T / grid), end = (int)((int64_t)(k + 1) * T / grid);
 
   uint32_t uses = 0;        // ring stage uses of this warp so far
   bool ok = true;           // no wait has run out
@@ -404,29 +465,26 @@ __global__ void __launch_bounds__(kThreads, 3)
   uint64_t* wbars = bars + warp * C::NST;
   const unsigned char* blocks = a.cache + g.blocks_off;
 
-  for (int64_t pos = start; pos < end;) {
+  for (int pos = start; pos < end;) {
     const int b = find_seq(prefix, n_seq, pos);
     const int L = lens[b];
     const int ng = L / G, Tb = L % G;
     const int wb = ng + (Tb ? 1 : 0);
-    const int64_t local = pos - prefix[b];
-    const int uis = (int)(local / wb);
-    const int slot0 = (int)(local % wb);
-    const int slot1 = (int)(((int64_t)slot0 + (end - pos)) < wb ? ((int64_t)slot0 + (end - pos)) : wb);
+    const int local = pos - prefix[b];
+    const int uis = local / wb;
+    const int slot0 = local - uis * wb;
+    const int slot1 = min(wb, slot0 + (end - pos));
     const int kvh = uis / g.slices, slice = uis % g.slices;
     const int unit = b * per_seq_units + uis;
     const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
     const int nh = min(kHeadsPerSlice, g.gqa - slice * kHeadsPerSlice);
     const int64_t ublk = ((int64_t)b * g.hkv + kvh) * g.max_groups;
 
-    uint32_t qh[C::KT][2], ql[C::KT][2];
-    load_query<D>(a.q, a.q_dtype, (int64_t)b * g.hq + hbase + g8, g8 < nh, i4, qh, ql);
-
     WarpState<D, KB, VB, G> st;
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
-    st.m = -INFINITY;
+    st.m[0] = st.m[1] = -INFINITY;
 
     // this warp's group slots: slot0 + warp + 4k below min(slot1, ng)
     const int gend = min(slot1, ng);
@@ -442,6 +500,10 @@ __global__ void __launch_bounds__(kThreads, 3)
                       &wbars[stg]);
       }
     }
+    // while the copies fly, warp 0 prepares the unit's query fragments
+    if (warp == 0)
+      load_query<D, KB>(a.q, a.q_dtype, (int64_t)b * g.hq + hbase + g8, g8 < nh, lane, qsm, qmsm);
+    __syncthreads();
     for (int it = 0; it < count; ++it) {
       const uint32_t u = uses + it;
       const int stg = u % C::NST;
@@ -452,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 3)
         if (lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
         break;
       }
-      process_group<D, KB, VB, G>(st, wring + stg * C::BLK, qh, ql, lane);
+      process_group<D, KB, VB, G>(st, wring + stg * C::BLK, qsm, qmsm, lane);
       __syncwarp();
       if (lane == 0 && it + C::NST < count) {
         fence_proxy_async_smem();
@@ -467,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (ok && Tb > 0 && slot1 == wb && slot0 <= ng && ((ng - slot0) % kWarps) == warp) {
       const __half* tk = reinterpret_cast<const __half*>(
           a.cache + g.tails_off + ((int64_t)b * g.hkv + kvh) * g.tail_bytes);
-      process_tail<D, KB, VB, G>(st, tk, tk + G * D, Tb, qh, ql, lane, wring);
+      process_tail<D, KB, VB, G>(st, tk, tk + G * D, Tb, qsm, lane, wring);
     }
 
     // ---- merge the 4 warps (the ring is idle: every issued copy was waited on)
@@ -495,17 +557,25 @@ __global__ void __launch_bounds__(kThreads, 3)
         mo[(2 * i4 + 1) * (D + 2) + c1] = st.o[mt][3] + zl1[j];
       }
       if (g8 == 0) {
+        mo[(2 * i4) * (D + 2) + D] = st.m[0];
+        mo[(2 * i4 + 1) * (D + 2) + D] = st.m[1];
         mo[(2 * i4) * (D + 2) + D + 1] = l0;
         mo[(2 * i4 + 1) * (D + 2) + D + 1] = l1;
       }
-      if (i4 == 0) mo[g8 * (D + 2) + D] = st.m;
     }
     __syncthreads();
 
     const bool whole = (slot0 == 0 && slot1 == wb);
-    const int64_t up = prefix[b] + (int64_t)uis * wb;   // first slot of the unit
-    const int64_t kf = cta_of(up), kl = cta_of(up + wb - 1);
-    const int64_t myslot = (k == kf && cta_start(k) < up) ? 2 * k + 1 : 2 * k;
+    // Partial slots: a CTA holds at most two split pieces, its first (slot
+    // 2k) and its last (2k + 1); pieces in between are whole units.
+    const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
+    if (slot0 == 0 && tid == 0) {
+      // split record of the unit for the combine kernel: its first partial
+      // slot and the number of CTAs holding a piece of it
+      const int64_t last = (int64_t)pos + wb - 1;   // the unit's last slot
+      const int kl = (int)(((last + 1) * grid - 1) / T);
+      *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
+    }
     for (int idx = tid; idx < nh * D; idx += kThreads) {
       const int h = idx / D, c = idx % D;
       float M = -INFINITY;
@@ -531,40 +601,88 @@ __global__ void __launch_bounds__(kThreads, 3)
         }
       }
     }
-    if (!whole) {
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        const int old = atomicAdd(&tickets[unit], 1);
-        ctl->last = (old == (int)(kl - kf));
-      }
-      __syncthreads();
-      if (ctl->last) {
-        __threadfence();
-        for (int idx = tid; idx < nh * D; idx += kThreads) {
-          const int h = idx / D, c = idx % D;
-          float M = -INFINITY;
-          for (int64_t kk = kf; kk <= kl; ++kk) {
-            const int64_t sl = (kk == kf && cta_start(kk) < up) ? 2 * kk + 1 : 2 * kk;
-            M = fmaxf(M, __ldcg(partials + sl * w.slot_floats + h * (D + 2) + D));
-          }
-          float Lsum = 0.f, O = 0.f;
-          for (int64_t kk = kf; kk <= kl; ++kk) {
-            const int64_t sl = (kk == kf && cta_start(kk) < up) ? 2 * kk + 1 : 2 * kk;
-            const float* ps = partials + sl * w.slot_floats + h * (D + 2);
-            const float f = fast_exp2(__ldcg(ps + D) - M);
-            Lsum += __ldcg(ps + D + 1) * f;
-            O += __ldcg(ps + c) * f;
-          }
-          reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-              __float2half_rn(O / Lsum);
-        }
-        if (tid == 0) tickets[unit] = 0;
-      }
-    }
     fence_proxy_async_smem();   // generic accesses before the next bulk copies
     __syncthreads();            // merge area and ctl are reused by the next piece
     pos += slot1 - slot0;
+  }
+}
+
+// Merges the pieces of every unit that the decode kernel split across CTAs.
+// One block per (unit, head, 32-channel chunk); units held by one CTA were
+// written by the decode kernel itself.  Runs as a programmatic dependent
+// launch of the decode grid and waits for it before touching the partials.
+// Warp 0 turns the pieces' (max, sum) into normalized weights; each warp
+// then folds every 4th piece for the block's 32 channels (lane = channel)
+// with up to 8 loads in flight, and the warps' sums meet in shared memory.
+constexpr int kCombineChunk = 32;
+constexpr int kCombineMaxPieces = 2 * kMaxDecodeCtas;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) combine_kernel(const Geom g, const WsLayout w,
+                                                           const DecodeArgs a) {
+  __shared__ float wgt[kCombineMaxPieces];
+  __shared__ float red[kWarps][32];
+  __shared__ float sinv;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int kChunks = D / kCombineChunk;
+  const int chunk = blockIdx.x % kChunks;
+  const int h = (blockIdx.x / kChunks) % kHeadsPerSlice;
+  const int unit = blockIdx.x / (kChunks * kHeadsPerSlice);
+  const int2 rec = *reinterpret_cast<const int2*>(a.ws + w.units_off + 8LL * unit);
+  const int npc = rec.y;
+  if (npc <= 1) return;   // whole unit: already written
+  const int per_seq = g.hkv * g.slices;
+  const int b = unit / per_seq, uis = unit % per_seq;
+  const int kvh = uis / g.slices, slice = uis % g.slices;
+  const int nh = min(kHeadsPerSlice, g.gqa - slice * kHeadsPerSlice);
+  if (h >= nh) return;
+  const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t sl0 = rec.x, kf = sl0 / 2;
+  const float* partials = reinterpret_cast<const float*>(a.ws + w.partials_off) + h * (D + 2);
+  auto piece = [&](int pc) { return partials + (pc == 0 ? sl0 : 2 * (kf + pc)) * w.slot_floats; };
+
+  if (warp == 0) {
+    // weights e^(m_k - M) / L, L = sum_k l_k e^(m_k - M)
+    float M = -INFINITY;
+    for (int pc = lane; pc < npc; pc += 32) M = fmaxf(M, __ldcg(piece(pc) + D));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int pc = lane; pc < npc; pc += 32) {
+      const float* ps = piece(pc);
+      const float wk = fast_exp2(__ldcg(ps + D) - M);
+      wgt[pc] = wk;
+      L += wk * __ldcg(ps + D + 1);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) sinv = 1.0f / L;
+  }
+  __syncthreads();
+  const int c = chunk * kCombineChunk + lane;
+  float acc = 0.f;
+  for (int p0 = warp; p0 < npc; p0 += 8 * kWarps) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int pc = p0 + u * kWarps;
+      v[u] = pc < npc ? __ldcg(piece(pc) + c) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int pc = p0 + u * kWarps;
+      if (pc < npc) acc += wgt[pc] * v[u];
+    }
+  }
+  red[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float o = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) o += red[ww][lane];
+    reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
+        __float2half_rn(o * sinv);
   }
 }
 
@@ -609,7 +727,20 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
     configured = true;
   }
   kern<<<grid, kThreads, sm, stream>>>(g, w, a);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the combine kernel, a programmatic dependent of the decode grid
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)(a.n_seq * g.hkv * g.slices * kHeadsPerSlice * (D / kCombineChunk)));
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, combine_kernel<D>, g, w, a);
 }
 
 }  // namespace

@@ -88,6 +88,14 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held one row-pair per lane
+// (lane 4r + c holds row r, columns 2c and 2c+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
@@ -106,26 +114,65 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Exact fp16 pair of the code pair in field f of a packed word.
-// BITS-bit codes, F = 16/BITS pairs per 32-bit word: the low element of
-// pair f sits at bits [BITS*f, BITS*f + BITS), the high element 16 bits
-// higher.  OR-ing a field into the mantissa of 1024.0 (0x6400) gives
-// 1024 + m*code with m = 2^(BITS*(f mod 8/BITS)); one fused multiply-add
-// by 1/m and -1024/m then yields the code exactly (all values are small
-// integers times powers of two).
+
+// Ticket increment with acquire-release semantics at GPU scope: the stores
+// that precede it (the CTA's, when a CTA barrier comes first) are visible to
+// whoever reads the incremented value, and it is ordered before the caller's
+// later accesses.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// fp16x2 arithmetic on packed 32-bit registers (round to nearest even).
+__device__ __forceinline__ uint32_t hfma2_b(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hmul2_b(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Code pair of field f of a packed word as the fp16 pair (1024 + m*code_lo,
+// 1024 + m*code_hi), m = 2^(BITS * (f mod 8/BITS)) (code_mul<BITS, f>()):
+// the field OR-ed into the mantissa of 1024.0.  One LOP3 (plus a shared
+// byte shift for the upper fields); the 1024 offset and the factor m are
+// removed on the other side of the tensor-core product.
 template <int BITS, int F_IDX>
-__device__ __forceinline__ uint32_t unpack_pair(uint32_t w) {
+__device__ __forceinline__ uint32_t code_offset(uint32_t w) {
   static_assert(BITS == 2 || BITS == 4, "2- or 4-bit codes");
-  constexpr int kPerByte = 8 / BITS;               // fields per byte half-word part
+  constexpr int kPerByte = 8 / BITS;
   constexpr int kShift = (F_IDX >= kPerByte) ? 8 : 0;
   constexpr int kF = F_IDX % kPerByte;
   constexpr uint32_t kLowMask = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
-  constexpr uint32_t kMask = kLowMask << (BITS * kF);
-  constexpr float kMul = float(1u << (BITS * kF));
-  const uint32_t x = ((w >> kShift) & kMask) | 0x64006400u;
-  const __half2 inv = __float2half2_rn(1.0f / kMul);
-  const __half2 off = __float2half2_rn(-1024.0f / kMul);
-  return h2_as_u32(__hfma2(u32_as_h2(x), inv, off));
+  const uint32_t mask = kLowMask << (BITS * kF);
+  const uint32_t one024 = 0x64006400u;
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w >> kShift), "r"(mask), "r"(one024));
+  return d;
+}
+template <int BITS, int F_IDX>
+__host__ __device__ constexpr int code_log2_mul() {
+  return BITS * (F_IDX % (8 / BITS));
+}
+// fp16x2 bit pattern of (2^-e, 2^-e).
+__host__ __device__ constexpr uint32_t h2_pow2_neg(int e) {
+  return ((uint32_t)(15 - e) << 10) | ((uint32_t)(15 - e) << 26);
+}
+constexpr uint32_t kH2One024 = 0x64006400u;   // (1024, 1024)
+
+// Exact fp16 pair (code_lo, code_hi) of field f of a packed word: the
+// offset pair 1024 + m*code (code_offset) times 1/m minus 1024/m in one
+// fused fp16x2 multiply-add (small integers times powers of two: exact).
+template <int BITS, int F_IDX>
+__device__ __forceinline__ uint32_t unpack_pair(uint32_t w) {
+  constexpr int e = code_log2_mul<BITS, F_IDX>();
+  constexpr uint32_t kOff = 0x8000u | ((uint32_t)(25 - e) << 10);   // -2^(10-e)
+  return hfma2_b(code_offset<BITS, F_IDX>(w), h2_pow2_neg(e), kOff | (kOff << 16));
 }
 
 // Compile-time loop: f(std::integral_constant<int, i>) for i = 0 .. N-1.

@@ -32,10 +32,11 @@ struct Geom {
   int64_t lens_off, counters_off, blocks_off, tails_off, tail_bytes, total_bytes;
 };
 
-// Workspace of kvq_decode: [error word | tickets | partials].
+// Workspace of kvq_decode: [error word | per-unit split records | partials].
+// A split record is {first partial slot, number of pieces} of one unit.
 struct WsLayout {
-  int64_t err_off, tickets_off, partials_off, total;
-  int32_t units;      // tickets
+  int64_t err_off, units_off, partials_off, total;
+  int32_t units;       // split records
   int32_t slot_floats; // floats per partial slot: heads * (d + 2)
 };
 
@@ -81,8 +82,8 @@ inline void make_ws_layout(const Geom& g, WsLayout* w) {
   w->units = g.max_seqs * g.hkv * g.slices;
   w->slot_floats = kHeadsPerSlice * (g.d + 2);
   w->err_off = 0;
-  w->tickets_off = 256;
-  w->partials_off = align_up(w->tickets_off + 4LL * w->units, 256);
+  w->units_off = 256;
+  w->partials_off = align_up(w->units_off + 8LL * w->units, 256);
   w->total = align_up(w->partials_off + 2LL * kMaxDecodeCtas * w->slot_floats * 4, 256);
 }
 

@@ -146,7 +146,7 @@ KVQ_API const char* kvq_last_error(void);
 KVQ_API kvq_status kvq_layout_for(const kvq_config* cfg, kvq_layout* out);
 
 /* Bytes the caller must provide: the cache buffer and the decode workspace
- * (split partials, per-unit tickets and an error word).  Either output
+ * (split partials, per-unit split records and an error word).  Either output
  * pointer may be NULL.  Host only.  Errors: KVQ_ERR_NULL, KVQ_ERR_CONFIG. */
 KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* cache_bytes,
                                     size_t* workspace_bytes);
@@ -188,8 +188,10 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kv
  * (fp16, bf16 or fp32, 16-byte aligned); out device [n_seq, n_q_heads, d]
  * fp16.  workspace: device buffer of at least the workspace_bytes reported
  * by kvq_cache_required_bytes, 256-byte aligned, zero-filled before its
- * first use (kvq_workspace_init); every completed call leaves it ready for
- * the next.  Calls that share a workspace must not overlap on the GPU.
+ * first use (kvq_workspace_init).  Calls that share a workspace must not
+ * overlap on the GPU.  The call launches the split-K decode kernel and a
+ * small combine kernel that merges the units split across CTAs (launched
+ * as a programmatic dependent of the first).
  * Errors (host side): KVQ_ERR_NULL, KVQ_ERR_ARG, KVQ_ERR_CAPACITY,
  * KVQ_ERR_EMPTY (some sequence has length 0), KVQ_ERR_DTYPE,
  * KVQ_ERR_ALIGN, KVQ_ERR_BUFFER_TOO_SMALL; KVQ_ERR_CUDA on launch failure.
@@ -209,18 +211,19 @@ KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype
  * every device allocation and has no workspace hook, and deployments that
  * forbid allocation after start-up.  The pages have no counterpart of this
  * call: it only changes where the decode scratch lives.
- * Instead of a caller workspace, the scratch (error word, per-unit tickets,
- * split partials) is a fixed 8 MiB device array inside the library
+ * Instead of a caller workspace, the scratch (error word, per-unit split
+ * records, split partials) is a fixed 8 MiB device array inside the library
  * (kvq_noalloc_scratch_bytes()); every GPU that loads the library holds it
- * until exit.  The call allocates nothing: it clears the error word and
- * tickets with cudaMemsetAsync, lowers the number of CTAs until the
+ * until exit.  The call allocates nothing: it clears the error word and the
+ * split records with cudaMemsetAsync, lowers the number of CTAs until the
  * partials fit, and launches the same decode kernel.  All calls share the
  * array, which keeps the last call's contents, so calls that overlap on the
  * GPU (other streams, other threads) race: serialize them.  The first call on
  * each device looks up the array's device address (cudaGetSymbolAddress);
  * make that first call before any stream capture.  Arguments and errors as
  * kvq_decode; KVQ_ERR_CAPACITY if the cache has so many (sequence, kv head,
- * head slice) units that even one CTA's partials do not fit.  A failed
+ * head slice) units that their split records leave no room for even one
+ * CTA's partials.  A failed
  * internal wait (never expected) is recorded only in the array's error
  * word, which the next call clears; use kvq_decode with a workspace where
  * that report matters.  Bit-for-bit
