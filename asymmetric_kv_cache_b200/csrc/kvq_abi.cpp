@@ -250,6 +250,26 @@ kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype 
   return ok();
 }
 
+namespace {
+// Decode grid: one CTA per resident slot up to the cap.  When every
+// sequence has the same number of slots and the units fit the cap, a
+// multiple of the unit count (if it keeps >= 80% of the cap) makes every
+// CTA range end on a unit boundary: one piece per CTA, no CTA pays a
+// second prologue and merge.
+int64_t choose_grid(const kvq::Geom& g, const int32_t* lens, int n_seq, int64_t slots, int cap) {
+  int64_t grid = std::min<int64_t>(slots, cap);
+  const int64_t units = (int64_t)n_seq * g.hkv * g.slices;
+  const int w0 = lens[0] / g.G + (lens[0] % g.G ? 1 : 0);
+  bool equal = true;
+  for (int b = 1; b < n_seq && equal; ++b) equal = (lens[b] / g.G + (lens[b] % g.G ? 1 : 0)) == w0;
+  if (equal && units <= cap) {
+    const int64_t alt = std::min<int64_t>(slots, units * (cap / units));
+    if (alt * 5 >= (int64_t)cap * 4) grid = alt;
+  }
+  return grid;
+}
+}  // namespace
+
 kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* out,
                       int32_t n_seq, void* workspace, size_t ws_bytes, void* stream) {
   if (!cache) return fail(KVQ_ERR_NULL, "cache is NULL");
@@ -283,7 +303,7 @@ kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* 
     const int v = std::atoi(env);
     if (v > 0) cap = std::min(cap, v);
   }
-  const int grid = (int)std::min<int64_t>(slots, cap);
+  const int grid = (int)choose_grid(g, cache->lens.data(), n_seq, slots, cap);
   kvq::DecodeArgs a;
   a.cache = cache->buf;
   a.q = q;
@@ -330,7 +350,7 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
     cudaError_t e = kvq::decode_max_ctas(g, &cache->max_ctas);
     if (e != cudaSuccess) return cuda_fail(e, "decode occupancy query");
   }
-  int64_t grid = std::min<int64_t>(slots, cache->max_ctas);
+  int64_t grid = choose_grid(g, cache->lens.data(), n_seq, slots, cache->max_ctas);
   grid = std::min<int64_t>(grid, room / slot_bytes);
   void* scratch = nullptr;
   cudaError_t e = kvq::noalloc_scratch(&scratch);

@@ -22,14 +22,16 @@
 //   * waits for the group block, brought into its own shared-memory ring by
 //     a 1-D bulk (TMA) copy issued NST groups ahead;
 //   * folds the per-channel key scales into the query: q'_c = q_c s_c, so
-//     q . k_hat = sum_c q'_c code_c + sum_c q_c z_c; the second sum (one per
-//     group and head) runs on the tensor core with q split into fp16 high and
-//     low halves (rows 0-7 and 8-15 of the tile) against the key mins;
-//   * unpacks key codes to exact fp16 pairs and runs S^T = codes q'^T on
-//     m16n8k16 tiles (rows = 16 tokens, columns = the 8 query heads of the
-//     GQA group), so each lane's softmax state covers two heads;
+//     q . k_hat = sum_c q'_c code_c + sum_c q_c z_c, the second sum (the
+//     key-min bias, one per group and head) on the tensor core as well;
+//   * runs S = q' codes^T on m16n8k16 tiles whose 16 rows are the 8 query
+//     heads of the GQA group twice: rows 0-7 carry q' rounded to fp16 and
+//     rows 8-15 the rounding residual, so the logits keep ~22 bits of q'
+//     at no extra tile; the 8 columns are 8 tokens, so a lane ends up with
+//     two tokens of one head per tile;
 //   * updates the running max / rescales, exponentiates (exp2 domain) and
-//     transposes the fp16 P tile in registers (movmatrix);
+//     packs P to fp16: the accumulator layout of S is already the B-operand
+//     layout of the value product;
 //   * runs O^T += V_code^T (p s_v) on tiles whose rows are channels and whose
 //     columns are heads, with the per-token value scale folded into p for
 //     each channel group, and sum_t p_t z_t (value mins) and sum_t p_t (the
@@ -49,6 +51,19 @@ constexpr int kThreads = 128;
 constexpr int kWarps = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Staging area of the fp16 tail (T tokens, 0 < T < G) of one (sequence, kv
+// head), 16 tokens at a time by cp.async: key rows and value token-pair
+// rows, padded so that the fragment reads are free of bank conflicts; rows
+// past T are zero-filled.  It is the tail warp's (idle) ring when that is
+// large enough, else a CTA area of its own (a piece has at most one tail).
+template <int D>
+struct TailStage {
+  static constexpr int KROW = 2 * D + 16;       // bytes per padded key row
+  static constexpr int VROW = 4 * D + 16;       // bytes per padded value pair-row
+  static constexpr int VOFF = 16 * KROW;
+  static constexpr int BYTES = VOFF + 8 * VROW;
+};
+
 template <int D, int KB, int VB, int G>
 struct DecCfg {
   static constexpr int KT = D / 16;   // 16-channel k-tiles of q.k
@@ -67,65 +82,81 @@ struct DecCfg {
   static constexpr int SEC_VSCALE = SEC_VCODES + G * D * VB / 8;
   static constexpr int SEC_VMIN = SEC_VSCALE + 2 * G * J;
   static constexpr int BLK = SEC_VMIN + 2 * G * J;
-  static constexpr int NST = (BLK <= 4096) ? 3 : 2;   // ring stages per warp
+  // Ring stages per warp.  Two keep more bytes in flight than the HBM
+  // latency needs at 4 CTAs per SM; deeper rings only lengthen the queue
+  // that every other request (the query, the next unit's first blocks)
+  // waits behind.
+  static constexpr int NST = 2;
   // resident CTAs per SM the register budget aims at (shared memory allows
-  // four CTAs with 3-stage rings of blocks up to 4 KB, three otherwise)
+  // four CTAs with blocks up to 4 KB, three otherwise)
   static constexpr int MIN_BLOCKS = (BLK <= 4096) ? 4 : 3;
   static constexpr int RING = kWarps * NST * BLK;
   // query fragments of the current unit, shared by the CTA's warps:
-  // [kt][lane][4 words] = {hi v0, lo v0, hi v1, lo v1}
+  // [kt][lane][4 words] = {hi v0, lo v0, hi v1, lo v1}.  The raw query rows
+  // of the unit (<= 8 heads x D, fp32 at most) land here first by a bulk
+  // copy and are converted in place.
   static constexpr int QA_OFF = RING;
   static constexpr int QA_BYTES = KT * 32 * 16;
-  // both parts divided by the key code multiplier m of their register,
-  // [kt][lane][4 words] (the B operand of q.k is (q_hi/m + q_lo/m) * s_k)
-  static constexpr int QM_OFF = QA_OFF + QA_BYTES;
-  static constexpr int QM_BYTES = KT * 32 * 16;
+  static_assert(kHeadsPerSlice * D * 4 <= QA_BYTES, "raw query rows fit the fragment area");
+  // merge area (in the idle ring between pieces): the warps' (o, m, l) per
+  // head, then the per-head weights of the 4 warps, the max and the sum
   static constexpr int MERGE_FLOATS = kWarps * kHeadsPerSlice * (D + 2);
-  static_assert(MERGE_FLOATS * 4 <= RING, "merge area must fit in the ring");
-  static constexpr int BAR_OFF = QM_OFF + QM_BYTES;
-  static constexpr int SMEM_FIXED = BAR_OFF + kWarps * NST * 8 + 64;
+  static constexpr int WTS_OFF = MERGE_FLOATS;
+  static_assert((MERGE_FLOATS + 6 * kHeadsPerSlice) * 4 <= RING, "merge area must fit in the ring");
+  // The tail (< G tokens, G/16 chunks of 16).  For 32-token groups the
+  // whole tail gets an area of its own: it is staged when the piece starts
+  // and processed first, its copy latency hidden behind the prologue.  For
+  // larger groups it goes through the tail warp's ring, after its groups.
+  static constexpr int TAIL_CHUNKS = G / 16;
+  static constexpr bool TAIL_EARLY = (G == 32);
+  static_assert(TAIL_EARLY || TailStage<D>::BYTES <= NST * BLK, "tail chunk fits a warp's ring");
+  static constexpr int TAIL_OFF = QA_OFF + QA_BYTES;
+  static constexpr int BAR_OFF = TAIL_OFF + (TAIL_EARLY ? TAIL_CHUNKS * TailStage<D>::BYTES : 0);
+  static constexpr int SMEM_FIXED = BAR_OFF + (kWarps * NST + 1) * 8 + 56;
 };
 
 template <int D, int KB, int VB, int G>
 struct WarpState {
   float o[D / 16][4];   // O^T: (channel 16mt + g, heads 2i, 2i+1), then channel + 8
   float z[4];           // rows: value-min terms (j < J) and sum p (row J); cols heads
-  float m[2];           // running max of heads 2i, 2i+1 (i = lane & 3), log2 domain
+  float m;              // running max of head lane/4, log2 domain
 };
 
 // Query fragments of head g = lane/4 (zeros for a padding head), channels
 // 16kt + 2i + {0,1} (v = 0) and + 8 (v = 1), i = lane & 3: q is scaled by
 // log2(e)/sqrt(d), split into fp16 high and low parts and stored per lane
 // as qs[kt * 32 + lane] = {hi v0, lo v0, hi v1, lo v1} - the A quad of the
-// key-min tile (rows g: high part, rows g + 8: low part).
-template <int D, int KB>
-__device__ __forceinline__ void load_query(const void* q, int dtype, int64_t row, bool valid,
-                                           int lane, uint4* __restrict__ qs,
-                                           uint4* __restrict__ qm) {
-  const int i4 = lane & 3;
+// q.k tiles (rows g: high part, rows g + 8: low part).  The unit's raw rows
+// (head g at g * D elements) were copied into the same bytes; every lane
+// reads its values before any lane writes.
+template <int D>
+__device__ __forceinline__ void load_query(int dtype, bool valid, int lane,
+                                           uint4* __restrict__ qs) {
+  const int g8 = lane >> 2, i4 = lane & 3;
   const float sc = kLog2e * rsqrtf((float)D);
+  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
   float2 x[D / 16][2];
 #pragma unroll
   for (int kt = 0; kt < D / 16; ++kt) {
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
-      const int64_t idx = row * D + 16 * kt + 8 * v + 2 * i4;
+      const int idx = g8 * D + 16 * kt + 8 * v + 2 * i4;
       float2 f = make_float2(0.f, 0.f);
       if (valid) {
         if (dtype == KVQ_FP16) {
-          f = __half22float2(*reinterpret_cast<const __half2*>(reinterpret_cast<const __half*>(q) + idx));
+          f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
         } else if (dtype == KVQ_BF16) {
-          f = __bfloat1622float2(
-              *reinterpret_cast<const __nv_bfloat162*>(reinterpret_cast<const __nv_bfloat16*>(q) + idx));
+          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
         } else {
-          f = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(q) + idx);
+          f = *reinterpret_cast<const float2*>(raw + 4 * idx);
         }
       }
       x[kt][v] = f;
     }
   }
-  static_for<D / 16>([&](auto kt_) {
-    constexpr int kt = decltype(kt_)::value;
+  __syncwarp();
+#pragma unroll
+  for (int kt = 0; kt < D / 16; ++kt) {
     uint32_t w[4];
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
@@ -136,37 +167,30 @@ __device__ __forceinline__ void load_query(const void* q, int dtype, int64_t row
       w[2 * v + 1] = pack_h2(x0 - hf.x, x1 - hf.y);
     }
     qs[kt * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-    constexpr int FK = 16 / KB;
-    constexpr int e0 = code_log2_mul<KB, (2 * kt) % FK>();
-    constexpr int e1 = code_log2_mul<KB, (2 * kt + 1) % FK>();
-    qm[kt * 32 + lane] = make_uint4(hmul2_b(w[0], h2_pow2_neg(e0)), hmul2_b(w[1], h2_pow2_neg(e0)),
-                                    hmul2_b(w[2], h2_pow2_neg(e1)), hmul2_b(w[3], h2_pow2_neg(e1)));
-  });
+  }
 }
 
-// Online-softmax update for new logits in the transposed tile layout:
-// s[mt] = {(token g, head 2i), (token g, head 2i+1), (token g+8, head 2i),
-// (token g+8, head 2i+1)} of a 16-token tile mt (g = lane/4, i = lane&3).
-// Produces the fp16 probabilities as B fragments of the p.v tile
-// (pt[mt] = {tokens 0-7, tokens 8-15} of head g, 2 tokens per lane).
-template <int D, int NM, int KB, int VB, int G>
-__device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, float (&s)[NM][4],
-                                               uint32_t (&pt)[NM][2]) {
-  float mx0 = -INFINITY, mx1 = -INFINITY;
+// Online-softmax update for new logits in the S tile layout: s[nt] =
+// {(head g, token 8nt + 2i), (head g, token 8nt + 2i + 1)} (g = lane/4,
+// i = lane&3).  Produces the fp16 probabilities pt[nt] in the same places,
+// which is the B fragment of the value product (tokens 2i, 2i+1 of head g).
+// The accumulators O^T and Z hold heads 2i and 2i+1 in their columns; their
+// rescale factors come from the lanes that own those heads.
+template <int D, int NT, int KB, int VB, int G>
+__device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, float (&s)[NT][2],
+                                               uint32_t (&pt)[NT], int i4) {
+  float mx = fmaxf(s[0][0], s[0][1]);
 #pragma unroll
-  for (int mt = 0; mt < NM; ++mt) {
-    mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
-    mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
-  }
-#pragma unroll
-  for (int o = 4; o <= 16; o <<= 1) {   // across the 8 token rows (lane bits 2-4)
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  const float n0 = fmaxf(st.m[0], mx0), n1 = fmaxf(st.m[1], mx1);
-  if (__any_sync(0xffffffffu, n0 > st.m[0] || n1 > st.m[1])) {
-    if (st.m[0] != -INFINITY) {   // accumulators hold data: rescale them
-      const float a0 = fast_exp2(st.m[0] - n0), a1 = fast_exp2(st.m[1] - n1);
+  for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s[nt][0], s[nt][1]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));   // the 4 lanes of head g
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float n = fmaxf(st.m, mx);
+  if (__any_sync(0xffffffffu, n > st.m)) {
+    // every head gets its first logits in the same call: uniform branch
+    if (st.m != -INFINITY) {   // accumulators hold data: rescale them
+      const float al = fast_exp2(st.m - n);
+      const float a0 = __shfl_sync(0xffffffffu, al, 8 * i4);
+      const float a1 = __shfl_sync(0xffffffffu, al, 8 * i4 + 4);
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) {
         st.o[mt][0] *= a0;
@@ -179,93 +203,89 @@ __device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, floa
       st.z[2] *= a0;
       st.z[3] *= a1;
     }
-    st.m[0] = n0;
-    st.m[1] = n1;
+    st.m = n;
   }
 #pragma unroll
-  for (int mt = 0; mt < NM; ++mt) {
-    pt[mt][0] = movmatrix_trans(
-        pack_h2(fast_exp2(s[mt][0] - st.m[0]), fast_exp2(s[mt][1] - st.m[1])));
-    pt[mt][1] = movmatrix_trans(
-        pack_h2(fast_exp2(s[mt][2] - st.m[0]), fast_exp2(s[mt][3] - st.m[1])));
-  }
+  for (int nt = 0; nt < NT; ++nt)
+    pt[nt] = pack_h2(fast_exp2(s[nt][0] - st.m), fast_exp2(s[nt][1] - st.m));
 }
 
 // One quantized group from the shared-memory stage `sp`.
 //
 // Key codes enter the tensor core as x = 1024 + m*code (code_offset) against
-// B = (q/m) * s_k, carried as an fp16 high + low pair (one fp16 rounding of
-// the product would cost ~2^-12 of each logit term, which matters for
-// channels with large scales); the offset is removed with tiles against a
-// constant 1024 operand, which sum exactly the fp16 B values the tensor core
-// saw.  Value
-// codes are unpacked to exact fp16 integers (unpack_pair).
+// A = q * (s_k/m) as fp16 high (rows 0-7) and residual (rows 8-15) parts
+// (one fp16 rounding of the product would cost ~2^-12 of each logit term,
+// which matters for channels with large scales); the offset is removed with
+// one tile per k-step against a constant -1024 operand, which sums exactly
+// the fp16 A values the tensor core saw, and accumulates with the key-min
+// bias.  Value codes are unpacked to exact fp16 integers (unpack_pair).
 template <int D, int KB, int VB, int G>
 __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
                                               const unsigned char* __restrict__ sp,
-                                              const uint4* __restrict__ qsm,
-                                              const uint4* __restrict__ qmsm, int lane) {
+                                              const uint4* __restrict__ qsm, int lane) {
   using C = DecCfg<D, KB, VB, G>;
-  constexpr int NM = G / 16;
+  constexpr int NT = G / 8;
+  // key-code words held at once per token tile: all of them when that is at
+  // most 8 registers, two at a time otherwise
+  constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
+  constexpr int KT_PER_CH = WCH * C::FK / 2;   // k-steps covered by a chunk
+  static_assert(C::KT % KT_PER_CH == 0, "k-steps split evenly into code chunks");
   const int g8 = lane >> 2, i4 = lane & 3;
 
-  // B = (q s_k) / m as an fp16 high + low pair, the key-min term and the
-  // offset correction
-  uint32_t qs[C::KT][2], ql[C::KT][2];
-  float bias[4] = {0.f, 0.f, 0.f, 0.f};
-  float kcor[4] = {0.f, 0.f, 0.f, 0.f};
-  {
-    uint32_t ksw[D / 8], kzw[D / 8];
-    lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8), ksw);
-    lds_words<D / 8>(reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8), kzw);
-    static_for<C::KT>([&](auto kt_) {
-      constexpr int kt = decltype(kt_)::value;
-      const uint4 q4 = qsm[kt * 32 + lane];
-      const uint4 qm = qmsm[kt * 32 + lane];
-      // high part: one rounding of hi*s + lo*s; low part: the rest of it,
-      // (hi*s - high) exact in one fused step, plus lo*s
-      const uint32_t s0 = ksw[2 * kt], s1 = ksw[2 * kt + 1];
-      qs[kt][0] = hfma2_b(qm.x, s0, hmul2_b(qm.y, s0));
-      qs[kt][1] = hfma2_b(qm.z, s1, hmul2_b(qm.w, s1));
-      ql[kt][0] = hfma2_b(qm.y, s0, hfma2_b(qm.x, s0, qs[kt][0] ^ 0x80008000u));
-      ql[kt][1] = hfma2_b(qm.w, s1, hfma2_b(qm.z, s1, qs[kt][1] ^ 0x80008000u));
-      mma16816(bias, q4.x, q4.y, q4.z, q4.w, kzw[2 * kt], kzw[2 * kt + 1]);
-      mma16816(kcor, kH2One024, kH2One024, kH2One024, kH2One024, qs[kt][0], qs[kt][1]);
-      mma16816(kcor, kH2One024, kH2One024, kH2One024, kH2One024, ql[kt][0], ql[kt][1]);
-    });
-  }
-  // bias of head g8 is in every lane of quad g8; fetch heads 2*i4 and 2*i4+1
-  const float bg = bias[0] + bias[2];
-  const float b0 = __shfl_sync(0xffffffffu, bg, 8 * i4) - kcor[0];
-  const float b1 = __shfl_sync(0xffffffffu, bg, 8 * i4 + 4) - kcor[1];
-
-  // S^T = codes q'^T: rows = tokens (two 8-token code tiles), cols = heads
-  float s[NM][4];
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
-  static_for<NM>([&](auto mt_) {
-    constexpr int mt = decltype(mt_)::value;
-    uint32_t kw0[C::LWK], kw1[C::LWK];
-    lds_words<C::LWK>(kcw + ((2 * mt) * 32 + lane) * C::LWK, kw0);
-    lds_words<C::LWK>(kcw + ((2 * mt + 1) * 32 + lane) * C::LWK, kw1);
-    float acc[4] = {b0, b1, b0, b1};
-    static_for<C::KT>([&](auto kt_) {
-      constexpr int kt = decltype(kt_)::value;
-      constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
-      const uint32_t a0 = code_offset<KB, p0 % C::FK>(kw0[p0 / C::FK]);   // token g
-      const uint32_t a1 = code_offset<KB, p0 % C::FK>(kw1[p0 / C::FK]);   // token g + 8
-      const uint32_t a2 = code_offset<KB, p1 % C::FK>(kw0[p1 / C::FK]);   // channels + 8
-      const uint32_t a3 = code_offset<KB, p1 % C::FK>(kw1[p1 / C::FK]);
-      mma16816(acc, a0, a1, a2, a3, qs[kt][0], qs[kt][1]);
-      mma16816(acc, a0, a1, a2, a3, ql[kt][0], ql[kt][1]);
-    });
-    s[mt][0] = acc[0];
-    s[mt][1] = acc[1];
-    s[mt][2] = acc[2];
-    s[mt][3] = acc[3];
-  });
+  const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
+  const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
+  constexpr uint32_t kH2Neg1024 = 0xE400E400u;   // (-1024, -1024)
 
-  uint32_t pt[NM][2];
-  softmax_update<D, NM, KB, VB, G>(st, s, pt);
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  float bacc[4] = {0.f, 0.f, 0.f, 0.f};   // key-min bias (rows: high, low part)
+  float cacc[4] = {0.f, 0.f, 0.f, 0.f};   // minus the code offset
+  static_for<C::KT / KT_PER_CH>([&](auto ch_) {
+    constexpr int ch = decltype(ch_)::value;
+    uint32_t kw[NT][WCH];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      lds_words<WCH>(kcw + (nt * 32 + lane) * C::LWK + ch * WCH, kw[nt]);
+    static_for<KT_PER_CH>([&](auto kk_) {
+      constexpr int kt = ch * KT_PER_CH + decltype(kk_)::value;
+      constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;   // code pairs: channels +0-7, +8-15
+      const uint2 s2 = *reinterpret_cast<const uint2*>(ksw + 2 * kt);
+      const uint2 z2 = *reinterpret_cast<const uint2*>(kzw + 2 * kt);
+      const uint4 q4 = qsm[kt * 32 + lane];
+      // s_k / m of the code pair's field (a power-of-two scaling: exact
+      // while s_k / m stays a normal fp16 number)
+      constexpr int e0 = code_log2_mul<KB, p0 % C::FK>(), e1 = code_log2_mul<KB, p1 % C::FK>();
+      const uint32_t sm0 = e0 ? hmul2_b(s2.x, h2_pow2_neg(e0)) : s2.x;
+      const uint32_t sm1 = e1 ? hmul2_b(s2.y, h2_pow2_neg(e1)) : s2.y;
+      // high part: one rounding of hi*s + lo*s; residual: (hi*s - high) in
+      // one fused step (exact), plus lo*s
+      const uint32_t a0 = hfma2_b(q4.x, sm0, hmul2_b(q4.y, sm0));
+      const uint32_t a2 = hfma2_b(q4.z, sm1, hmul2_b(q4.w, sm1));
+      const uint32_t a1 = hfma2_b(q4.y, sm0, hfma2_negc_b(q4.x, sm0, a0));
+      const uint32_t a3 = hfma2_b(q4.w, sm1, hfma2_negc_b(q4.z, sm1, a2));
+      mma16816(bacc, q4.x, q4.y, q4.z, q4.w, z2.x, z2.y);
+      mma16816(cacc, a0, a1, a2, a3, kH2Neg1024, kH2Neg1024);
+      static_for<NT>([&](auto nt_) {
+        constexpr int nt = decltype(nt_)::value;
+        constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
+        mma16816(acc[nt], a0, a1, a2, a3, code_offset<KB, p0 % C::FK>(kw[nt][w0]),
+                 code_offset<KB, p1 % C::FK>(kw[nt][w1]));
+      });
+    });
+  });
+  // head g's bias: both row halves (every column holds the same value)
+  const float bias = (bacc[0] + cacc[0]) + (bacc[2] + cacc[2]);
+  float s[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    s[nt][0] = (acc[nt][0] + acc[nt][2]) + bias;
+    s[nt][1] = (acc[nt][1] + acc[nt][3]) + bias;
+  }
+
+  uint32_t pt[NT];
+  softmax_update<D, NT, KB, VB, G>(st, s, pt, lane & 3);
 
   // O^T += V^T (p * s_v); Z += [z_v; 1]^T p
   const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
@@ -277,7 +297,7 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
   static_for<C::KV>([&](auto kv_) {
     constexpr int kv = decltype(kv_)::value;
-    const uint32_t bp0 = pt[kv][0], bp1 = pt[kv][1];
+    const uint32_t bp0 = pt[2 * kv], bp1 = pt[2 * kv + 1];
     const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
     mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
 
@@ -305,67 +325,60 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   });
 }
 
-// The fp16 tail (T tokens, 0 < T < G) of one (sequence, kv head), staged
-// 16 tokens at a time through the warp's (idle) ring with cp.async: key rows
-// and value token-pair rows, padded so that the fragment reads below are
-// free of bank conflicts; rows past T are zero-filled.
+// Issue the cp.async copies of tail chunk kv (16 tokens: key rows and
+// value token-pair rows) into `buf`; nothing waits here.
 template <int D>
-struct TailStage {
-  static constexpr int KROW = 2 * D + 16;       // bytes per padded key row
-  static constexpr int VROW = 4 * D + 16;       // bytes per padded value pair-row
-  static constexpr int VOFF = 16 * KROW;
-  static constexpr int BYTES = VOFF + 8 * VROW;
-};
+__device__ __forceinline__ void stage_tail_chunk(unsigned char* __restrict__ buf,
+                                                 const __half* __restrict__ tk,
+                                                 const __half* __restrict__ tv, int T, int kv,
+                                                 int lane) {
+  using TS = TailStage<D>;
+  for (int seg = lane; seg < 16 * (D / 8); seg += 32) {
+    const int r = seg / (D / 8), cs = seg % (D / 8), t = 16 * kv + r;
+    cp_async16(buf + r * TS::KROW + cs * 16, tk + (t < T ? (int64_t)t * D + cs * 8 : 0),
+               t < T ? 16u : 0u);
+  }
+  for (int seg = lane; seg < 8 * (D / 4); seg += 32) {
+    const int pr = seg / (D / 4), cs = seg % (D / 4), pp = 8 * kv + pr;
+    cp_async16(buf + TS::VOFF + pr * TS::VROW + cs * 16,
+               tv + (2 * pp < T ? (int64_t)pp * 2 * D + cs * 8 : 0), 2 * pp < T ? 16u : 0u);
+  }
+}
 
+// Attention over staged tail chunk kv (tokens 16kv .. 16kv + 15, those
+// past T masked out).
 template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
-                                             const __half* __restrict__ tk,
-                                             const __half* __restrict__ tv, int T,
-                                             const uint4* __restrict__ qsm, int lane,
-                                             unsigned char* __restrict__ buf) {
+__device__ __forceinline__ void tail_chunk(WarpState<D, KB, VB, G>& st,
+                                           const unsigned char* __restrict__ buf, int T, int kv,
+                                           const uint4* __restrict__ qsm, int lane) {
   using C = DecCfg<D, KB, VB, G>;
   using TS = TailStage<D>;
-  static_assert(TS::BYTES <= C::NST * C::BLK, "tail chunk must fit in a warp's ring");
   const int g8 = lane >> 2, i4 = lane & 3;
-  for (int kv = 0; kv * 16 < T; ++kv) {
-    // stage 16 key rows and 8 value pair-rows (16-byte pieces)
-    for (int seg = lane; seg < 16 * (D / 8); seg += 32) {
-      const int r = seg / (D / 8), cs = seg % (D / 8), t = 16 * kv + r;
-      cp_async16(buf + r * TS::KROW + cs * 16, tk + (t < T ? (int64_t)t * D + cs * 8 : 0),
-                 t < T ? 16u : 0u);
-    }
-    for (int seg = lane; seg < 8 * (D / 4); seg += 32) {
-      const int pr = seg / (D / 4), cs = seg % (D / 4), pp = 8 * kv + pr;
-      cp_async16(buf + TS::VOFF + pr * TS::VROW + cs * 16,
-                 tv + (2 * pp < T ? (int64_t)pp * 2 * D + cs * 8 : 0), 2 * pp < T ? 16u : 0u);
-    }
-    cp_async_wait_all();
-    __syncwarp();
-
-    // S^T = K q^T with q = high + low parts (two products per tile)
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    // S = q K^T, rows: q high / low parts, columns: 8 tokens per tile
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
-    const unsigned char* k1 = k0 + 8 * TS::KROW;
 #pragma unroll
     for (int kt = 0; kt < C::KT; ++kt) {
-      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(k0 + 32 * kt);
-      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(k1 + 32 * kt);
-      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16);
-      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16);
       const uint4 q4 = qsm[kt * 32 + lane];
-      mma16816(acc, a0, a1, a2, a3, q4.x, q4.z);
-      mma16816(acc, a0, a1, a2, a3, q4.y, q4.w);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const unsigned char* kr = k0 + 8 * nt * TS::KROW + 32 * kt;
+        mma16816(acc[nt], q4.x, q4.y, q4.z, q4.w, *reinterpret_cast<const uint32_t*>(kr),
+                 *reinterpret_cast<const uint32_t*>(kr + 16));
+      }
     }
-    const int t0 = 16 * kv + g8, t1 = t0 + 8;
-    float s[1][4];
-    s[0][0] = (t0 < T) ? acc[0] : -INFINITY;
-    s[0][1] = (t0 < T) ? acc[1] : -INFINITY;
-    s[0][2] = (t1 < T) ? acc[2] : -INFINITY;
-    s[0][3] = (t1 < T) ? acc[3] : -INFINITY;
-    uint32_t pt[1][2];
-    softmax_update<D, 1, KB, VB, G>(st, s, pt);
+    float s[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int t = 16 * kv + 8 * nt + 2 * i4;
+      s[nt][0] = (t < T) ? acc[nt][0] + acc[nt][2] : -INFINITY;
+      s[nt][1] = (t + 1 < T) ? acc[nt][1] + acc[nt][3] : -INFINITY;
+    }
+    uint32_t pt[2];
+    softmax_update<D, 2, KB, VB, G>(st, s, pt, i4);
     const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
-    mma16816(st.z, ones, 0u, ones, 0u, pt[0][0], pt[0][1]);
+    mma16816(st.z, ones, 0u, ones, 0u, pt[0], pt[1]);
     // V^T fragments; the second token of the last pair may be stale: mask it
     const int ta = 16 * kv + 2 * i4, tb = ta + 8;
     const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
@@ -378,9 +391,8 @@ __device__ __forceinline__ void process_tail(WarpState<D, KB, VB, G>& st,
       const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
       const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
       const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
-      mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
+      mma16816(st.o[mt], a0, a1, a2, a3, pt[0], pt[1]);
     }
-    __syncwarp();   // every lane is done with this chunk before the next copy
   }
 }
 
@@ -394,6 +406,34 @@ __device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int pos) {
   return lo;
 }
 
+// The part of unit `unit` (sequence b, kv head kvh, head slice `slice`)
+// that a CTA processes: slots [slot0, slot1) of the unit's wb slots.
+struct Piece {
+  int b, L, ng, Tb, wb, slot0, slot1, kvh, slice, unit, hbase, nh;
+};
+
+// Built from the slot position alone, so that it can be rebuilt after the
+// group loop instead of holding registers through it.
+__device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix,
+                                            const int32_t* slen, int n_seq, int pos, int end) {
+  Piece p;
+  p.b = find_seq(prefix, n_seq, pos);
+  p.L = slen[p.b];
+  p.ng = p.L / g.G;
+  p.Tb = p.L - p.ng * g.G;
+  p.wb = p.ng + (p.Tb ? 1 : 0);
+  const int local = pos - prefix[p.b];
+  const int uis = local / p.wb;
+  p.slot0 = local - uis * p.wb;
+  p.slot1 = min(p.wb, p.slot0 + (end - pos));
+  p.kvh = uis / g.slices;
+  p.slice = uis - p.kvh * g.slices;
+  p.unit = p.b * (g.hkv * g.slices) + uis;
+  p.hbase = p.kvh * g.gqa + p.slice * kHeadsPerSlice;
+  p.nh = min(kHeadsPerSlice, g.gqa - p.slice * kHeadsPerSlice);
+  return p;
+}
+
 template <int D, int KB, int VB, int G>
 __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
@@ -402,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   unsigned char* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint4* qsm = reinterpret_cast<uint4*>(smem + C::QA_OFF);
-  uint4* qmsm = reinterpret_cast<uint4*>(smem + C::QM_OFF);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::SMEM_FIXED);
+  int32_t* slen = prefix + (a.n_seq + 1);   // the sequences' lengths
   float* merge = reinterpret_cast<float*>(smem);   // reuses the ring between pieces
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -420,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) mbar_init(&bars[warp * C::NST + s], 1);
+    if (warp == 0) mbar_init(&bars[kWarps * C::NST], 1);   // the query copy
     fence_mbar_init();
   }
   // ---- slot prefix over sequences: slots(b) = units(b) * (groups + has_tail)
@@ -449,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       const int L = lens[bb];
       acc += per_seq_units * (L / G + (L % G ? 1 : 0));
       prefix[bb + 1] = acc;
+      slen[bb] = L;
     }
   }
   __syncthreads();
@@ -460,50 +502,81 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   const int start = (int)((int64_t)k * T / grid), end = (int)((int64_t)(k + 1) * T / grid);
 
   uint32_t uses = 0;        // ring stage uses of this warp so far
+  uint32_t qphase = 0;      // query copies so far (one per piece)
   bool ok = true;           // no wait has run out
   unsigned char* wring = ring + warp * C::NST * C::BLK;
   uint64_t* wbars = bars + warp * C::NST;
   const unsigned char* blocks = a.cache + g.blocks_off;
 
+  uint64_t* qbar = bars + kWarps * C::NST;
   for (int pos = start; pos < end;) {
-    const int b = find_seq(prefix, n_seq, pos);
-    const int L = lens[b];
-    const int ng = L / G, Tb = L % G;
-    const int wb = ng + (Tb ? 1 : 0);
-    const int local = pos - prefix[b];
-    const int uis = local / wb;
-    const int slot0 = local - uis * wb;
-    const int slot1 = min(wb, slot0 + (end - pos));
-    const int kvh = uis / g.slices, slice = uis % g.slices;
-    const int unit = b * per_seq_units + uis;
-    const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
-    const int nh = min(kHeadsPerSlice, g.gqa - slice * kHeadsPerSlice);
-    const int64_t ublk = ((int64_t)b * g.hkv + kvh) * g.max_groups;
-
     WarpState<D, KB, VB, G> st;
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
-    st.m[0] = st.m[1] = -INFINITY;
+    st.m = -INFINITY;
 
-    // this warp's group slots: slot0 + warp + 4k below min(slot1, ng)
-    const int gend = min(slot1, ng);
-    const int first = slot0 + warp;
-    const int count = (ok && first < gend) ? (gend - first + kWarps - 1) / kWarps : 0;
-    if (lane == 0) {
-      for (int s = 0; s < min(C::NST, count); ++s) {
-        const uint32_t u = uses + s;
-        const int stg = u % C::NST;
+    int first, count, nh;
+    int64_t ublk;
+    bool my_tail;
+    {
+      const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+      ublk = ((int64_t)p.b * g.hkv + p.kvh) * g.max_groups;
+      nh = p.nh;
+      // this warp's group slots: slot0 + warp + 4k below min(slot1, ng);
+      // the tail slot (index ng), if in this piece, belongs to warp
+      // (ng - slot0) % 4
+      const int gend = min(p.slot1, p.ng);
+      first = p.slot0 + warp;
+      count = (ok && first < gend) ? (gend - first + kWarps - 1) / kWarps : 0;
+      my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng &&
+                ((p.ng - p.slot0) % kWarps) == warp;
+      // the unit's raw query rows first, so that they are not queued behind
+      // the group blocks
+      if (tid == 0) {
+        const int esz = a.q_dtype == KVQ_FP32 ? 4 : 2;
+        const uint32_t qbytes = (uint32_t)(p.nh * D * esz);
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&wbars[stg], C::BLK);
-        bulk_copy_g2s(wring + stg * C::BLK, blocks + (ublk + first + kWarps * s) * C::BLK, C::BLK,
-                      &wbars[stg]);
+        mbar_arrive_expect_tx(qbar, qbytes);
+        bulk_copy_g2s(qsm,
+                      static_cast<const unsigned char*>(a.q) +
+                          ((int64_t)p.b * g.hq + p.hbase) * D * esz,
+                      qbytes, qbar);
+      }
+      if (lane == 0) {
+        for (int s = 0; s < min(C::NST, count); ++s) {
+          const uint32_t u = uses + s;
+          const int stg = u % C::NST;
+          mbar_arrive_expect_tx(&wbars[stg], C::BLK);
+          bulk_copy_g2s(wring + stg * C::BLK, blocks + (ublk + first + kWarps * s) * C::BLK,
+                        C::BLK, &wbars[stg]);
+        }
+      }
+      if (C::TAIL_EARLY && my_tail) {
+        const __half* tk = reinterpret_cast<const __half*>(
+            a.cache + g.tails_off + ((int64_t)p.b * g.hkv + p.kvh) * g.tail_bytes);
+        for (int kv = 0; kv * 16 < p.Tb; ++kv)
+          stage_tail_chunk<D>(smem + C::TAIL_OFF + kv * TailStage<D>::BYTES, tk, tk + G * D,
+                              p.Tb, kv, lane);
       }
     }
-    // while the copies fly, warp 0 prepares the unit's query fragments
-    if (warp == 0)
-      load_query<D, KB>(a.q, a.q_dtype, (int64_t)b * g.hq + hbase + g8, g8 < nh, lane, qsm, qmsm);
+    // while the blocks fly, warp 0 turns the query rows into fragments
+    if (warp == 0) {
+      bool got = mbar_wait_bounded(qbar, qphase & 1);
+      got = __all_sync(0xffffffffu, got);
+      if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
+      load_query<D>(a.q_dtype, got && g8 < nh, lane, qsm);
+    }
+    ++qphase;
     __syncthreads();
+    if (C::TAIL_EARLY && my_tail) {
+      cp_async_wait_all();
+      __syncwarp();
+      const int Tb = slen[find_seq(prefix, n_seq, pos)] % G;
+      for (int kv = 0; kv * 16 < Tb; ++kv)
+        tail_chunk<D, KB, VB, G>(st, smem + C::TAIL_OFF + kv * TailStage<D>::BYTES, Tb, kv, qsm,
+                                 lane);
+    }
     for (int it = 0; it < count; ++it) {
       const uint32_t u = uses + it;
       const int stg = u % C::NST;
@@ -514,10 +587,12 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
         if (lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
         break;
       }
-      process_group<D, KB, VB, G>(st, wring + stg * C::BLK, qsm, qmsm, lane);
+      process_group<D, KB, VB, G>(st, wring + stg * C::BLK, qsm, lane);
       __syncwarp();
+      // refill the stage: the warp's reads of it are complete (their values
+      // were consumed before __syncwarp), and a bulk copy that overwrites
+      // bytes which were only read needs no proxy fence
       if (lane == 0 && it + C::NST < count) {
-        fence_proxy_async_smem();
         mbar_arrive_expect_tx(&wbars[stg], C::BLK);
         bulk_copy_g2s(wring + stg * C::BLK,
                       blocks + (ublk + first + kWarps * (it + C::NST)) * C::BLK, C::BLK,
@@ -525,11 +600,21 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       }
     }
     uses += count;
-    // the tail slot (index ng) belongs to warp (ng - slot0) % 4
-    if (ok && Tb > 0 && slot1 == wb && slot0 <= ng && ((ng - slot0) % kWarps) == warp) {
+    // the piece again (rebuilt rather than kept through the group loop)
+    const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+    const int b = p.b, slot0 = p.slot0, slot1 = p.slot1, wb = p.wb, unit = p.unit;
+    const int hbase = p.hbase;
+    const int Tb = p.Tb;
+    if (!C::TAIL_EARLY && my_tail && ok) {   // through the (now idle) ring
       const __half* tk = reinterpret_cast<const __half*>(
-          a.cache + g.tails_off + ((int64_t)b * g.hkv + kvh) * g.tail_bytes);
-      process_tail<D, KB, VB, G>(st, tk, tk + G * D, Tb, qsm, lane, wring);
+          a.cache + g.tails_off + ((int64_t)b * g.hkv + p.kvh) * g.tail_bytes);
+      for (int kv = 0; kv * 16 < Tb; ++kv) {
+        stage_tail_chunk<D>(wring, tk, tk + G * D, Tb, kv, lane);
+        cp_async_wait_all();
+        __syncwarp();
+        tail_chunk<D, KB, VB, G>(st, wring, Tb, kv, qsm, lane);
+        __syncwarp();   // every lane is done with this chunk before the next copy
+      }
     }
 
     // ---- merge the 4 warps (the ring is idle: every issued copy was waited on)
@@ -556,9 +641,8 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
         mo[(2 * i4) * (D + 2) + c1] = st.o[mt][2] + zl0[j];
         mo[(2 * i4 + 1) * (D + 2) + c1] = st.o[mt][3] + zl1[j];
       }
+      if (i4 == 0) mo[g8 * (D + 2) + D] = st.m;
       if (g8 == 0) {
-        mo[(2 * i4) * (D + 2) + D] = st.m[0];
-        mo[(2 * i4 + 1) * (D + 2) + D] = st.m[1];
         mo[(2 * i4) * (D + 2) + D + 1] = l0;
         mo[(2 * i4 + 1) * (D + 2) + D + 1] = l1;
       }
@@ -566,6 +650,24 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
     __syncthreads();
 
     const bool whole = (slot0 == 0 && slot1 == wb);
+    float* wts = merge + C::WTS_OFF;   // [h][4 warps] weights, then [h] max, [h] sum
+    if (warp == 0) {
+      // lane = 4h + w: warp w's share of head h
+      const int h = g8, ww = i4;
+      const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
+      const float mw = mo[D];
+      float M = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
+      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+      const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+      float Ls = f * mo[D + 1];
+      Ls += __shfl_xor_sync(0xffffffffu, Ls, 1);
+      Ls += __shfl_xor_sync(0xffffffffu, Ls, 2);
+      wts[4 * h + ww] = whole ? f / Ls : f;
+      if (ww == 0) {
+        wts[4 * kHeadsPerSlice + h] = M;
+        wts[5 * kHeadsPerSlice + h] = Ls;
+      }
+    }
     // Partial slots: a CTA holds at most two split pieces, its first (slot
     // 2k) and its last (2k + 1); pieces in between are whole units.
     const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
@@ -576,28 +678,22 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       const int kl = (int)(((last + 1) * grid - 1) / T);
       *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
+    __syncthreads();
     for (int idx = tid; idx < nh * D; idx += kThreads) {
       const int h = idx / D, c = idx % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, merge[(ww * kHeadsPerSlice + h) * (D + 2) + D]);
-      float Lsum = 0.f, O = 0.f;
-#pragma unroll
-      for (int ww = 0; ww < kWarps; ++ww) {
-        const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
-        const float f = (mo[D] == -INFINITY) ? 0.f : fast_exp2(mo[D] - M);
-        Lsum += mo[D + 1] * f;
-        O += mo[c] * f;
-      }
+      const float4 f = *reinterpret_cast<const float4*>(wts + 4 * h);
+      const float* mo = merge + h * (D + 2) + c;
+      constexpr int WS = kHeadsPerSlice * (D + 2);   // stride between the warps' areas
+      const float O = f.x * mo[0] + f.y * mo[WS] + f.z * mo[2 * WS] + f.w * mo[3 * WS];
       if (whole) {
         reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-            __float2half_rn(O / Lsum);
+            __float2half_rn(O);
       } else {
-        float* ps = partials + myslot * w.slot_floats + h * (D + 2);
+        float* ps = partials + myslot * w.slot_floats + h * (D + 4);
         ps[c] = O;
         if (c == 0) {
-          ps[D] = M;
-          ps[D + 1] = Lsum;
+          ps[D] = wts[4 * kHeadsPerSlice + h];
+          ps[D + 1] = wts[5 * kHeadsPerSlice + h];
         }
       }
     }
@@ -607,88 +703,111 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   }
 }
 
-// Merges the pieces of every unit that the decode kernel split across CTAs.
-// One block per (unit, head, 32-channel chunk); units held by one CTA were
-// written by the decode kernel itself.  Runs as a programmatic dependent
-// launch of the decode grid and waits for it before touching the partials.
-// Warp 0 turns the pieces' (max, sum) into normalized weights; each warp
-// then folds every 4th piece for the block's 32 channels (lane = channel)
-// with up to 8 loads in flight, and the warps' sums meet in shared memory.
-constexpr int kCombineChunk = 32;
-constexpr int kCombineMaxPieces = 2 * kMaxDecodeCtas;
+// Merges the pieces of every unit that the decode kernel split across CTAs;
+// units held by one CTA were written by the decode kernel itself.  Runs as a
+// programmatic dependent launch of the decode grid and waits for it before
+// touching the partials.  An item is (unit, head of its slice); `wpi` warps
+// of a 256-thread block share an item and stride over its pieces, 4 pieces
+// in flight per warp, each lane holding D/32 channels (one 16- or 8-byte
+// load per piece).  The launch picks wpi from the expected pieces per unit.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const Geom g, const WsLayout w,
-                                                           const DecodeArgs a) {
-  __shared__ float wgt[kCombineMaxPieces];
-  __shared__ float red[kWarps][32];
-  __shared__ float sinv;
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Geom g, const WsLayout w,
+                                                                  const DecodeArgs a, int wpi,
+                                                                  int heads, int n_items) {
+  constexpr int CPL = D / 32;   // channels per lane
+  __shared__ __align__(16) float red[kCombineWarps][D + 4];
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  constexpr int kChunks = D / kCombineChunk;
-  const int chunk = blockIdx.x % kChunks;
-  const int h = (blockIdx.x / kChunks) % kHeadsPerSlice;
-  const int unit = blockIdx.x / (kChunks * kHeadsPerSlice);
-  const int2 rec = *reinterpret_cast<const int2*>(a.ws + w.units_off + 8LL * unit);
-  const int npc = rec.y;
-  if (npc <= 1) return;   // whole unit: already written
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * (kCombineWarps / wpi) + warp / wpi;
+  const int wi = warp % wpi;
+  const int unit = item / heads, h = item % heads;
+  bool active = item < n_items;
+  int npc = 0, sl0 = 0;
+  if (active) {
+    const int2 rec = *reinterpret_cast<const int2*>(a.ws + w.units_off + 8LL * unit);
+    sl0 = rec.x;
+    npc = rec.y;
+  }
   const int per_seq = g.hkv * g.slices;
   const int b = unit / per_seq, uis = unit % per_seq;
   const int kvh = uis / g.slices, slice = uis % g.slices;
   const int nh = min(kHeadsPerSlice, g.gqa - slice * kHeadsPerSlice);
-  if (h >= nh) return;
-  const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t sl0 = rec.x, kf = sl0 / 2;
-  const float* partials = reinterpret_cast<const float*>(a.ws + w.partials_off) + h * (D + 2);
-  auto piece = [&](int pc) { return partials + (pc == 0 ? sl0 : 2 * (kf + pc)) * w.slot_floats; };
+  active = active && npc > 1 && h < nh;
+  const float* part = reinterpret_cast<const float*>(a.ws + w.partials_off) + h * (D + 4);
+  const int kf = sl0 / 2;
+  auto piece = [&](int pc) { return part + (int64_t)(pc == 0 ? sl0 : 2 * (kf + pc)) * w.slot_floats; };
 
-  if (warp == 0) {
-    // weights e^(m_k - M) / L, L = sum_k l_k e^(m_k - M)
+  float acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  float lsum = 0.f;
+  if (active) {
     float M = -INFINITY;
     for (int pc = lane; pc < npc; pc += 32) M = fmaxf(M, __ldcg(piece(pc) + D));
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int pc = lane; pc < npc; pc += 32) {
-      const float* ps = piece(pc);
-      const float wk = fast_exp2(__ldcg(ps + D) - M);
-      wgt[pc] = wk;
-      L += wk * __ldcg(ps + D + 1);
-    }
+    for (int p0 = wi; p0 < npc; p0 += 4 * wpi) {
+      float2 ml[4];
+      float ov[4][CPL];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) sinv = 1.0f / L;
+      for (int u = 0; u < 4; ++u) {
+        const int pc = p0 + u * wpi;
+        ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ov[u][c] = 0.f;
+        if (pc < npc) {
+          const float* ps = piece(pc);
+          ml[u] = __ldcg(reinterpret_cast<const float2*>(ps + D));
+          if constexpr (CPL == 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(ps) + lane);
+            ov[u][0] = v.x; ov[u][1] = v.y; ov[u][2] = v.z; ov[u][3] = v.w;
+          } else {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(ps) + lane);
+            ov[u][0] = v.x; ov[u][1] = v.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wk = ml[u].x == -INFINITY ? 0.f : fast_exp2(ml[u].x - M);
+        lsum += wk * ml[u].y;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] += wk * ov[u][c];
+      }
+    }
   }
-  __syncthreads();
-  const int c = chunk * kCombineChunk + lane;
-  float acc = 0.f;
-  for (int p0 = warp; p0 < npc; p0 += 8 * kWarps) {
-    float v[8];
+  if (wpi > 1) {   // uniform over the block
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int pc = p0 + u * kWarps;
-      v[u] = pc < npc ? __ldcg(piece(pc) + c) : 0.f;
-    }
+    for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = acc[c];
+    if (lane == 0) red[warp][D] = lsum;
+    __syncthreads();
+    if (wi == 0 && active) {
+      for (int ww = 1; ww < wpi; ++ww) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int pc = p0 + u * kWarps;
-      if (pc < npc) acc += wgt[pc] * v[u];
+        for (int c = 0; c < CPL; ++c) acc[c] += red[warp + ww][lane * CPL + c];
+        lsum += red[warp + ww][D];
+      }
     }
   }
-  red[warp][lane] = acc;
-  __syncthreads();
-  if (warp == 0) {
-    float o = 0.f;
-#pragma unroll
-    for (int ww = 0; ww < kWarps; ++ww) o += red[ww][lane];
-    reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-        __float2half_rn(o * sinv);
+  if (wi == 0 && active) {
+    const float inv = 1.0f / lsum;
+    const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
+    __half* o = reinterpret_cast<__half*>(a.out) + ((int64_t)b * g.hq + hbase + h) * D + lane * CPL;
+    if constexpr (CPL == 4) {
+      *reinterpret_cast<uint2*>(o) =
+          make_uint2(pack_h2(acc[0] * inv, acc[1] * inv), pack_h2(acc[2] * inv, acc[3] * inv));
+    } else {
+      *reinterpret_cast<uint32_t*>(o) = pack_h2(acc[0] * inv, acc[1] * inv);
+    }
   }
 }
 
 template <int D, int KB, int VB, int G>
-size_t smem_bytes(int n_seq) {
-  return DecCfg<D, KB, VB, G>::SMEM_FIXED + 4 * (size_t)(n_seq + 1);
+size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
+  return DecCfg<D, KB, VB, G>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
 }
 
 template <int D, int KB, int VB, int G>
@@ -697,7 +816,7 @@ cudaError_t max_ctas_t(int* out) {
   auto kern = decode_kernel<D, KB, VB, G>;
   const size_t sm = smem_bytes<D, KB, VB, G>(64);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(C::SMEM_FIXED + 4 * (kMaxSeqsDecode + 1)));
+                                       (int)smem_bytes<D, KB, VB, G>(kMaxSeqsDecode));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, sm);
@@ -722,17 +841,24 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
   static bool configured = false;   // attribute set once, before any capture
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(C::SMEM_FIXED + 4 * (kMaxSeqsDecode + 1)));
+                                         (int)smem_bytes<D, KB, VB, G>(kMaxSeqsDecode));
     if (e != cudaSuccess) return e;
     configured = true;
   }
   kern<<<grid, kThreads, sm, stream>>>(g, w, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // the combine kernel, a programmatic dependent of the decode grid
+  // the combine kernel, a programmatic dependent of the decode grid; warps
+  // per item from the expected pieces of a split unit (grid / units + 1)
+  const int units = a.n_seq * g.hkv * g.slices;
+  const int npc_est = grid / units + 1;
+  const int wpi = npc_est <= 4 ? 1 : npc_est <= 8 ? 2 : npc_est <= 16 ? 4 : 8;
+  const int heads = g.gqa < kHeadsPerSlice ? g.gqa : kHeadsPerSlice;
+  const int n_items = units * heads;
+  const int ipb = kCombineWarps / wpi;
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3((unsigned)(a.n_seq * g.hkv * g.slices * kHeadsPerSlice * (D / kCombineChunk)));
-  lc.blockDim = dim3(kThreads);
+  lc.gridDim = dim3((unsigned)((n_items + ipb - 1) / ipb));
+  lc.blockDim = dim3(kCombineThreads);
   lc.dynamicSmemBytes = 0;
   lc.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -740,7 +866,7 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, combine_kernel<D>, g, w, a);
+  return cudaLaunchKernelEx(&lc, combine_kernel<D>, g, w, a, wpi, heads, n_items);
 }
 
 }  // namespace

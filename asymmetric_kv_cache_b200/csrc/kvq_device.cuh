@@ -131,6 +131,13 @@ __device__ __forceinline__ uint32_t hfma2_b(uint32_t a, uint32_t b, uint32_t c) 
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
+// a * b - c (the negation folds into the multiply-add)
+__device__ __forceinline__ uint32_t hfma2_negc_b(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("{\n.reg .b32 t;\nneg.f16x2 t, %3;\nfma.rn.f16x2 %0, %1, %2, t;\n}"
+      : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 __device__ __forceinline__ uint32_t hmul2_b(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));

@@ -37,7 +37,7 @@ struct Geom {
 struct WsLayout {
   int64_t err_off, units_off, partials_off, total;
   int32_t units;       // split records
-  int32_t slot_floats; // floats per partial slot: heads * (d + 2)
+  int32_t slot_floats; // floats per partial slot: heads x (o[d], m, l, 2 pad)
 };
 
 inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -80,7 +80,7 @@ inline void make_geom(const kvq_config& c, Geom* g) {
 
 inline void make_ws_layout(const Geom& g, WsLayout* w) {
   w->units = g.max_seqs * g.hkv * g.slices;
-  w->slot_floats = kHeadsPerSlice * (g.d + 2);
+  w->slot_floats = kHeadsPerSlice * (g.d + 4);
   w->err_off = 0;
   w->units_off = 256;
   w->partials_off = align_up(w->units_off + 8LL * w->units, 256);
