@@ -23,7 +23,7 @@ struct kvq_cache {
   unsigned char* buf;
   size_t buf_bytes;
   std::vector<int32_t> lens;   // host mirror of the device lengths
-  int max_ctas;                // decode CTA cap (0 until first queried)
+  int max_ctas[2];             // decode CTA caps, narrow / wide (0 until queried)
 };
 
 namespace {
@@ -177,7 +177,7 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_buf, size_t bytes, 
   c->buf = static_cast<unsigned char*>(dev_buf);
   c->buf_bytes = bytes;
   c->lens.assign(cfg->max_seqs, 0);
-  c->max_ctas = 0;
+  c->max_ctas[0] = c->max_ctas[1] = 0;
   *out = c;
   return ok();
 }
@@ -268,6 +268,46 @@ int64_t choose_grid(const kvq::Geom& g, const int32_t* lens, int n_seq, int64_t 
   }
   return grid;
 }
+
+// One decode + combine pair per chunk of at most kSeqsPerLaunch sequences
+// (stream order keeps the chunks from overlapping on the workspace).
+cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
+                                 const int32_t* lens, const void* q, int q_dtype, void* out,
+                                 unsigned char* ws, int n_seq, int* max_ctas, int64_t max_grid,
+                                 const unsigned char* cache_buf, cudaStream_t stream) {
+  for (int wide = 0; wide < 2; ++wide) {
+    if (max_ctas[wide] == 0) {
+      cudaError_t e = kvq::decode_max_ctas(g, wide != 0, &max_ctas[wide]);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  int env_cap = 0;
+  if (const char* env = std::getenv("KVQ_DECODE_MAX_CTAS")) env_cap = std::atoi(env);
+  const int64_t qrow = (int64_t)g.hq * g.d * (q_dtype == KVQ_FP32 ? 4 : 2);
+  const int64_t orow = (int64_t)g.hq * g.d * 2;
+  for (int s0 = 0; s0 < n_seq; s0 += kvq::kSeqsPerLaunch) {
+    const int ns = std::min(kvq::kSeqsPerLaunch, n_seq - s0);
+    // wide CTAs (one per SM) while there are at most as many units as SMs
+    const bool wide = (int64_t)ns * g.hkv * g.slices <= max_ctas[1];
+    int cap = max_ctas[wide ? 1 : 0];
+    if (env_cap > 0) cap = std::min(cap, env_cap);
+    int64_t slots = 0;
+    for (int b = s0; b < s0 + ns; ++b)
+      slots += (int64_t)g.hkv * g.slices * (lens[b] / g.G + (lens[b] % g.G ? 1 : 0));
+    const int64_t grid = std::min(max_grid, choose_grid(g, lens + s0, ns, slots, cap));
+    kvq::DecodeArgs a;
+    a.cache = cache_buf;
+    a.q = static_cast<const unsigned char*>(q) + s0 * qrow;
+    a.q_dtype = q_dtype;
+    a.out = static_cast<unsigned char*>(out) + s0 * orow;
+    a.ws = ws;
+    a.n_seq = ns;
+    a.seq0 = s0;
+    cudaError_t e = kvq::launch_decode(g, w, a, (int)grid, wide, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 }  // namespace
 
 kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* out,
@@ -288,30 +328,12 @@ kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype, void* 
     return fail(KVQ_ERR_BUFFER_TOO_SMALL, "workspace has %zu bytes, needs %lld", ws_bytes,
                 (long long)cache->ws.total);
   const kvq::Geom& g = cache->geom;
-  int64_t slots = 0;
-  for (int b = 0; b < n_seq; ++b) {
-    const int L = cache->lens[b];
-    if (L <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
-    slots += (int64_t)g.hkv * g.slices * (L / g.G + (L % g.G ? 1 : 0));
-  }
-  if (cache->max_ctas == 0) {
-    cudaError_t e = kvq::decode_max_ctas(g, &cache->max_ctas);
-    if (e != cudaSuccess) return cuda_fail(e, "decode occupancy query");
-  }
-  int cap = cache->max_ctas;
-  if (const char* env = std::getenv("KVQ_DECODE_MAX_CTAS")) {
-    const int v = std::atoi(env);
-    if (v > 0) cap = std::min(cap, v);
-  }
-  const int grid = (int)choose_grid(g, cache->lens.data(), n_seq, slots, cap);
-  kvq::DecodeArgs a;
-  a.cache = cache->buf;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.out = out;
-  a.ws = static_cast<unsigned char*>(workspace);
-  a.n_seq = n_seq;
-  cudaError_t e = kvq::launch_decode(g, cache->ws, a, grid, (cudaStream_t)stream);
+  for (int b = 0; b < n_seq; ++b)
+    if (cache->lens[b] <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
+  cudaError_t e = launch_decode_chunks(g, cache->ws, cache->lens.data(), q, q_dtype, out,
+                                       static_cast<unsigned char*>(workspace), n_seq,
+                                       cache->max_ctas, kvq::kMaxDecodeCtas, cache->buf,
+                                       (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }
@@ -330,12 +352,8 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
   if (s != KVQ_OK) return s;
   if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_ERR_ALIGN, "q and out must be 16-byte aligned");
   const kvq::Geom& g = cache->geom;
-  int64_t slots = 0;
-  for (int b = 0; b < n_seq; ++b) {
-    const int L = cache->lens[b];
-    if (L <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
-    slots += (int64_t)g.hkv * g.slices * (L / g.G + (L % g.G ? 1 : 0));
-  }
+  for (int b = 0; b < n_seq; ++b)
+    if (cache->lens[b] <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
   // The fixed scratch holds [error word | per-unit split records | two
   // partial slots per CTA]; the CTA count is lowered until the partials fit.
   kvq::WsLayout w = cache->ws;
@@ -346,28 +364,18 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
                 "kvq_decode_noalloc: %d (sequence, kv head, head slice) units need more than the "
                 "%lld-byte fixed scratch; use kvq_decode with a workspace",
                 w.units, (long long)kvq::kNoAllocScratchBytes);
-  if (cache->max_ctas == 0) {
-    cudaError_t e = kvq::decode_max_ctas(g, &cache->max_ctas);
-    if (e != cudaSuccess) return cuda_fail(e, "decode occupancy query");
-  }
-  int64_t grid = choose_grid(g, cache->lens.data(), n_seq, slots, cache->max_ctas);
-  grid = std::min<int64_t>(grid, room / slot_bytes);
+  const int64_t max_grid = std::min<int64_t>(kvq::kMaxDecodeCtas, room / slot_bytes);
   void* scratch = nullptr;
   cudaError_t e = kvq::noalloc_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed decode scratch");
   // the error word must start at zero; the array keeps whatever the previous
-  // call left (the split records are rewritten by every call)
+  // call left (the split records are rewritten by every launch)
   e = cudaMemsetAsync(scratch, 0, (size_t)w.partials_off, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed decode scratch");
-  w.total = w.partials_off + grid * slot_bytes;
-  kvq::DecodeArgs a;
-  a.cache = cache->buf;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.out = out;
-  a.ws = static_cast<unsigned char*>(scratch);
-  a.n_seq = n_seq;
-  e = kvq::launch_decode(g, w, a, (int)grid, (cudaStream_t)stream);
+  w.total = w.partials_off + max_grid * slot_bytes;
+  e = launch_decode_chunks(g, w, cache->lens.data(), q, q_dtype, out,
+                           static_cast<unsigned char*>(scratch), n_seq, cache->max_ctas, max_grid,
+                           cache->buf, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }

@@ -12,11 +12,13 @@
 // heads).  A unit's work is a row of slots: one per key group plus one for
 // the fp16 tail.  All units' slots form one sequence that is cut into
 // `gridDim.x` equal ranges, one per CTA (a stream-K split: every CTA gets the
-// same number of slots whatever the lengths are).  Inside a CTA the 4 warps
-// take the slots of each unit round-robin, each with its own online softmax,
-// and merge through shared memory at the end of the unit's piece.  A unit
-// cut by CTA boundaries writes per-piece partials (m, l, o); the last CTA to
-// finish it (atomic ticket, no waiting) merges them and writes the output.
+// same number of slots whatever the lengths are); the grid is one CTA per SM.
+// Inside a CTA the 12-16 warps claim the groups of the current unit piece
+// one at a time from a shared counter (so warps that the schedulers favour
+// simply take more groups and all finish together), each with its own
+// online softmax, and merge through shared memory at the end of the piece.
+// A unit cut by CTA boundaries writes per-piece partials (m, l, o) that the
+// combine kernel merges.
 //
 // Per group (one 32/64-token slot) a warp:
 //   * waits for the group block, brought into its own shared-memory ring by
@@ -47,8 +49,6 @@
 namespace kvq {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Staging area of the fp16 tail (T tokens, 0 < T < G) of one (sequence, kv
@@ -64,7 +64,7 @@ struct TailStage {
   static constexpr int BYTES = VOFF + 8 * VROW;
 };
 
-template <int D, int KB, int VB, int G>
+template <int D, int KB, int VB, int G, bool WIDE = true>
 struct DecCfg {
   static constexpr int KT = D / 16;   // 16-channel k-tiles of q.k
   static constexpr int NT = G / 8;    // 8-token n-tiles of q.k
@@ -82,15 +82,21 @@ struct DecCfg {
   static constexpr int SEC_VSCALE = SEC_VCODES + G * D * VB / 8;
   static constexpr int SEC_VMIN = SEC_VSCALE + 2 * G * J;
   static constexpr int BLK = SEC_VMIN + 2 * G * J;
+  // Wide: one CTA per SM - 16 warps (128 registers each) for blocks up to
+  // 4 KB, 12 (up to 168 registers) up to 7.5 KB, 8 above, so that the
+  // 2-stage rings fit shared memory - for calls whose units are at most one
+  // per SM, so that a CTA meets at most two unit pieces.  Narrow: 4 warps,
+  // 4 CTAs per SM (3 above 4 KB blocks), for calls with more units, whose
+  // CTAs cross many unit boundaries: the prologue and merge of one CTA's
+  // piece then overlap the other CTAs' groups.
+  static constexpr int NW = !WIDE ? 4 : (BLK <= 4096) ? 16 : (BLK <= 7680) ? 12 : 8;
+  static constexpr int THREADS = NW * 32;
+  static constexpr int MIN_BLOCKS = WIDE ? 1 : (BLK <= 4096) ? 4 : 3;
   // Ring stages per warp.  Two keep more bytes in flight than the HBM
-  // latency needs at 4 CTAs per SM; deeper rings only lengthen the queue
-  // that every other request (the query, the next unit's first blocks)
-  // waits behind.
+  // latency needs; deeper rings only lengthen the queue that every other
+  // request (the query, the next unit's first blocks) waits behind.
   static constexpr int NST = 2;
-  // resident CTAs per SM the register budget aims at (shared memory allows
-  // four CTAs with blocks up to 4 KB, three otherwise)
-  static constexpr int MIN_BLOCKS = (BLK <= 4096) ? 4 : 3;
-  static constexpr int RING = kWarps * NST * BLK;
+  static constexpr int RING = NW * NST * BLK;
   // query fragments of the current unit, shared by the CTA's warps:
   // [kt][lane][4 words] = {hi v0, lo v0, hi v1, lo v1}.  The raw query rows
   // of the unit (<= 8 heads x D, fp32 at most) land here first by a bulk
@@ -99,27 +105,34 @@ struct DecCfg {
   static constexpr int QA_BYTES = KT * 32 * 16;
   static_assert(kHeadsPerSlice * D * 4 <= QA_BYTES, "raw query rows fit the fragment area");
   // merge area (in the idle ring between pieces): the warps' (o, m, l) per
-  // head, then the per-head weights of the 4 warps, the max and the sum
-  static constexpr int MERGE_FLOATS = kWarps * kHeadsPerSlice * (D + 2);
+  // head, then the per-head weights of the NW warps, the max and the sum
+  static constexpr int MERGE_FLOATS = NW * kHeadsPerSlice * (D + 2);
   static constexpr int WTS_OFF = MERGE_FLOATS;
-  static_assert((MERGE_FLOATS + 6 * kHeadsPerSlice) * 4 <= RING, "merge area must fit in the ring");
-  // The tail (< G tokens, G/16 chunks of 16).  For 32-token groups the
-  // whole tail gets an area of its own: it is staged when the piece starts
-  // and processed first, its copy latency hidden behind the prologue.  For
-  // larger groups it goes through the tail warp's ring, after its groups.
+  static_assert((MERGE_FLOATS + (NW + 2) * kHeadsPerSlice) * 4 <= RING,
+                "merge area must fit in the ring");
+  // The tail (< G tokens, G/16 chunks of 16): chunk kv belongs to warp kv,
+  // which stages it when the piece starts (its copy latency hidden behind
+  // the query's) and processes it before claiming groups.  For 32-token
+  // groups the chunks get an area of their own, for larger ones they go
+  // through the warp's ring, which then starts its group copies late.
   static constexpr int TAIL_CHUNKS = G / 16;
   static constexpr bool TAIL_EARLY = (G == 32);
   static_assert(TAIL_EARLY || TailStage<D>::BYTES <= NST * BLK, "tail chunk fits a warp's ring");
+  static_assert(TAIL_CHUNKS <= NW, "a warp per tail chunk");
   static constexpr int TAIL_OFF = QA_OFF + QA_BYTES;
   static constexpr int BAR_OFF = TAIL_OFF + (TAIL_EARLY ? TAIL_CHUNKS * TailStage<D>::BYTES : 0);
-  static constexpr int SMEM_FIXED = BAR_OFF + (kWarps * NST + 1) * 8 + 56;
+  static constexpr int SMEM_FIXED = BAR_OFF + (NW * NST + 1) * 8 + 56;
 };
 
-template <int D, int KB, int VB, int G>
+// PK (packed): the GQA group has at most 4 heads, and the q.k tiles run
+// transposed - rows 16 tokens, columns 4 heads' high parts then their low
+// parts - so that no tile row or column is idle.
+template <int D, int KB, int VB, int G, bool PK = false>
 struct WarpState {
   float o[D / 16][4];   // O^T: (channel 16mt + g, heads 2i, 2i+1), then channel + 8
   float z[4];           // rows: value-min terms (j < J) and sum p (row J); cols heads
-  float m;              // running max of head lane/4, log2 domain
+  float m[PK ? 2 : 1];  // running max, log2 domain: head lane/4, or (PK) heads
+                        // 2(i&1), 2(i&1)+1
 };
 
 // Query fragments of head g = lane/4 (zeros for a padding head), channels
@@ -184,11 +197,11 @@ __device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, floa
   for (int nt = 1; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s[nt][0], s[nt][1]));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));   // the 4 lanes of head g
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const float n = fmaxf(st.m, mx);
-  if (__any_sync(0xffffffffu, n > st.m)) {
+  const float n = fmaxf(st.m[0], mx);
+  if (__any_sync(0xffffffffu, n > st.m[0])) {
     // every head gets its first logits in the same call: uniform branch
-    if (st.m != -INFINITY) {   // accumulators hold data: rescale them
-      const float al = fast_exp2(st.m - n);
+    if (st.m[0] != -INFINITY) {   // accumulators hold data: rescale them
+      const float al = fast_exp2(st.m[0] - n);
       const float a0 = __shfl_sync(0xffffffffu, al, 8 * i4);
       const float a1 = __shfl_sync(0xffffffffu, al, 8 * i4 + 4);
 #pragma unroll
@@ -203,11 +216,56 @@ __device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, floa
       st.z[2] *= a0;
       st.z[3] *= a1;
     }
-    st.m = n;
+    st.m[0] = n;
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
-    pt[nt] = pack_h2(fast_exp2(s[nt][0] - st.m), fast_exp2(s[nt][1] - st.m));
+    pt[nt] = pack_h2(fast_exp2(s[nt][0] - st.m[0]), fast_exp2(s[nt][1] - st.m[0]));
+}
+
+// The value side of a group (O^T += V^T (p s_v), Z += [z_v; 1]^T p), shared
+// by both layouts: pt[kv] = B fragments of 16 tokens.
+template <int D, int KB, int VB, int G, bool PK>
+__device__ __forceinline__ void value_side(WarpState<D, KB, VB, G, PK>& st,
+                                           const unsigned char* __restrict__ sp,
+                                           const uint32_t (&pt)[G / 16][2], int lane) {
+  using C = DecCfg<D, KB, VB, G>;
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
+  const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
+  const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
+  // rows of the Z tile: row g8 < J takes its group's value mins, row J is (1, 1)
+  const int zrow = g8 < C::J ? g8 : 0;
+  const uint32_t zsel = g8 < C::J ? 0xFFFFFFFFu : 0u;
+  const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
+  static_for<C::KV>([&](auto kv_) {
+    constexpr int kv = decltype(kv_)::value;
+    const uint32_t bp0 = pt[kv][0], bp1 = pt[kv][1];
+    const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
+    mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
+
+    uint32_t sw[2 * C::J];
+    lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
+    uint32_t bs[C::J][2];
+#pragma unroll
+    for (int j = 0; j < C::J; ++j) {
+      bs[j][0] = hmul2_b(bp0, sw[2 * j]);
+      bs[j][1] = hmul2_b(bp1, sw[2 * j + 1]);
+    }
+    uint32_t vw[C::LWV];
+    lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
+    static_for<C::MT>([&](auto mt_) {
+      constexpr int mt = decltype(mt_)::value;
+      constexpr int TPW = C::FV / 4;     // channel tiles per word
+      constexpr int wd = mt / TPW, u = mt % TPW;
+      constexpr int j = (16 * mt) / G;
+      const uint32_t a0 = unpack_pair<VB, 2 * u>(vw[wd]);
+      const uint32_t a1 = unpack_pair<VB, 2 * u + 1>(vw[wd]);
+      const uint32_t a2 = unpack_pair<VB, 2 * u + C::FV / 2>(vw[wd]);
+      const uint32_t a3 = unpack_pair<VB, 2 * u + 1 + C::FV / 2>(vw[wd]);
+      mma16816(st.o[mt], a0, a1, a2, a3, bs[j][0], bs[j][1]);
+    });
+  });
 }
 
 // One quantized group from the shared-memory stage `sp`.
@@ -284,45 +342,10 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
     s[nt][1] = (acc[nt][1] + acc[nt][3]) + bias;
   }
 
-  uint32_t pt[NT];
-  softmax_update<D, NT, KB, VB, G>(st, s, pt, lane & 3);
-
-  // O^T += V^T (p * s_v); Z += [z_v; 1]^T p
-  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
-  const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
-  const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
-  // rows of the Z tile: row g8 < J takes its group's value mins, row J is (1, 1)
-  const int zrow = g8 < C::J ? g8 : 0;
-  const uint32_t zsel = g8 < C::J ? 0xFFFFFFFFu : 0u;
-  const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
-  static_for<C::KV>([&](auto kv_) {
-    constexpr int kv = decltype(kv_)::value;
-    const uint32_t bp0 = pt[2 * kv], bp1 = pt[2 * kv + 1];
-    const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
-    mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
-
-    uint32_t sw[2 * C::J];
-    lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
-    uint32_t bs[C::J][2];
-#pragma unroll
-    for (int j = 0; j < C::J; ++j) {
-      bs[j][0] = hmul2_b(bp0, sw[2 * j]);
-      bs[j][1] = hmul2_b(bp1, sw[2 * j + 1]);
-    }
-    uint32_t vw[C::LWV];
-    lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
-    static_for<C::MT>([&](auto mt_) {
-      constexpr int mt = decltype(mt_)::value;
-      constexpr int TPW = C::FV / 4;     // channel tiles per word
-      constexpr int wd = mt / TPW, u = mt % TPW;
-      constexpr int j = (16 * mt) / G;
-      const uint32_t a0 = unpack_pair<VB, 2 * u>(vw[wd]);
-      const uint32_t a1 = unpack_pair<VB, 2 * u + 1>(vw[wd]);
-      const uint32_t a2 = unpack_pair<VB, 2 * u + C::FV / 2>(vw[wd]);
-      const uint32_t a3 = unpack_pair<VB, 2 * u + 1 + C::FV / 2>(vw[wd]);
-      mma16816(st.o[mt], a0, a1, a2, a3, bs[j][0], bs[j][1]);
-    });
-  });
+  uint32_t pt[G / 16][2];   // B fragments of the value product, 16 tokens each
+  softmax_update<D, NT, KB, VB, G>(st, s, *reinterpret_cast<uint32_t(*)[NT]>(&pt[0][0]),
+                                   lane & 3);
+  value_side<D, KB, VB, G, false>(st, sp, pt, lane);
 }
 
 // Issue the cp.async copies of tail chunk kv (16 tokens: key rows and
@@ -396,6 +419,226 @@ __device__ __forceinline__ void tail_chunk(WarpState<D, KB, VB, G>& st,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Packed variant (GQA group of at most 4 heads).
+//
+// S^T = codes q'^T on m16n8k16 tiles: rows = 16 tokens (two 8-token code
+// tiles), columns n = heads 0-3 with q' rounded to fp16 (n < 4) and the
+// rounding residual of the same heads (n >= 4).  Lane (g, i) then holds the
+// B operand of column g, so each lane computes either a high or a low part:
+// its query words (load_query_pk) are y = q_hi and x = (low lane ? q_lo : 0),
+// and with f = (low lane ? 1 : 0),
+//   h = y s,  B = x s + (y s - f h)
+// gives h on high lanes and the exact residual of h on low lanes with the
+// same instructions.  The two halves of a logit meet with one shuffle
+// (lane i and i ^ 2 hold columns n and n + 4).
+
+template <int D>
+__device__ __forceinline__ void load_query_pk(int dtype, int nh, bool ok, int lane,
+                                              uint4* __restrict__ qs) {
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const int hh = g8 & 3;
+  const bool low = g8 >= 4;
+  const bool valid = ok && hh < nh;
+  const float sc = kLog2e * rsqrtf((float)D);
+  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
+  float2 x[D / 16][2];
+#pragma unroll
+  for (int kt = 0; kt < D / 16; ++kt) {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int idx = hh * D + 16 * kt + 8 * v + 2 * i4;
+      float2 f = make_float2(0.f, 0.f);
+      if (valid) {
+        if (dtype == KVQ_FP16) {
+          f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
+        } else if (dtype == KVQ_BF16) {
+          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
+        } else {
+          f = *reinterpret_cast<const float2*>(raw + 4 * idx);
+        }
+      }
+      x[kt][v] = f;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int kt = 0; kt < D / 16; ++kt) {
+    uint32_t w[4];
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const float x0 = x[kt][v].x * sc, x1 = x[kt][v].y * sc;
+      const __half2 h = __floats2half2_rn(x0, x1);
+      const float2 hf = __half22float2(h);
+      w[2 * v] = h2_as_u32(h);
+      w[2 * v + 1] = low ? pack_h2(x0 - hf.x, x1 - hf.y) : 0u;
+    }
+    qs[kt * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Online softmax in the S^T layout: s[mt] = {(token g, head 2i'), (g, 2i'+1),
+// (g+8, 2i'), (g+8, 2i'+1)}, i' = i & 1 (lanes i and i ^ 2 agree).  P goes
+// through movmatrix into the B fragments of the value product; its columns
+// 4-7 repeat heads 0-3 and are never read back.
+template <int D, int NM, int KB, int VB, int G>
+__device__ __forceinline__ void softmax_pk(WarpState<D, KB, VB, G, true>& st, float (&s)[NM][4],
+                                           uint32_t (&pt)[NM][2]) {
+  float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
+#pragma unroll
+  for (int mt = 1; mt < NM; ++mt) {
+    mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+    mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
+  }
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {   // across the 8 token rows (lane bits 2-4)
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float n0 = fmaxf(st.m[0], mx0), n1 = fmaxf(st.m[1], mx1);
+  if (__any_sync(0xffffffffu, n0 > st.m[0] || n1 > st.m[1])) {
+    if (st.m[0] != -INFINITY) {   // accumulators hold data: rescale them
+      const float a0 = fast_exp2(st.m[0] - n0), a1 = fast_exp2(st.m[1] - n1);
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        st.o[mt][0] *= a0;
+        st.o[mt][1] *= a1;
+        st.o[mt][2] *= a0;
+        st.o[mt][3] *= a1;
+      }
+      st.z[0] *= a0;
+      st.z[1] *= a1;
+      st.z[2] *= a0;
+      st.z[3] *= a1;
+    }
+    st.m[0] = n0;
+    st.m[1] = n1;
+  }
+#pragma unroll
+  for (int mt = 0; mt < NM; ++mt) {
+    pt[mt][0] = movmatrix_trans(
+        pack_h2(fast_exp2(s[mt][0] - st.m[0]), fast_exp2(s[mt][1] - st.m[1])));
+    pt[mt][1] = movmatrix_trans(
+        pack_h2(fast_exp2(s[mt][2] - st.m[0]), fast_exp2(s[mt][3] - st.m[1])));
+  }
+}
+
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& st,
+                                                 const unsigned char* __restrict__ sp,
+                                                 const uint4* __restrict__ qsm, int lane) {
+  using C = DecCfg<D, KB, VB, G>;
+  constexpr int NM = G / 16;
+  constexpr int NT = G / 8;
+  constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
+  constexpr int KT_PER_CH = WCH * C::FK / 2;
+  static_assert(C::KT % KT_PER_CH == 0, "k-steps split evenly into code chunks");
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const uint32_t f1 = g8 >= 4 ? 0x3C003C00u : 0u;    // (1, 1) on low lanes
+  const uint32_t nf1 = g8 >= 4 ? 0u : 0x3C003C00u;   // (1, 1) on high lanes
+  const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
+  const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
+  const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
+  constexpr uint32_t kH2Neg1024 = 0xE400E400u;
+
+  float acc[NM][4];
+#pragma unroll
+  for (int mt = 0; mt < NM; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float bacc[4] = {0.f, 0.f, 0.f, 0.f};   // key-min bias minus the code offset, per column
+  static_for<C::KT / KT_PER_CH>([&](auto ch_) {
+    constexpr int ch = decltype(ch_)::value;
+    uint32_t kw[NT][WCH];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      lds_words<WCH>(kcw + (nt * 32 + lane) * C::LWK + ch * WCH, kw[nt]);
+    static_for<KT_PER_CH>([&](auto kk_) {
+      constexpr int kt = ch * KT_PER_CH + decltype(kk_)::value;
+      constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
+      const uint2 s2 = *reinterpret_cast<const uint2*>(ksw + 2 * kt);
+      const uint2 z2 = *reinterpret_cast<const uint2*>(kzw + 2 * kt);
+      const uint4 q4 = qsm[kt * 32 + lane];   // {y v0, x v0, y v1, x v1}
+      constexpr int e0 = code_log2_mul<KB, p0 % C::FK>(), e1 = code_log2_mul<KB, p1 % C::FK>();
+      const uint32_t sm0 = e0 ? hmul2_b(s2.x, h2_pow2_neg(e0)) : s2.x;
+      const uint32_t sm1 = e1 ? hmul2_b(s2.y, h2_pow2_neg(e1)) : s2.y;
+      const uint32_t h0 = hmul2_b(q4.x, sm0), h1 = hmul2_b(q4.z, sm1);
+      const uint32_t b0 = hfma2_b(q4.y, sm0, hfma2_negc_b(q4.x, sm0, hmul2_b(h0, f1)));
+      const uint32_t b1 = hfma2_b(q4.w, sm1, hfma2_negc_b(q4.z, sm1, hmul2_b(h1, f1)));
+      // the key-min bias against the raw query part of the column,
+      // y (1 - f) + x: q_hi on high lanes, q_lo on low lanes
+      const uint32_t qb0 = hfma2_b(q4.x, nf1, q4.y), qb1 = hfma2_b(q4.z, nf1, q4.w);
+      mma16816(bacc, z2.x, z2.x, z2.y, z2.y, qb0, qb1);
+      mma16816(bacc, kH2Neg1024, kH2Neg1024, kH2Neg1024, kH2Neg1024, b0, b1);
+      static_for<NM>([&](auto mt_) {
+        constexpr int mt = decltype(mt_)::value;
+        constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
+        mma16816(acc[mt], code_offset<KB, p0 % C::FK>(kw[2 * mt][w0]),
+                 code_offset<KB, p0 % C::FK>(kw[2 * mt + 1][w0]),
+                 code_offset<KB, p1 % C::FK>(kw[2 * mt][w1]),
+                 code_offset<KB, p1 % C::FK>(kw[2 * mt + 1][w1]), b0, b1);
+      });
+    });
+  });
+  float s[NM][4];
+#pragma unroll
+  for (int mt = 0; mt < NM; ++mt) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float x = acc[mt][r] + bacc[r & 1];
+      s[mt][r] = x + __shfl_xor_sync(0xffffffffu, x, 2);   // high + low columns
+    }
+  }
+  uint32_t pt[NM][2];
+  softmax_pk<D, NM, KB, VB, G>(st, s, pt);
+  value_side<D, KB, VB, G, true>(st, sp, pt, lane);
+}
+
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void tail_chunk_pk(WarpState<D, KB, VB, G, true>& st,
+                                              const unsigned char* __restrict__ buf, int T, int kv,
+                                              const uint4* __restrict__ qsm, int lane) {
+  using C = DecCfg<D, KB, VB, G>;
+  using TS = TailStage<D>;
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const uint32_t nf = g8 >= 4 ? 0u : 0x3C003C00u;   // (1, 1) on high lanes
+  // S^T = K q^T: rows 16 tokens, columns q_hi (n < 4) / q_lo (n >= 4)
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
+  const unsigned char* k1 = k0 + 8 * TS::KROW;
+#pragma unroll
+  for (int kt = 0; kt < C::KT; ++kt) {
+    const uint4 q4 = qsm[kt * 32 + lane];
+    const uint32_t b0 = hfma2_b(q4.x, nf, q4.y), b1 = hfma2_b(q4.z, nf, q4.w);
+    mma16816(acc, *reinterpret_cast<const uint32_t*>(k0 + 32 * kt),
+             *reinterpret_cast<const uint32_t*>(k1 + 32 * kt),
+             *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16),
+             *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16), b0, b1);
+  }
+  const int t0 = 16 * kv + g8, t1 = t0 + 8;
+  float s[1][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float x = acc[r] + __shfl_xor_sync(0xffffffffu, acc[r], 2);
+    s[0][r] = ((r < 2 ? t0 : t1) < T) ? x : -INFINITY;
+  }
+  uint32_t pt[1][2];
+  softmax_pk<D, 1, KB, VB, G>(st, s, pt);
+  const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
+  mma16816(st.z, ones, 0u, ones, 0u, pt[0][0], pt[0][1]);
+  const int ta = 16 * kv + 2 * i4, tb = ta + 8;
+  const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+  const uint32_t mb = (tb + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+  const unsigned char* va = buf + TS::VOFF + i4 * TS::VROW + 4 * g8;
+  const unsigned char* vb = va + 4 * TS::VROW;
+#pragma unroll
+  for (int mt = 0; mt < C::MT; ++mt) {
+    const uint32_t a0 = *reinterpret_cast<const uint32_t*>(va + 64 * mt) & ma;
+    const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
+    const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
+    const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
+    mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
+  }
+}
+
 // Largest b in [0, n) with prefix[b] <= pos (prefix[0] = 0, increasing).
 __device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int pos) {
   int lo = 0, hi = n;
@@ -434,12 +677,16 @@ __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix
   return p;
 }
 
-template <int D, int KB, int VB, int G>
-__global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
+template <int D, int KB, int VB, int G, bool PK, bool WIDE>
+__global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
+                                  DecCfg<D, KB, VB, G, WIDE>::MIN_BLOCKS)
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
-  using C = DecCfg<D, KB, VB, G>;
+  using C = DecCfg<D, KB, VB, G, WIDE>;
+  constexpr int NW = C::NW;
+  static_assert(C::NST == 2, "the ring rotation below holds two stages");
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* ring = smem;
+  __shared__ int32_t wsum[NW];
+  __shared__ int32_t claim;   // next unclaimed group of the current piece
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint4* qsm = reinterpret_cast<uint4*>(smem + C::QA_OFF);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::SMEM_FIXED);
@@ -450,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   const int g8 = lane >> 2, i4 = lane & 3;
   const int n_seq = a.n_seq;
   const int per_seq_units = g.hkv * g.slices;
-  const int32_t* lens = reinterpret_cast<const int32_t*>(a.cache + g.lens_off);
+  const int32_t* lens = reinterpret_cast<const int32_t*>(a.cache + g.lens_off) + a.seq0;
   int32_t* err = reinterpret_cast<int32_t*>(a.ws + w.err_off);
   float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
 
@@ -460,13 +707,16 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) mbar_init(&bars[warp * C::NST + s], 1);
-    if (warp == 0) mbar_init(&bars[kWarps * C::NST], 1);   // the query copy
+    if (warp == 0) mbar_init(&bars[NW * C::NST], 1);   // the query copy
     fence_mbar_init();
   }
   // ---- slot prefix over sequences: slots(b) = units(b) * (groups + has_tail)
-  if (tid == 0) prefix[0] = 0;
+  if (tid == 0) {
+    prefix[0] = 0;
+    claim = 0;
+  }
   {
-    const int chunk = (n_seq + kThreads - 1) / kThreads;
+    const int chunk = (n_seq + C::THREADS - 1) / C::THREADS;
     const int b0 = tid * chunk, b1 = min(n_seq, b0 + chunk);
     int32_t run = 0;
     for (int bb = b0; bb < b1; ++bb) {
@@ -480,7 +730,6 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    __shared__ int32_t wsum[kWarps];
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     int32_t base = 0;
@@ -501,36 +750,34 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
   const int k = blockIdx.x;
   const int start = (int)((int64_t)k * T / grid), end = (int)((int64_t)(k + 1) * T / grid);
 
-  uint32_t uses = 0;        // ring stage uses of this warp so far
+  // The warp's 2-stage ring: `head` is the stage consumed next, bit s of
+  // `phase` the parity of stage s's next completion.
+  int head = 0;
+  uint32_t phase = 0;
   uint32_t qphase = 0;      // query copies so far (one per piece)
   bool ok = true;           // no wait has run out
-  unsigned char* wring = ring + warp * C::NST * C::BLK;
+  unsigned char* wring = smem + warp * C::NST * C::BLK;
   uint64_t* wbars = bars + warp * C::NST;
+  uint64_t* qbar = bars + NW * C::NST;
   const unsigned char* blocks = a.cache + g.blocks_off;
 
-  uint64_t* qbar = bars + kWarps * C::NST;
   for (int pos = start; pos < end;) {
-    WarpState<D, KB, VB, G> st;
+    WarpState<D, KB, VB, G, PK> st;
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
-    st.m = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < (PK ? 2 : 1); ++r) st.m[r] = -INFINITY;
 
-    int first, count, nh;
-    int64_t ublk;
-    bool my_tail;
+    int ngr, nh;         // groups in this piece, heads of the unit
+    int64_t gb;          // global block index of the piece's first group
+    bool my_tail;        // this warp owns tail chunk `warp`
     {
       const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
-      ublk = ((int64_t)p.b * g.hkv + p.kvh) * g.max_groups;
+      gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
+      ngr = max(0, min(p.slot1, p.ng) - p.slot0);
       nh = p.nh;
-      // this warp's group slots: slot0 + warp + 4k below min(slot1, ng);
-      // the tail slot (index ng), if in this piece, belongs to warp
-      // (ng - slot0) % 4
-      const int gend = min(p.slot1, p.ng);
-      first = p.slot0 + warp;
-      count = (ok && first < gend) ? (gend - first + kWarps - 1) / kWarps : 0;
-      my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng &&
-                ((p.ng - p.slot0) % kWarps) == warp;
+      my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng && warp * 16 < p.Tb;
       // the unit's raw query rows first, so that they are not queued behind
       // the group blocks
       if (tid == 0) {
@@ -543,83 +790,89 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
                           ((int64_t)p.b * g.hq + p.hbase) * D * esz,
                       qbytes, qbar);
       }
-      if (lane == 0) {
-        for (int s = 0; s < min(C::NST, count); ++s) {
-          const uint32_t u = uses + s;
-          const int stg = u % C::NST;
+      if (my_tail) {
+        const __half* tk = reinterpret_cast<const __half*>(
+            a.cache + g.tails_off + ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.tail_bytes);
+        stage_tail_chunk<D>(C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES
+                                          : wring,
+                            tk, tk + G * D, p.Tb, warp, lane);
+      }
+    }
+    // Claim a group (lane 0) and start its copy into stage `stg`; -1 once
+    // the piece has none left.
+    auto claim_into = [&](int stg) -> int {
+      int gi = -1;
+      if (lane == 0 && ok) {
+        const int c = atomicAdd(&claim, 1);
+        if (c < ngr) {
+          gi = c;
           mbar_arrive_expect_tx(&wbars[stg], C::BLK);
-          bulk_copy_g2s(wring + stg * C::BLK, blocks + (ublk + first + kWarps * s) * C::BLK,
-                        C::BLK, &wbars[stg]);
+          bulk_copy_g2s(wring + stg * C::BLK, blocks + (gb + c) * C::BLK, C::BLK, &wbars[stg]);
         }
       }
-      if (C::TAIL_EARLY && my_tail) {
-        const __half* tk = reinterpret_cast<const __half*>(
-            a.cache + g.tails_off + ((int64_t)p.b * g.hkv + p.kvh) * g.tail_bytes);
-        for (int kv = 0; kv * 16 < p.Tb; ++kv)
-          stage_tail_chunk<D>(smem + C::TAIL_OFF + kv * TailStage<D>::BYTES, tk, tk + G * D,
-                              p.Tb, kv, lane);
-      }
+      return __shfl_sync(0xffffffffu, gi, 0);
+    };
+    // the ring's two items: cur in stage head, nxt in stage head ^ 1
+    int cur = -1, nxt = -1;
+    if (!(my_tail && !C::TAIL_EARLY)) {   // a ring that stages a tail starts later
+      cur = claim_into(head);
+      nxt = cur >= 0 ? claim_into(head ^ 1) : -1;
     }
     // while the blocks fly, warp 0 turns the query rows into fragments
     if (warp == 0) {
       bool got = mbar_wait_bounded(qbar, qphase & 1);
       got = __all_sync(0xffffffffu, got);
       if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-      load_query<D>(a.q_dtype, got && g8 < nh, lane, qsm);
+      if constexpr (PK) load_query_pk<D>(a.q_dtype, nh, got, lane, qsm);
+      else load_query<D>(a.q_dtype, got && g8 < nh, lane, qsm);
     }
     ++qphase;
     __syncthreads();
-    if (C::TAIL_EARLY && my_tail) {
+    if (my_tail) {
       cp_async_wait_all();
       __syncwarp();
-      const int Tb = slen[find_seq(prefix, n_seq, pos)] % G;
-      for (int kv = 0; kv * 16 < Tb; ++kv)
-        tail_chunk<D, KB, VB, G>(st, smem + C::TAIL_OFF + kv * TailStage<D>::BYTES, Tb, kv, qsm,
-                                 lane);
+      const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+      const unsigned char* tb =
+          C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
+      if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+      else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+      if (!C::TAIL_EARLY) {   // the ring is free again: start its copies
+        __syncwarp();
+        cur = claim_into(head);
+        nxt = cur >= 0 ? claim_into(head ^ 1) : -1;
+      }
     }
-    for (int it = 0; it < count; ++it) {
-      const uint32_t u = uses + it;
-      const int stg = u % C::NST;
-      bool got = mbar_wait_bounded(&wbars[stg], (u / C::NST) & 1);
+    while (cur >= 0) {
+      bool got = mbar_wait_bounded(&wbars[head], (phase >> head) & 1);
       got = __all_sync(0xffffffffu, got);
       if (!got) {
         ok = false;
         if (lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
         break;
       }
-      process_group<D, KB, VB, G>(st, wring + stg * C::BLK, qsm, lane);
+      phase ^= 1u << head;
+      if constexpr (PK) process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+      else process_group<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
       __syncwarp();
       // refill the stage: the warp's reads of it are complete (their values
       // were consumed before __syncwarp), and a bulk copy that overwrites
-      // bytes which were only read needs no proxy fence
-      if (lane == 0 && it + C::NST < count) {
-        mbar_arrive_expect_tx(&wbars[stg], C::BLK);
-        bulk_copy_g2s(wring + stg * C::BLK,
-                      blocks + (ublk + first + kWarps * (it + C::NST)) * C::BLK, C::BLK,
-                      &wbars[stg]);
-      }
+      // bytes which were only read needs no proxy fence.  Claims come in
+      // increasing order, so once one fails every later one does.
+      const int nn = nxt >= 0 ? claim_into(head) : -1;
+      cur = nxt;
+      nxt = nn;
+      head ^= 1;
     }
-    uses += count;
+
+    // ---- merge the NW warps (the rings are idle: every issued copy was
+    // waited on, except after a failed wait)
+    fence_proxy_async_smem();
+    __syncthreads();
     // the piece again (rebuilt rather than kept through the group loop)
     const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
     const int b = p.b, slot0 = p.slot0, slot1 = p.slot1, wb = p.wb, unit = p.unit;
     const int hbase = p.hbase;
-    const int Tb = p.Tb;
-    if (!C::TAIL_EARLY && my_tail && ok) {   // through the (now idle) ring
-      const __half* tk = reinterpret_cast<const __half*>(
-          a.cache + g.tails_off + ((int64_t)b * g.hkv + p.kvh) * g.tail_bytes);
-      for (int kv = 0; kv * 16 < Tb; ++kv) {
-        stage_tail_chunk<D>(wring, tk, tk + G * D, Tb, kv, lane);
-        cp_async_wait_all();
-        __syncwarp();
-        tail_chunk<D, KB, VB, G>(st, wring, Tb, kv, qsm, lane);
-        __syncwarp();   // every lane is done with this chunk before the next copy
-      }
-    }
-
-    // ---- merge the 4 warps (the ring is idle: every issued copy was waited on)
-    fence_proxy_async_smem();
-    __syncthreads();
+    if (tid == 0) claim = 0;   // for the next piece (published by the barriers below)
     {
       float* mo = merge + (warp * kHeadsPerSlice) * (D + 2);
       // value-min terms for channel group j and heads 2*i4, 2*i4+1 live in
@@ -632,16 +885,26 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       }
       const float l0 = __shfl_sync(0xffffffffu, st.z[0], 4 * C::J + i4);
       const float l1 = __shfl_sync(0xffffffffu, st.z[1], 4 * C::J + i4);
+      // (packed: columns 4-7 repeat heads 0-3 and are skipped)
+      if (!PK || i4 < 2) {
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt) {
-        const int c0 = 16 * mt + g8, c1 = c0 + 8;
-        const int j = (16 * mt) / G;
-        mo[(2 * i4) * (D + 2) + c0] = st.o[mt][0] + zl0[j];
-        mo[(2 * i4 + 1) * (D + 2) + c0] = st.o[mt][1] + zl1[j];
-        mo[(2 * i4) * (D + 2) + c1] = st.o[mt][2] + zl0[j];
-        mo[(2 * i4 + 1) * (D + 2) + c1] = st.o[mt][3] + zl1[j];
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int c0 = 16 * mt + g8, c1 = c0 + 8;
+          const int j = (16 * mt) / G;
+          mo[(2 * i4) * (D + 2) + c0] = st.o[mt][0] + zl0[j];
+          mo[(2 * i4 + 1) * (D + 2) + c0] = st.o[mt][1] + zl1[j];
+          mo[(2 * i4) * (D + 2) + c1] = st.o[mt][2] + zl0[j];
+          mo[(2 * i4 + 1) * (D + 2) + c1] = st.o[mt][3] + zl1[j];
+        }
       }
-      if (i4 == 0) mo[g8 * (D + 2) + D] = st.m;
+      if constexpr (PK) {
+        if (g8 == 0 && i4 < 2) {
+          mo[(2 * i4) * (D + 2) + D] = st.m[0];
+          mo[(2 * i4 + 1) * (D + 2) + D] = st.m[1];
+        }
+      } else {
+        if (i4 == 0) mo[g8 * (D + 2) + D] = st.m[0];
+      }
       if (g8 == 0) {
         mo[(2 * i4) * (D + 2) + D + 1] = l0;
         mo[(2 * i4 + 1) * (D + 2) + D + 1] = l1;
@@ -650,23 +913,25 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
     __syncthreads();
 
     const bool whole = (slot0 == 0 && slot1 == wb);
-    float* wts = merge + C::WTS_OFF;   // [h][4 warps] weights, then [h] max, [h] sum
-    if (warp == 0) {
-      // lane = 4h + w: warp w's share of head h
-      const int h = g8, ww = i4;
-      const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
-      const float mw = mo[D];
-      float M = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, 1));
-      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
-      const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-      float Ls = f * mo[D + 1];
-      Ls += __shfl_xor_sync(0xffffffffu, Ls, 1);
-      Ls += __shfl_xor_sync(0xffffffffu, Ls, 2);
-      wts[4 * h + ww] = whole ? f / Ls : f;
-      if (ww == 0) {
-        wts[4 * kHeadsPerSlice + h] = M;
-        wts[5 * kHeadsPerSlice + h] = Ls;
+    // [h][NW] weights of the warps' shares, then [h] max and [h] sum
+    float* wts = merge + C::WTS_OFF;
+    if (tid < kHeadsPerSlice) {
+      const int h = tid;
+      float M = -INFINITY;
+      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, merge[(ww * kHeadsPerSlice + h) * (D + 2) + D]);
+      float Ls = 0.f;
+      for (int ww = 0; ww < NW; ++ww) {
+        const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
+        const float f = (mo[D] == -INFINITY) ? 0.f : fast_exp2(mo[D] - M);
+        wts[h * NW + ww] = f;
+        Ls += f * mo[D + 1];
       }
+      if (whole) {
+        const float inv = 1.0f / Ls;
+        for (int ww = 0; ww < NW; ++ww) wts[h * NW + ww] *= inv;
+      }
+      wts[NW * kHeadsPerSlice + h] = M;
+      wts[(NW + 1) * kHeadsPerSlice + h] = Ls;
     }
     // Partial slots: a CTA holds at most two split pieces, its first (slot
     // 2k) and its last (2k + 1); pieces in between are whole units.
@@ -679,12 +944,14 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
       *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
     __syncthreads();
-    for (int idx = tid; idx < nh * D; idx += kThreads) {
+    for (int idx = tid; idx < nh * D; idx += C::THREADS) {
       const int h = idx / D, c = idx % D;
-      const float4 f = *reinterpret_cast<const float4*>(wts + 4 * h);
+      const float* f = wts + h * NW;
       const float* mo = merge + h * (D + 2) + c;
       constexpr int WS = kHeadsPerSlice * (D + 2);   // stride between the warps' areas
-      const float O = f.x * mo[0] + f.y * mo[WS] + f.z * mo[2 * WS] + f.w * mo[3 * WS];
+      float O = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < NW; ++ww) O += f[ww] * mo[ww * WS];
       if (whole) {
         reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
             __float2half_rn(O);
@@ -692,8 +959,8 @@ __global__ void __launch_bounds__(kThreads, (DecCfg<D, KB, VB, G>::MIN_BLOCKS))
         float* ps = partials + myslot * w.slot_floats + h * (D + 4);
         ps[c] = O;
         if (c == 0) {
-          ps[D] = wts[4 * kHeadsPerSlice + h];
-          ps[D + 1] = wts[5 * kHeadsPerSlice + h];
+          ps[D] = wts[NW * kHeadsPerSlice + h];
+          ps[D + 1] = wts[(NW + 1) * kHeadsPerSlice + h];
         }
       }
     }
@@ -805,21 +1072,21 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Geom g, 
   }
 }
 
-template <int D, int KB, int VB, int G>
+template <int D, int KB, int VB, int G, bool WIDE>
 size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
-  return DecCfg<D, KB, VB, G>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
+  return DecCfg<D, KB, VB, G, WIDE>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
 }
 
-template <int D, int KB, int VB, int G>
+template <int D, int KB, int VB, int G, bool PK, bool WIDE>
 cudaError_t max_ctas_t(int* out) {
-  using C = DecCfg<D, KB, VB, G>;
-  auto kern = decode_kernel<D, KB, VB, G>;
-  const size_t sm = smem_bytes<D, KB, VB, G>(64);
+  using C = DecCfg<D, KB, VB, G, WIDE>;
+  auto kern = decode_kernel<D, KB, VB, G, PK, WIDE>;
+  const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(64);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_bytes<D, KB, VB, G>(kMaxSeqsDecode));
+                                       (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, sm);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, sm);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
@@ -830,22 +1097,22 @@ cudaError_t max_ctas_t(int* out) {
   return cudaSuccess;
 }
 
-template <int D, int KB, int VB, int G>
+template <int D, int KB, int VB, int G, bool PK, bool WIDE>
 cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
                      cudaStream_t stream) {
-  using C = DecCfg<D, KB, VB, G>;
+  using C = DecCfg<D, KB, VB, G, WIDE>;
   if (g.block_bytes != C::BLK || g.sec_vmin != C::SEC_VMIN || g.sec_kscale != C::SEC_KSCALE)
     return cudaErrorInvalidValue;
-  auto kern = decode_kernel<D, KB, VB, G>;
-  const size_t sm = smem_bytes<D, KB, VB, G>(a.n_seq);
+  auto kern = decode_kernel<D, KB, VB, G, PK, WIDE>;
+  const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(a.n_seq);
   static bool configured = false;   // attribute set once, before any capture
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<D, KB, VB, G>(kMaxSeqsDecode));
+                                         (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, kThreads, sm, stream>>>(g, w, a);
+  kern<<<grid, C::THREADS, sm, stream>>>(g, w, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // the combine kernel, a programmatic dependent of the decode grid; warps
@@ -871,37 +1138,46 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
 
 }  // namespace
 
-#define KVQ_DECODE_DISPATCH(FN, ...)                                                     \
-  do {                                                                                   \
-    if (g.d == 128 && g.kb == 4 && g.vb == 2 && g.G == 32) return FN<128, 4, 2, 32>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 2 && g.vb == 2 && g.G == 32) return FN<128, 2, 2, 32>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 4 && g.vb == 2 && g.G == 64) return FN<128, 4, 2, 64>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 2 && g.vb == 2 && g.G == 64) return FN<128, 2, 2, 64>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 4 && g.vb == 4 && g.G == 32) return FN<128, 4, 4, 32>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 2 && g.vb == 4 && g.G == 32) return FN<128, 2, 4, 32>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 4 && g.vb == 4 && g.G == 64) return FN<128, 4, 4, 64>(__VA_ARGS__); \
-    if (g.d == 128 && g.kb == 2 && g.vb == 4 && g.G == 64) return FN<128, 2, 4, 64>(__VA_ARGS__); \
-    if (g.d == 64 && g.kb == 4 && g.vb == 2 && g.G == 32) return FN<64, 4, 2, 32>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 2 && g.vb == 2 && g.G == 32) return FN<64, 2, 2, 32>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 4 && g.vb == 2 && g.G == 64) return FN<64, 4, 2, 64>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 2 && g.vb == 2 && g.G == 64) return FN<64, 2, 2, 64>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 4 && g.vb == 4 && g.G == 32) return FN<64, 4, 4, 32>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 2 && g.vb == 4 && g.G == 32) return FN<64, 2, 4, 32>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 4 && g.vb == 4 && g.G == 64) return FN<64, 4, 4, 64>(__VA_ARGS__);   \
-    if (g.d == 64 && g.kb == 2 && g.vb == 4 && g.G == 64) return FN<64, 2, 4, 64>(__VA_ARGS__);   \
-    return cudaErrorInvalidValue;                                                        \
+// One instantiation per (head dim, key bits, value bits, group), per
+// layout (packed when the GQA group has at most 4 heads) and per CTA width.
+#define KVQ_DECODE_CASE(FN, D_, KB_, VB_, G_, ...)                                     \
+  if (g.d == D_ && g.kb == KB_ && g.vb == VB_ && g.G == G_)                             \
+    return g.gqa <= 4 ? (wide ? FN<D_, KB_, VB_, G_, true, true>(__VA_ARGS__)           \
+                              : FN<D_, KB_, VB_, G_, true, false>(__VA_ARGS__))         \
+                      : (wide ? FN<D_, KB_, VB_, G_, false, true>(__VA_ARGS__)          \
+                              : FN<D_, KB_, VB_, G_, false, false>(__VA_ARGS__));
+#define KVQ_DECODE_DISPATCH(FN, ...)                                                   \
+  do {                                                                                 \
+    KVQ_DECODE_CASE(FN, 128, 4, 2, 32, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 2, 2, 32, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 4, 2, 64, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 2, 2, 64, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 4, 4, 32, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 2, 4, 32, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 4, 4, 64, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 128, 2, 4, 64, __VA_ARGS__)                                  \
+    KVQ_DECODE_CASE(FN, 64, 4, 2, 32, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 2, 2, 32, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 4, 2, 64, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 2, 2, 64, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 4, 4, 32, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 2, 4, 32, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 4, 4, 64, __VA_ARGS__)                                   \
+    KVQ_DECODE_CASE(FN, 64, 2, 4, 64, __VA_ARGS__)                                   \
+    return cudaErrorInvalidValue;                                                      \
   } while (0)
 
-cudaError_t decode_max_ctas(const Geom& g, int* max_ctas) {
+cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
   KVQ_DECODE_DISPATCH(max_ctas_t, max_ctas);
 }
 
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
-                          cudaStream_t stream) {
+                          bool wide, cudaStream_t stream) {
   KVQ_DECODE_DISPATCH(launch_t, g, w, a, grid, stream);
 }
 
 #undef KVQ_DECODE_DISPATCH
+#undef KVQ_DECODE_CASE
 
 // ---------------------------------------------------------------------------
 // Decode without a caller workspace.

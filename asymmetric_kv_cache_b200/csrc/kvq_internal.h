@@ -21,8 +21,11 @@ constexpr int kHeadsPerSlice = 8;
 // Sequences per append launch (per-sequence arguments travel as kernel
 // parameters); longer batches are split into several launches.
 constexpr int kAppendMaxSeqs = 512;
-// Sequences per decode call (the CTA-local slot prefix lives in shared memory).
+// Sequences per decode call, and per decode launch (the CTA-local slot
+// prefix and lengths live in shared memory); a call with more sequences runs
+// one decode + combine pair per chunk of kSeqsPerLaunch.
 constexpr int kMaxSeqsDecode = 8192;
+constexpr int kSeqsPerLaunch = 2048;
 
 struct Geom {
   int32_t kb, vb, G, d, hq, hkv, gqa, J, slices;
@@ -110,13 +113,15 @@ struct DecodeArgs {
   int32_t q_dtype;
   void* out;             // fp16 [n_seq][hq][d]
   unsigned char* ws;
-  int32_t n_seq;
+  int32_t n_seq;         // sequences of this launch
+  int32_t seq0;          // cache index of its first sequence (q, out start there)
 };
 
 // Resident-CTA cap of the decode kernel for this geometry on the current device.
-cudaError_t decode_max_ctas(const Geom& g, int* max_ctas);
+// wide: one 12-16 warp CTA per SM; else 4-warp CTAs, several per SM.
+cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas);
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
-                          cudaStream_t stream);
+                          bool wide, cudaStream_t stream);
 
 // Size of the fixed device scratch used by kvq_decode_noalloc, and the device
 // address of that array on the current device (looked up on first use).

@@ -189,9 +189,13 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kv
  * fp16.  workspace: device buffer of at least the workspace_bytes reported
  * by kvq_cache_required_bytes, 256-byte aligned, zero-filled before its
  * first use (kvq_workspace_init).  Calls that share a workspace must not
- * overlap on the GPU.  The call launches the split-K decode kernel and a
- * small combine kernel that merges the units split across CTAs (launched
- * as a programmatic dependent of the first).
+ * overlap on the GPU.  For each chunk of up to 2048 sequences the call
+ * launches the split-K decode kernel (one CTA per SM) and a small combine
+ * kernel that merges the units split across CTAs (launched as a
+ * programmatic dependent of the first).  Inside a CTA the warps claim key
+ * groups dynamically, so repeated calls are not bit-identical: the fp16
+ * attention weights are rounded relative to a running max that depends on
+ * the order a warp meets its groups (outputs move by ~1e-5..1e-4).
  * Errors (host side): KVQ_ERR_NULL, KVQ_ERR_ARG, KVQ_ERR_CAPACITY,
  * KVQ_ERR_EMPTY (some sequence has length 0), KVQ_ERR_DTYPE,
  * KVQ_ERR_ALIGN, KVQ_ERR_BUFFER_TOO_SMALL; KVQ_ERR_CUDA on launch failure.
