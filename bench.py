@@ -305,12 +305,13 @@ def run_ours(args, rank, world, device):
         achieved = (alg_bytes / wl.K) / (dec_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": _traffic(),
-                "kernel": "kvq decode_kernel<128,4,2,32>", "peak_kind": peak_kind,
+                "kernel": "kvq decode_kernel<128,4,2,32,packed,wide> + combine_kernel<128>",
+                "peak_kind": peak_kind,
                 "bytes_per_launch": int(alg_bytes / wl.K),
                 "avg_launch_us": round(dec_avg_ms * 1e3, 3)}
     return {
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
-        "clocks": clocks, "gpu_launches": 2 * wl.K, "wl": wl,
+        "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K,
     }
 
