@@ -111,6 +111,26 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# ranks: every rank takes the same collective steps in the same order
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time (all-reduce MAX over the default group; the
+    tensor lives on `device`: CUDA under NCCL, CPU under gloo)."""
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    tdist.barrier()
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processed the same units (weak
+    scaling), divided by the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------
 class Workload:
@@ -284,11 +304,7 @@ def run_ours(args, rank, world, device):
     clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
     if dist:
-        import torch.distributed as tdist
-        tt = torch.tensor([total_ms], device=device)
-        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-        tdist.barrier()
+        total_ms = max_over_ranks(total_ms, device)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, wl, caches, nk, nv, q, stream, device)
@@ -297,7 +313,7 @@ def run_ours(args, rank, world, device):
         if cache.workspace_status(stream) != 0:
             raise RuntimeError("decode kernel reported a failed wait")
 
-    value = kv_tokens * world / (total_ms / 1e3)
+    value = weak_scaling_value(kv_tokens, world, total_ms)
     dec_avg_ms = statistics.fmean(decode_ms) if decode_ms and elapsed_ok else None
     peak, peak_kind = _peaks()
     roof = None
