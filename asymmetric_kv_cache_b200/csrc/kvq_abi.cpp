@@ -380,6 +380,82 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
   return ok();
 }
 
+namespace {
+// Geometry of an fp16 baseline call (slots of 16 tokens; no block layout).
+kvq_status fp16_geom(int32_t n_seq, int32_t hq, int32_t hkv, int32_t d, kvq::Geom* g,
+                     kvq::WsLayout* w) {
+  if (n_seq < 1) return fail(KVQ_ERR_ARG, "n_seq %d < 1", n_seq);
+  if (n_seq > kvq::kMaxSeqsDecode)
+    return fail(KVQ_ERR_CAPACITY, "n_seq %d > %d sequences per decode call", n_seq,
+                kvq::kMaxSeqsDecode);
+  if (d != 64 && d != 128) return fail(KVQ_ERR_CONFIG, "head_dim %d not in {64, 128}", d);
+  if (hkv < 1 || hq < hkv || hq % hkv) return fail(KVQ_ERR_CONFIG, "heads %d / %d", hq, hkv);
+  *g = kvq::Geom{};
+  g->d = d;
+  g->hq = hq;
+  g->hkv = hkv;
+  g->gqa = hq / hkv;
+  g->slices = (g->gqa + kvq::kHeadsPerSlice - 1) / kvq::kHeadsPerSlice;
+  g->max_seqs = n_seq;
+  g->G = 16;
+  kvq::make_ws_layout(*g, w);
+  return KVQ_OK;
+}
+}  // namespace
+
+kvq_status kvq_fp16_workspace_bytes(int32_t n_seq, int32_t n_q_heads, int32_t n_kv_heads,
+                                    int32_t head_dim, size_t* bytes) {
+  if (!bytes) return fail(KVQ_ERR_NULL, "bytes is NULL");
+  kvq::Geom g;
+  kvq::WsLayout w;
+  kvq_status s = fp16_geom(n_seq, n_q_heads, n_kv_heads, head_dim, &g, &w);
+  if (s != KVQ_OK) return s;
+  *bytes = (size_t)w.total;
+  return ok();
+}
+
+kvq_status kvq_decode_fp16(const void* k, const void* v, const int32_t* lens, int32_t max_tokens,
+                           int32_t n_seq, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                           const void* q, kvq_dtype q_dtype, void* out, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (!k || !v || !lens || !q || !out || !workspace)
+    return fail(KVQ_ERR_NULL, "a pointer argument is NULL");
+  if (max_tokens < 1) return fail(KVQ_ERR_ARG, "max_tokens %d < 1", max_tokens);
+  kvq::Geom g;
+  kvq::WsLayout w;
+  kvq_status s = fp16_geom(n_seq, n_q_heads, n_kv_heads, head_dim, &g, &w);
+  if (s != KVQ_OK) return s;
+  s = dtype_ok(q_dtype);
+  if (s != KVQ_OK) return s;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(q, 16) || !aligned(out, 16) ||
+      !aligned(lens, 4))
+    return fail(KVQ_ERR_ALIGN, "k, v, q and out must be 16-byte aligned, lens 4-byte");
+  if (!aligned(workspace, 256)) return fail(KVQ_ERR_ALIGN, "workspace must be 256-byte aligned");
+  if ((int64_t)ws_bytes < w.total)
+    return fail(KVQ_ERR_BUFFER_TOO_SMALL, "workspace has %zu bytes, needs %lld", ws_bytes,
+                (long long)w.total);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const int64_t qrow = (int64_t)n_q_heads * head_dim * (q_dtype == KVQ_FP32 ? 4 : 2);
+  const int64_t orow = (int64_t)n_q_heads * head_dim * 2;
+  for (int s0 = 0; s0 < n_seq; s0 += kvq::kSeqsPerLaunch) {
+    kvq::DecodeArgs a;
+    a.cache = nullptr;
+    a.q = static_cast<const unsigned char*>(q) + s0 * qrow;
+    a.q_dtype = q_dtype;
+    a.out = static_cast<unsigned char*>(out) + s0 * orow;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.n_seq = std::min(kvq::kSeqsPerLaunch, n_seq - s0);
+    a.seq0 = s0;
+    e = kvq::launch_decode_fp16(g, w, a, k, v, lens, max_tokens, std::min(sms, kvq::kMaxDecodeCtas),
+                                (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "fp16 decode launch");
+  }
+  return ok();
+}
+
 size_t kvq_noalloc_scratch_bytes(void) { return (size_t)kvq::kNoAllocScratchBytes; }
 
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, void* stream) {

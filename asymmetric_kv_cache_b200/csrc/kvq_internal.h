@@ -122,6 +122,11 @@ struct DecodeArgs {
 cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas);
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
                           bool wide, cudaStream_t stream);
+// fp16 decode baseline over K, V [n_seq][Hkv][max_tokens][d] (a.seq0 and the
+// device lengths `lens` index the cache; q and out start at a.seq0).
+cudaError_t launch_decode_fp16(const Geom& g, const WsLayout& w, const DecodeArgs& a,
+                               const void* k, const void* v, const int32_t* lens,
+                               int max_tokens, int grid, cudaStream_t stream);
 
 // Size of the fixed device scratch used by kvq_decode_noalloc, and the device
 // address of that array on the current device (looked up on first use).

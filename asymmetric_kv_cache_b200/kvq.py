@@ -76,12 +76,18 @@ kvq_get_lengths = _sig("kvq_get_lengths", [_vp, _P(ctypes.c_int32), ctypes.c_int
 kvq_sync_lengths = _sig("kvq_sync_lengths", [_vp, _vp])
 kvq_decode_noalloc = _sig("kvq_decode_noalloc", [_vp, _vp, ctypes.c_int32, _vp, ctypes.c_int32, _vp])
 kvq_noalloc_scratch_bytes = _sig("kvq_noalloc_scratch_bytes", [], ctypes.c_size_t)
+kvq_fp16_workspace_bytes = _sig("kvq_fp16_workspace_bytes",
+                                [ctypes.c_int32] * 4 + [ctypes.POINTER(ctypes.c_size_t)])
+kvq_decode_fp16 = _sig("kvq_decode_fp16",
+                       [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                        ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp,
+                        ctypes.c_size_t, _vp])
 
 EXPORTED = ["kvq_status_string", "kvq_last_error", "kvq_layout_for", "kvq_cache_required_bytes",
             "kvq_cache_create", "kvq_cache_destroy", "kvq_reset", "kvq_append", "kvq_decode",
             "kvq_workspace_init", "kvq_workspace_status", "kvq_cache_config",
             "kvq_cache_layout", "kvq_get_lengths", "kvq_sync_lengths", "kvq_decode_noalloc",
-            "kvq_noalloc_scratch_bytes"]
+            "kvq_noalloc_scratch_bytes", "kvq_fp16_workspace_bytes", "kvq_decode_fp16"]
 
 
 class KvqError(RuntimeError):
@@ -255,3 +261,30 @@ class KVQCache:
     def device_lengths(self) -> torch.Tensor:
         L = self.layout
         return self.buffer[L["lens_offset"]: L["lens_offset"] + 4 * self.spec.max_seqs].view(torch.int32)
+
+
+def decode_fp16(k: torch.Tensor, v: torch.Tensor, lens: torch.Tensor, q: torch.Tensor,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """kvq_decode_fp16, the unquantized comparison kernel: k, v fp16 CUDA
+    tensors [n_seq, n_kv_heads, max_tokens, head_dim], lens int32 CUDA
+    [n_seq], q [n_seq, n_q_heads, head_dim] fp16/bf16/fp32."""
+    if k.dtype != torch.float16 or v.dtype != torch.float16 or k.shape != v.shape or k.dim() != 4:
+        raise ValueError("k and v must be fp16 [n_seq, n_kv_heads, max_tokens, head_dim]")
+    n_seq, hkv, max_tokens, d = k.shape
+    if q.dtype not in DTYPE_CODES or q.dim() != 3 or q.shape[0] != n_seq or q.shape[2] != d:
+        raise ValueError("q must be [n_seq, n_q_heads, head_dim] fp16/bf16/fp32")
+    if lens.dtype != torch.int32 or tuple(lens.shape) != (n_seq,):
+        raise ValueError("lens must be int32 [n_seq]")
+    hq = q.shape[1]
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float16, device=q.device)
+    nbytes = ctypes.c_size_t()
+    check(kvq_fp16_workspace_bytes(n_seq, hq, hkv, d, ctypes.byref(nbytes)), "kvq_fp16_workspace_bytes")
+    if workspace is None or workspace.numel() < nbytes.value:
+        workspace = torch.zeros(nbytes.value, dtype=torch.uint8, device=q.device)
+    check(kvq_decode_fp16(_dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(lens, "lens"), max_tokens,
+                          n_seq, hq, hkv, d, _dev_ptr(q, "q"), DTYPE_CODES[q.dtype],
+                          _dev_ptr(out, "out"), workspace.data_ptr(), workspace.numel(),
+                          _stream(stream)), "kvq_decode_fp16")
+    return out

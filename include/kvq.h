@@ -236,6 +236,31 @@ KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype
 KVQ_API kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype,
                                       void* out, int32_t n_seq, void* stream);
 
+/* fp16 decode baseline (comparison kernel; not part of the quantized path).
+ * The same decode attention over an unquantized fp16 cache: k and v device
+ * [n_seq][n_kv_heads][max_tokens][head_dim] fp16, 16-byte aligned; lens a
+ * DEVICE int32 array [n_seq] of lengths in [1, max_tokens] (the kernel
+ * clamps lengths to [0, max_tokens], so no access leaves the arrays; a
+ * sequence of length 0 gets an undefined output); q, out as for kvq_decode.  The
+ * pages compare the quantized cache against this unquantized baseline
+ * ("WUSH-KV" page, InnerQ abstract; FlashDecoding in the first page, §IV):
+ * 2 * head_dim * 2 bytes per token-head instead of the packed codes.  Same
+ * split-K design (stream-K over one CTA per SM, dynamic 16-token slots,
+ * fp16 high/low query on the tensor core, combine kernel).  head_dim 64 or
+ * 128, n_q_heads a multiple of n_kv_heads.  workspace: at least
+ * kvq_fp16_workspace_bytes(n_seq, ...) bytes, 256-byte aligned,
+ * zero-filled before first use.  Errors (host side): KVQ_ERR_NULL,
+ * KVQ_ERR_CONFIG (shape), KVQ_ERR_ARG, KVQ_ERR_CAPACITY (n_seq > 8192),
+ * KVQ_ERR_DTYPE, KVQ_ERR_ALIGN, KVQ_ERR_BUFFER_TOO_SMALL; KVQ_ERR_CUDA on
+ * launch failure. */
+KVQ_API kvq_status kvq_fp16_workspace_bytes(int32_t n_seq, int32_t n_q_heads, int32_t n_kv_heads,
+                                            int32_t head_dim, size_t* bytes);
+KVQ_API kvq_status kvq_decode_fp16(const void* k, const void* v, const int32_t* lens,
+                                   int32_t max_tokens, int32_t n_seq, int32_t n_q_heads,
+                                   int32_t n_kv_heads, int32_t head_dim, const void* q,
+                                   kvq_dtype q_dtype, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 /* Size in bytes of the fixed scratch array used by kvq_decode_noalloc. */
 KVQ_API size_t kvq_noalloc_scratch_bytes(void);
 

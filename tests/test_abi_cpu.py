@@ -117,3 +117,22 @@ def test_null_handle_calls(kvq):
     assert kvq.kvq_cache_destroy(None) == 0
     assert kvq.kvq_status_string(5).startswith(b"KVQ_ERR_EMPTY")
     assert kvq.kvq_status_string(0) == b"KVQ_OK"
+
+
+def test_fp16_baseline_argument_checks(kvq):
+    """The fp16 comparison entry point validates on the host (no GPU use)."""
+    import ctypes
+    n = ctypes.c_size_t()
+    assert kvq.kvq_fp16_workspace_bytes(8, 32, 8, 128, ctypes.byref(n)) == 0
+    assert n.value > 0 and n.value % 256 == 0
+    CONFIG, ARG, CAP, NULL, ALIGN, SMALL = 2, 9, 4, 1, 8, 3
+    assert kvq.kvq_fp16_workspace_bytes(8, 32, 8, 96, ctypes.byref(n)) == CONFIG
+    assert kvq.kvq_fp16_workspace_bytes(8, 30, 8, 128, ctypes.byref(n)) == CONFIG
+    assert kvq.kvq_fp16_workspace_bytes(0, 32, 8, 128, ctypes.byref(n)) == ARG
+    assert kvq.kvq_fp16_workspace_bytes(9000, 32, 8, 128, ctypes.byref(n)) == CAP
+    p = 1 << 20   # never dereferenced: every call below fails its checks first
+    assert kvq.kvq_decode_fp16(None, p, p, 64, 1, 4, 1, 64, p, 0, p, p, 1 << 30, None) == NULL
+    assert kvq.kvq_decode_fp16(p + 2, p, p, 64, 1, 4, 1, 64, p, 0, p, p, 1 << 30, None) == ALIGN
+    assert kvq.kvq_decode_fp16(p, p, p, 64, 1, 4, 1, 64, p, 0, p, p, 16, None) == SMALL
+    assert kvq.kvq_decode_fp16(p, p, p, 0, 1, 4, 1, 64, p, 0, p, p, 1 << 30, None) == ARG
+    assert kvq.kvq_decode_fp16(p, p, p, 64, 1, 4, 1, 64, p, 7, p, p, 1 << 30, None) != 0
