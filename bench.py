@@ -308,6 +308,7 @@ def run_ours(args, rank, world, device):
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, wl, caches, nk, nv, q, stream, device)
+    fp16 = run_fp16_baseline(wl, ks, vs, q, stream, device)
 
     for cache in caches:
         if cache.workspace_status(stream) != 0:
@@ -327,9 +328,47 @@ def run_ours(args, rank, world, device):
                 "avg_launch_us": round(dec_avg_ms * 1e3, 3)}
     return {
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
-        "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl,
+        "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K,
     }
+
+
+def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
+    """The unquantized comparison kernel (kvq_decode_fp16) on the same layer
+    shape: contexts of `wl.center` tokens, fp16 K/V [B, Hkv, n, d], two or
+    more copies rotated so that every decode reads HBM."""
+    import torch
+    from asymmetric_kv_cache_b200 import kvq
+    n = min(wl.center, ks.shape[1])
+    one = wl.batch * wl.hkv * n * wl.d * 2 * 2
+    copies = max(2, math.ceil(2 * L2_BYTES / one))
+    kk = torch.from_numpy(np.ascontiguousarray(ks[:, :n].transpose(0, 2, 1, 3))).to(device)
+    vv = torch.from_numpy(np.ascontiguousarray(vs[:, :n].transpose(0, 2, 1, 3))).to(device)
+    kc = [kk] + [kk.clone() for _ in range(copies - 1)]
+    vc = [vv] + [vv.clone() for _ in range(copies - 1)]
+    lens = torch.full((wl.batch,), n, dtype=torch.int32, device=device)
+    qd = torch.from_numpy(q[0]).to(device)
+    out = torch.empty_like(qd)
+    ws = None
+    with torch.cuda.stream(stream):
+        for i in range(4):
+            out = kvq.decode_fp16(kc[i % copies], vc[i % copies], lens, qd, out=out, stream=stream)
+        nb = __import__("ctypes").c_size_t()
+        kvq.kvq_fp16_workspace_bytes(wl.batch, wl.hq, wl.hkv, wl.d, __import__("ctypes").byref(nb))
+        ws = torch.zeros(nb.value, dtype=torch.uint8, device=device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(iters):
+            kvq.decode_fp16(kc[i % copies], vc[i % copies], lens, qd, out=out, workspace=ws,
+                            stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    byts = wl.batch * wl.hkv * n * wl.d * 4 + wl.batch * wl.hq * wl.d * 2
+    return {"kernel": "kvq_decode_fp16 (f16_decode_kernel<128,packed> + combine)",
+            "context": n, "bytes_per_launch": byts, "avg_launch_us": round(us, 3),
+            "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
 
 
 def run_e2e(args, wl, caches, nk, nv, q, stream, device):
@@ -534,6 +573,11 @@ def main():
                 "e2e": res["e2e"], "roofline": res["roofline"], "cpu_baseline": cb,
                 "clocks": res["clocks"], "gpu_launches": res["gpu_launches"],
                 "kv_tokens_per_step": res["kv_tokens_per_step"]}
+        fp16 = res["fp16"]
+        if fp16 and res["roofline"]:
+            fp16["quantized_decode_speedup"] = round(
+                fp16["avg_launch_us"] / res["roofline"]["avg_launch_us"], 3)
+        line["fp16_baseline"] = fp16
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as tdist
