@@ -125,6 +125,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   __half* vs = reinterpret_cast<__half*>(sm + C::SM_VS);
   __half* vz = reinterpret_cast<__half*>(sm + C::SM_VZ);
 
+  // a decode launched next as a programmatic dependent may start launching
+  // now; it waits for this grid's completion before it reads the cache
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x;
   const int task = blockIdx.x;
   const int kvh = blockIdx.y;

@@ -477,6 +477,89 @@ __device__ __forceinline__ void load_query_pk(int dtype, int nh, bool ok, int la
   }
 }
 
+// The query conversion split over NCW warps (k-tiles cw, cw + NCW, ...):
+// every converting warp reads its raw values first, the warps meet at a
+// named barrier, then they write their fragments into the same bytes.  The
+// layouts are those of load_query (PK = false) and load_query_pk (PK).
+template <int D, bool PK, int NCW>
+__device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw, int lane,
+                                              uint4* __restrict__ qs) {
+  constexpr int KT = D / 16;
+  static_assert(KT % NCW == 0, "k-tiles split evenly over the converting warps");
+  constexpr int J = KT / NCW;
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const int hh = PK ? (g8 & 3) : g8;
+  const bool low = PK && g8 >= 4;
+  const bool valid = ok && hh < nh;
+  const float sc = kLog2e * rsqrtf((float)D);
+  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
+  float2 x[J][2];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int kt = cw + j * NCW;
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int idx = hh * D + 16 * kt + 8 * v + 2 * i4;
+      float2 f = make_float2(0.f, 0.f);
+      if (valid) {
+        if (dtype == KVQ_FP16) {
+          f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
+        } else if (dtype == KVQ_BF16) {
+          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
+        } else {
+          f = *reinterpret_cast<const float2*>(raw + 4 * idx);
+        }
+      }
+      x[j][v] = f;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int kt = cw + j * NCW;
+    uint32_t wv[4];
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const float x0 = x[j][v].x * sc, x1 = x[j][v].y * sc;
+      const __half2 h = __floats2half2_rn(x0, x1);
+      const float2 hf = __half22float2(h);
+      wv[2 * v] = h2_as_u32(h);
+      const uint32_t lo = pack_h2(x0 - hf.x, x1 - hf.y);
+      wv[2 * v + 1] = PK ? (low ? lo : 0u) : lo;
+    }
+    qs[kt * 32 + lane] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  }
+}
+
+// Per-head weights of the NW warps' pieces, (h, warp) per thread: the
+// head's max M and sum L over the warps, and each warp's factor
+// 2^(m_w - M) (divided by L when the piece is the whole unit).
+template <int D, int NW>
+__device__ __forceinline__ void merge_weights(const float* __restrict__ merge,
+                                              float* __restrict__ wts, bool whole, int tid) {
+  constexpr int NWP = NW <= 4 ? 4 : NW <= 8 ? 8 : 16;   // lanes per head
+  static_assert(NW <= 16, "at most 16 warps");
+  if (tid < kHeadsPerSlice * NWP) {   // whole warps: 8 * NWP is a multiple of 32
+    const int h = tid / NWP, ww = tid % NWP;
+    const bool v = ww < NW;
+    const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
+    const float mw = v ? mo[D] : -INFINITY;
+    const float lw = v ? mo[D + 1] : 0.f;
+    float M = mw;
+#pragma unroll
+    for (int o = 1; o < NWP; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+    float Ls = f * lw;
+#pragma unroll
+    for (int o = 1; o < NWP; o <<= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (v) wts[h * NW + ww] = whole ? f / Ls : f;
+    if (ww == 0) {
+      wts[NW * kHeadsPerSlice + h] = M;
+      wts[(NW + 1) * kHeadsPerSlice + h] = Ls;
+    }
+  }
+}
+
 // Online softmax in the S^T layout: s[mt] = {(token g, head 2i'), (g, 2i'+1),
 // (g+8, 2i'), (g+8, 2i'+1)}, i' = i & 1 (lanes i and i ^ 2 agree).  P goes
 // through movmatrix into the B fragments of the value product; its columns
@@ -704,6 +787,9 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
   // the combine kernel (a programmatic dependent of this grid) may be
   // scheduled now; it waits for this grid's completion before reading
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // launched as a programmatic dependent of the previous kernel on the
+  // stream (the append, typically): nothing it writes is read before this
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) mbar_init(&bars[warp * C::NST + s], 1);
@@ -826,13 +912,15 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       cur = claim_into(head);
       nxt = cur >= 0 ? claim_into(head ^ 1) : -1;
     }
-    // while the blocks fly, warp 0 turns the query rows into fragments
-    if (warp == 0) {
-      bool got = mbar_wait_bounded(qbar, qphase & 1);
-      got = __all_sync(0xffffffffu, got);
-      if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-      if constexpr (PK) load_query_pk<D>(a.q_dtype, nh, got, lane, qsm);
-      else load_query<D>(a.q_dtype, got && g8 < nh, lane, qsm);
+    // while the blocks fly, the first warps turn the query rows into fragments
+    {
+      constexpr int NCW = (NW < D / 16) ? NW : D / 16;   // converting warps
+      if (warp < NCW) {
+        bool got = mbar_wait_bounded(qbar, qphase & 1);
+        got = __all_sync(0xffffffffu, got);
+        if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
+        convert_query<D, PK, NCW>(a.q_dtype, nh, got, warp, lane, qsm);
+      }
     }
     ++qphase;
     __syncthreads();
@@ -923,24 +1011,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     const bool whole = (slot0 == 0 && slot1 == wb);
     // [h][NW] weights of the warps' shares, then [h] max and [h] sum
     float* wts = merge + C::WTS_OFF;
-    if (tid < kHeadsPerSlice) {
-      const int h = tid;
-      float M = -INFINITY;
-      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, merge[(ww * kHeadsPerSlice + h) * (D + 2) + D]);
-      float Ls = 0.f;
-      for (int ww = 0; ww < NW; ++ww) {
-        const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
-        const float f = (mo[D] == -INFINITY) ? 0.f : fast_exp2(mo[D] - M);
-        wts[h * NW + ww] = f;
-        Ls += f * mo[D + 1];
-      }
-      if (whole) {
-        const float inv = 1.0f / Ls;
-        for (int ww = 0; ww < NW; ++ww) wts[h * NW + ww] *= inv;
-      }
-      wts[NW * kHeadsPerSlice + h] = M;
-      wts[(NW + 1) * kHeadsPerSlice + h] = Ls;
-    }
+    merge_weights<D, NW>(merge, wts, whole, tid);
     // Partial slots: a CTA holds at most two split pieces, its first (slot
     // 2k) and its last (2k + 1); pieces in between are whole units.
     const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
@@ -1122,9 +1193,22 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, C::THREADS, sm, stream>>>(g, w, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    // a programmatic dependent of the previous kernel (it waits for it
+    // before reading anything): its launch overlaps the append's tail
+    cudaLaunchConfig_t dc = {};
+    dc.gridDim = dim3((unsigned)grid);
+    dc.blockDim = dim3(C::THREADS);
+    dc.dynamicSmemBytes = sm;
+    dc.stream = stream;
+    cudaLaunchAttribute da[1];
+    da[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    da[0].val.programmaticStreamSerializationAllowed = 1;
+    dc.attrs = da;
+    dc.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&dc, kern, g, w, a);
+    if (e != cudaSuccess) return e;
+  }
   // the combine kernel, a programmatic dependent of the decode grid; warps
   // per item from the expected pieces of a split unit (grid / units + 1)
   const int units = a.n_seq * g.hkv * g.slices;
@@ -1306,6 +1390,7 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
   float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // as in decode_kernel
   if (tid == 0) {
     mbar_init(qbar, 1);
     fence_mbar_init();
@@ -1393,12 +1478,14 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
     };
     int cur = claim_into(head);
     int nxt = cur >= 0 ? claim_into(head ^ 1) : -1;
-    if (warp == 0) {
-      bool got = mbar_wait_bounded(qbar, qphase & 1);
-      got = __all_sync(0xffffffffu, got);
-      if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-      if constexpr (PK) load_query_pk<D>(a.q_dtype, nh, got, lane, qsm);
-      else load_query<D>(a.q_dtype, got && g8 < nh, lane, qsm);
+    {
+      constexpr int NCW = (NW < D / 16) ? NW : D / 16;   // converting warps
+      if (warp < NCW) {
+        bool got = mbar_wait_bounded(qbar, qphase & 1);
+        got = __all_sync(0xffffffffu, got);
+        if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
+        convert_query<D, PK, NCW>(a.q_dtype, nh, got, warp, lane, qsm);
+      }
     }
     ++qphase;
     __syncthreads();
@@ -1447,24 +1534,7 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
     __syncthreads();
     const bool whole = (s0 == 0 && s1 == wb);
     float* wts = merge + F::WTS_OFF;
-    if (tid < kHeadsPerSlice) {
-      const int h = tid;
-      float M = -INFINITY;
-      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, merge[(ww * kHeadsPerSlice + h) * (D + 2) + D]);
-      float Ls = 0.f;
-      for (int ww = 0; ww < NW; ++ww) {
-        const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
-        const float f = (mo[D] == -INFINITY) ? 0.f : fast_exp2(mo[D] - M);
-        wts[h * NW + ww] = f;
-        Ls += f * mo[D + 1];
-      }
-      if (whole) {
-        const float inv = 1.0f / Ls;
-        for (int ww = 0; ww < NW; ++ww) wts[h * NW + ww] *= inv;
-      }
-      wts[NW * kHeadsPerSlice + h] = M;
-      wts[(NW + 1) * kHeadsPerSlice + h] = Ls;
-    }
+    merge_weights<D, NW>(merge, wts, whole, tid);
     const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
     if (s0 == 0 && tid == 0) {
       const int64_t last = (int64_t)pos + wb - 1;
@@ -1517,10 +1587,20 @@ cudaError_t f16_launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a,
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, F::THREADS, f16_smem_bytes<D>(a.n_seq), stream>>>(g, w, a, kc, vc, lens,
-                                                                   max_tokens);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    cudaLaunchConfig_t dc = {};
+    dc.gridDim = dim3((unsigned)grid);
+    dc.blockDim = dim3(F::THREADS);
+    dc.dynamicSmemBytes = f16_smem_bytes<D>(a.n_seq);
+    dc.stream = stream;
+    cudaLaunchAttribute da[1];
+    da[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    da[0].val.programmaticStreamSerializationAllowed = 1;
+    dc.attrs = da;
+    dc.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&dc, kern, g, w, a, kc, vc, lens, max_tokens);
+    if (e != cudaSuccess) return e;
+  }
   const int units = a.n_seq * g.hkv * g.slices;
   const int npc_est = grid / units + 1;
   const int wpi = npc_est <= 4 ? 1 : npc_est <= 8 ? 2 : npc_est <= 16 ? 4 : 8;
