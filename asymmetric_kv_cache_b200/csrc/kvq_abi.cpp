@@ -303,6 +303,12 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     a.ws = ws;
     a.n_seq = ns;
     a.seq0 = s0;
+    // wide CTAs (one unit piece each) with few pieces per split unit: the
+    // last CTA of each unit merges them (no combine kernel).  Otherwise the
+    // combine kernel: a narrow CTA moves on to its next piece, which an
+    // in-kernel merge would delay; many pieces merge faster spread out.
+    const int64_t units = (int64_t)ns * g.hkv * g.slices;
+    a.inline_merge = (wide && (grid / units + 1) <= 4) ? 1 : 0;
     cudaError_t e = kvq::launch_decode(g, w, a, (int)grid, wide, stream);
     if (e != cudaSuccess) return e;
   }
@@ -449,6 +455,7 @@ kvq_status kvq_decode_fp16(const void* k, const void* v, const int32_t* lens, in
     a.ws = static_cast<unsigned char*>(workspace);
     a.n_seq = std::min(kvq::kSeqsPerLaunch, n_seq - s0);
     a.seq0 = s0;
+    a.inline_merge = 0;
     e = kvq::launch_decode_fp16(g, w, a, k, v, lens, max_tokens, std::min(sms, kvq::kMaxDecodeCtas),
                                 (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "fp16 decode launch");

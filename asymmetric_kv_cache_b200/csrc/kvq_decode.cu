@@ -732,6 +732,112 @@ __device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int pos) {
   return lo;
 }
 
+// The last CTA to finish a split unit merges the unit's pieces.  Every
+// piece's CTA has written its partial (o, m, l per head); the CTA's threads
+// meet at a barrier, one thread bumps the unit's ticket with an acquire-
+// release atomic at GPU scope (so the partials written before it by any
+// piece's CTA are visible to whoever sees the final count), and the CTA
+// that brings the count to the number of pieces reads every piece back
+// from L2 and writes the output.  Piece 0 is the unit's first slot's CTA
+// kf (partial slot 2kf if the unit starts its range, else 2kf + 1); pieces
+// 1.. are the first pieces of CTAs kf + 1 .. kl (slots 2k).
+template <int D, int THREADS>
+__device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
+                                               const DecodeArgs& a, int unit, int64_t p0,
+                                               int wb, int T, int grid, int b, int hbase, int nh,
+                                               float* __restrict__ scratch, int max_pieces,
+                                               int* __restrict__ flag, int tid) {
+  int32_t* tickets = reinterpret_cast<int32_t*>(a.ws + w.tickets_off);
+  const float* partials = reinterpret_cast<const float*>(a.ws + w.partials_off);
+  __syncthreads();
+  if (tid == 0) {
+    const int kf = (int)(((p0 + 1) * grid - 1) / T);
+    const int kl = (int)(((p0 + wb) * grid - 1) / T);
+    const int npc = kl - kf + 1;
+    const int old = atomic_add_acq_rel_gpu(tickets + unit, 1);
+    const bool last = old == npc - 1;
+    if (last) tickets[unit] = 0;   // every piece has counted: ready for the next call
+    flag[0] = last ? npc : 0;
+    flag[1] = kf;
+    flag[2] = ((int64_t)kf * T / grid == p0) ? 2 * kf : 2 * kf + 1;
+  }
+  __syncthreads();
+  const int npc = flag[0], kf = flag[1], s0 = flag[2];
+  if (npc == 0) return;
+  auto piece = [&](int pc, int h) {
+    return partials + (int64_t)(pc == 0 ? s0 : 2 * (kf + pc)) * w.slot_floats + h * (D + 4);
+  };
+  if (npc <= max_pieces) {
+    // (m, l) of every (piece, head) in one round of loads, then the per-head
+    // weights, then every element's pieces with all loads in flight
+    float* mlw = scratch;                              // [pc][h]: m, l
+    float* wt = scratch + 2 * kHeadsPerSlice * npc;    // [pc][h]: weight
+    for (int i = tid; i < npc * kHeadsPerSlice; i += THREADS) {
+      const int pc = i / kHeadsPerSlice, h = i % kHeadsPerSlice;
+      const float2 ml = h < nh ? __ldcg(reinterpret_cast<const float2*>(piece(pc, h) + D))
+                               : make_float2(-INFINITY, 0.f);
+      mlw[2 * i] = ml.x;
+      mlw[2 * i + 1] = ml.y;
+    }
+    __syncthreads();
+    if (tid < kHeadsPerSlice) {
+      const int h = tid;
+      float M = -INFINITY;
+      for (int pc = 0; pc < npc; ++pc) M = fmaxf(M, mlw[2 * (pc * kHeadsPerSlice + h)]);
+      float L = 0.f;
+      for (int pc = 0; pc < npc; ++pc) {
+        const float m = mlw[2 * (pc * kHeadsPerSlice + h)];
+        const float f = m == -INFINITY ? 0.f : fast_exp2(m - M);
+        wt[pc * kHeadsPerSlice + h] = f;
+        L += f * mlw[2 * (pc * kHeadsPerSlice + h) + 1];
+      }
+      const float inv = 1.0f / L;
+      for (int pc = 0; pc < npc; ++pc) wt[pc * kHeadsPerSlice + h] *= inv;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < nh * D; idx += THREADS) {
+      const int h = idx / D, c = idx % D;
+      float O = 0.f;
+      int pc = 0;
+      for (; pc + 4 <= npc; pc += 4) {
+        float x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = __ldcg(piece(pc + u, h) + c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float f = wt[(pc + u) * kHeadsPerSlice + h];
+          if (f != 0.f) O += f * x[u];
+        }
+      }
+      for (; pc < npc; ++pc) {
+        const float f = wt[pc * kHeadsPerSlice + h];
+        if (f != 0.f) O += f * __ldcg(piece(pc, h) + c);
+      }
+      reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
+          __float2half_rn(O);
+    }
+    return;
+  }
+  // more pieces than the scratch holds: an online merge per element
+  for (int idx = tid; idx < nh * D; idx += THREADS) {
+    const int h = idx / D, c = idx % D;
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    for (int pc = 0; pc < npc; ++pc) {
+      const float* ps = piece(pc, h);
+      const float m = __ldcg(ps + D);
+      if (m == -INFINITY) continue;
+      const float l = __ldcg(ps + D + 1), o = __ldcg(ps + c);
+      const float Mn = fmaxf(M, m);
+      const float sa = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn), sb = fast_exp2(m - Mn);
+      L = L * sa + l * sb;
+      O = O * sa + o * sb;
+      M = Mn;
+    }
+    reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
+        __float2half_rn(O / L);
+  }
+}
+
 // The part of unit `unit` (sequence b, kv head kvh, head slice `slice`)
 // that a CTA processes: slots [slot0, slot1) of the unit's wb slots.
 struct Piece {
@@ -770,6 +876,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int32_t wsum[NW];
   __shared__ int32_t claim;   // next unclaimed group of the current piece
+  __shared__ int32_t ticket_flag[3];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint4* qsm = reinterpret_cast<uint4*>(smem + C::QA_OFF);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::SMEM_FIXED);
@@ -1043,6 +1150,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         }
       }
     }
+    if (!whole && a.inline_merge)
+      finish_split_unit<D, C::THREADS>(g, w, a, unit, (int64_t)pos - slot0, wb, T, grid, b, hbase,
+                                       nh, merge, C::RING / (4 * 3 * kHeadsPerSlice), ticket_flag,
+                                       tid);
     fence_proxy_async_smem();   // generic accesses before the next bulk copies
     __syncthreads();            // merge area and ctl are reused by the next piece
     pos += slot1 - slot0;
@@ -1209,6 +1320,7 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
     cudaError_t e = cudaLaunchKernelEx(&dc, kern, g, w, a);
     if (e != cudaSuccess) return e;
   }
+  if (a.inline_merge) return cudaSuccess;   // split units merged in the kernel
   // the combine kernel, a programmatic dependent of the decode grid; warps
   // per item from the expected pieces of a split unit (grid / units + 1)
   const int units = a.n_seq * g.hkv * g.slices;

@@ -35,10 +35,12 @@ struct Geom {
   int64_t lens_off, counters_off, blocks_off, tails_off, tail_bytes, total_bytes;
 };
 
-// Workspace of kvq_decode: [error word | per-unit split records | partials].
-// A split record is {first partial slot, number of pieces} of one unit.
+// Workspace of kvq_decode: [error word | per-unit split records | per-unit
+// tickets | partials].  A split record is {first partial slot, number of
+// pieces} of one unit; a ticket counts the unit's finished pieces when the
+// last CTA to finish merges them (it resets the ticket to 0).
 struct WsLayout {
-  int64_t err_off, units_off, partials_off, total;
+  int64_t err_off, units_off, tickets_off, partials_off, total;
   int32_t units;       // split records
   int32_t slot_floats; // floats per partial slot: heads x (o[d], m, l, 2 pad)
 };
@@ -86,7 +88,8 @@ inline void make_ws_layout(const Geom& g, WsLayout* w) {
   w->slot_floats = kHeadsPerSlice * (g.d + 4);
   w->err_off = 0;
   w->units_off = 256;
-  w->partials_off = align_up(w->units_off + 8LL * w->units, 256);
+  w->tickets_off = align_up(w->units_off + 8LL * w->units, 256);   // zero between calls
+  w->partials_off = align_up(w->tickets_off + 4LL * w->units, 256);
   w->total = align_up(w->partials_off + 2LL * kMaxDecodeCtas * w->slot_floats * 4, 256);
 }
 
@@ -115,6 +118,7 @@ struct DecodeArgs {
   unsigned char* ws;
   int32_t n_seq;         // sequences of this launch
   int32_t seq0;          // cache index of its first sequence (q, out start there)
+  int32_t inline_merge;  // split units merged by their last CTA (no combine kernel)
 };
 
 // Resident-CTA cap of the decode kernel for this geometry on the current device.
