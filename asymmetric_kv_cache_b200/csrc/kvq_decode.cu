@@ -1046,6 +1046,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       }
     }
     while (cur >= 0) {
+      // the claim for this stage's refill goes out now: its latency hides
+      // behind the wait and the group's arithmetic
+      int nc = -1;
+      if (lane == 0 && nxt >= 0) nc = atomicAdd(&claim, 1);
       bool got = mbar_wait_bounded(&wbars[head], (phase >> head) & 1);
       got = __all_sync(0xffffffffu, got);
       if (!got) {
@@ -1061,7 +1065,13 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       // were consumed before __syncwarp), and a bulk copy that overwrites
       // bytes which were only read needs no proxy fence.  Claims come in
       // increasing order, so once one fails every later one does.
-      const int nn = nxt >= 0 ? claim_into(head) : -1;
+      int nn = -1;
+      if (lane == 0 && nc >= 0 && nc < ngr) {
+        nn = nc;
+        mbar_arrive_expect_tx(&wbars[head], C::BLK);
+        bulk_copy_g2s(wring + head * C::BLK, blocks + (gb + nc) * C::BLK, C::BLK, &wbars[head]);
+      }
+      nn = __shfl_sync(0xffffffffu, nn, 0);
       cur = nxt;
       nxt = nn;
       head ^= 1;
