@@ -38,16 +38,18 @@ struct AppCfg {
   static constexpr int VWORDS_PER_LANE = D * VB / 64;    // per 16-token tile
   static constexpr int KWORDS = G * D * KB / 32;
   static constexpr int VWORDS = G * D * VB / 32;
-  // dynamic shared memory: fp16 K and V of the group, their codes, metadata
+  // dynamic shared memory: fp16 K and V of the group, the fp16 metadata in
+  // slot order, and per key channel / per (token, value group) the fp32
+  // parameters of the code computation {z, 1/s, s}
   static constexpr int SM_K = 0;
   static constexpr int SM_V = SM_K + 2 * G * D;
-  static constexpr int SM_KC = SM_V + 2 * G * D;
-  static constexpr int SM_VC = SM_KC + G * D;
-  static constexpr int SM_KS = SM_VC + G * D;
+  static constexpr int SM_KS = SM_V + 2 * G * D;
   static constexpr int SM_KZ = SM_KS + 2 * D;
   static constexpr int SM_VS = SM_KZ + 2 * D;
   static constexpr int SM_VZ = SM_VS + 2 * G * J;
-  static constexpr int SM_TOTAL = SM_VZ + 2 * G * J;
+  static constexpr int SM_KP = (SM_VZ + 2 * G * J + 15) / 16 * 16;
+  static constexpr int SM_VP = SM_KP + 16 * D;
+  static constexpr int SM_TOTAL = SM_VP + 16 * G * J;
 };
 
 // Eight consecutive input elements (16-byte aligned) rounded to fp16
@@ -109,6 +111,37 @@ __device__ __forceinline__ int quant_code(float x, float zf, float sf, int Q) {
   return c > Q ? Q : c;
 }
 
+// Code computation in pairs (sm_100 packed fp32x2 arithmetic, IEEE round
+// to nearest per element, so each element is exactly the scalar result):
+// d = x - z (exact: both are fp16 values), t = d * (1/s) with 1/s correctly
+// rounded, rne(t) by adding 1.5 * 2^23 (whose mantissa then holds the
+// integer).  t is within 3e-6 of the correctly rounded quotient d / s used
+// by the definition, so the two round to the same integer unless d / s lies
+// within 6.1e-5 of a half-integer; such a pair is flagged and recomputed with
+// IEEE division.  z is the group minimum, so d >= 0 and the code needs no
+// lower clamp; the upper clamp to Q stays (a subnormal s is rounded coarsely,
+// and d / s can then pass Q + 1/2).  s == 0 has 1/s stored as 0: code 0.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void codes2(float x0, float x1, float z0, float z1, float r0, float r1,
+                                       uint32_t Q, uint32_t& c0, uint32_t& c1, bool& near_tie) {
+  uint64_t d, t, y, k, e;
+  const uint64_t magic = f32x2(12582912.0f, 12582912.0f);
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f32x2(x0, x1)), "l"(f32x2(z0, z1)));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(d), "l"(f32x2(r0, r1)));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(t), "l"(magic));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(k) : "l"(y), "l"(magic));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(e) : "l"(t), "l"(k));
+  c0 = min((uint32_t)y & 0xFFu, Q);
+  c1 = min((uint32_t)(y >> 32) & 0xFFu, Q);
+  // |e| >= 0.5 - 2^-14 in either half (e in [-0.5, 0.5])
+  const uint32_t a0 = (uint32_t)e & 0x7FFFFFFFu, a1 = (uint32_t)(e >> 32) & 0x7FFFFFFFu;
+  near_tie |= (a0 >= 0x3EFFF800u) | (a1 >= 0x3EFFF800u);   // 0.5 - 2048 ulp
+}
+
 template <int D, int G, int KB, int VB>
 __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char* __restrict__ cache,
                                                      const void* __restrict__ kin,
@@ -118,8 +151,6 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   extern __shared__ __align__(16) unsigned char sm[];
   __half* sk = reinterpret_cast<__half*>(sm + C::SM_K);
   __half* sv = reinterpret_cast<__half*>(sm + C::SM_V);
-  uint8_t* kc = sm + C::SM_KC;
-  uint8_t* vc = sm + C::SM_VC;
   __half* ks = reinterpret_cast<__half*>(sm + C::SM_KS);
   __half* kz = reinterpret_cast<__half*>(sm + C::SM_KZ);
   __half* vs = reinterpret_cast<__half*>(sm + C::SM_VS);
@@ -212,68 +243,126 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   }
   __syncthreads();
 
-  // ---- keys: one (scale, min) per channel over the G tokens
-  for (int c = tid; c < D; c += blockDim.x) {
-    float mn = __half2float(sk[c]), mx = mn;
-    for (int r = 1; r < G; ++r) {
-      const float x = __half2float(sk[r * D + c]);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+  // ---- statistics.  Warps 0-1: keys, two channels per thread (fp16x2
+  // min/max over the G tokens).  Warps 2-3: values, (token, group of G
+  // channels) items, 16-byte loads.  fp16 min/max of fp16 values is exact.
+  float4* kp = reinterpret_cast<float4*>(sm + C::SM_KP);   // [c]: {z, 1/s, s, -}
+  float4* vp = reinterpret_cast<float4*>(sm + C::SM_VP);   // [r * J + j]
+  if (tid < 64) {
+    const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
+    for (int cp = tid; cp < D / 2; cp += 64) {
+      __half2 mn = sk2[cp], mx = mn;
+      for (int r = 1; r < G; ++r) {
+        const __half2 x = sk2[r * (D / 2) + cp];
+        mn = __hmin2(mn, x);
+        mx = __hmax2(mx, x);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = 2 * cp + e;
+        const float mnf = e ? __high2float(mn) : __low2float(mn);
+        const float mxf = e ? __high2float(mx) : __low2float(mx);
+        const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)C::QK));
+        const __half z16 = __float2half_rn(mnf);
+        const float sf = __half2float(s16);
+        kp[c] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
+        // metadata slot i*(D/4) + 4kt + 2v + e
+        const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3, ee = c & 1;
+        const int slot = i * (D / 4) + 4 * kt + 2 * v + ee;
+        ks[slot] = s16;
+        kz[slot] = z16;
+      }
     }
-    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)C::QK));
-    const __half z16 = __float2half_rn(mn);
-    const float sf = __half2float(s16), zf = __half2float(z16);
-    for (int r = 0; r < G; ++r) kc[r * D + c] = (uint8_t)quant_code(__half2float(sk[r * D + c]), zf, sf, C::QK);
-    // metadata slot i*(D/4) + 4kt + 2v + e
-    const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3, e = c & 1;
-    const int slot = i * (D / 4) + 4 * kt + 2 * v + e;
-    ks[slot] = s16;
-    kz[slot] = z16;
-  }
-  // ---- values: one (scale, min) per (token, group of G channels)
-  for (int q = tid; q < G * C::J; q += blockDim.x) {
-    const int r = q / C::J, j = q % C::J;
-    const __half* row = sv + r * D + j * G;
-    // start each thread at a different channel to spread shared-memory banks
-    float mn = __half2float(row[r % G]), mx = mn;
-    for (int k = 1; k < G; ++k) {
-      const float x = __half2float(row[(k + r) % G]);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+  } else {
+    for (int q = tid - 64; q < G * C::J; q += 64) {
+      const int r = q / C::J, j = q % C::J;
+      const uint4* row = reinterpret_cast<const uint4*>(sv + r * D + j * G);
+      constexpr int NV = G / 8;
+      uint4 w0 = row[r % NV];
+      __half2 mn = *reinterpret_cast<__half2*>(&w0.x), mx = mn;
+#pragma unroll
+      for (int u = 0; u < NV; ++u) {
+        const uint4 w = row[(u + r) % NV];   // rotate the start: fewer bank conflicts
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const __half2 x = *reinterpret_cast<const __half2*>(&ws[h]);
+          mn = __hmin2(mn, x);
+          mx = __hmax2(mx, x);
+        }
+      }
+      const float mnf = fminf(__low2float(mn), __high2float(mn));
+      const float mxf = fmaxf(__low2float(mx), __high2float(mx));
+      const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)C::QV));
+      const __half z16 = __float2half_rn(mnf);
+      const float sf = __half2float(s16);
+      vp[q] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
+      // metadata slot ((4kv + i)*J + j)*4 + 2kh + e
+      const int kv = r >> 4, kh = (r >> 3) & 1, i = (r >> 1) & 3, e = r & 1;
+      const int slot = ((4 * kv + i) * C::J + j) * 4 + 2 * kh + e;
+      vs[slot] = s16;
+      vz[slot] = z16;
     }
-    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)C::QV));
-    const __half z16 = __float2half_rn(mn);
-    const float sf = __half2float(s16), zf = __half2float(z16);
-    for (int k = 0; k < G; ++k) {
-      const int kk = (k + r) % G;
-      vc[r * D + j * G + kk] = (uint8_t)quant_code(__half2float(row[kk]), zf, sf, C::QV);
-    }
-    // metadata slot ((4kv + i)*J + j)*4 + 2kh + e
-    const int kv = r >> 4, kh = (r >> 3) & 1, i = (r >> 1) & 3, e = r & 1;
-    const int slot = ((4 * kv + i) * C::J + j) * 4 + 2 * kh + e;
-    vs[slot] = s16;
-    vz[slot] = z16;
   }
   __syncthreads();
 
-  // ---- pack into the group block
+  // ---- codes, quantized and packed word by word into the group block
   unsigned char* blk = cache + g.blocks_off +
                        (unit * g.max_groups + (N0 / G + tau)) * (int64_t)g.block_bytes;
   uint32_t* kw = reinterpret_cast<uint32_t*>(blk + g.sec_kcodes);
-  for (int wi = tid; wi < C::KWORDS; wi += blockDim.x) {
-    const int w = wi % C::KWORDS_PER_LANE;
-    const int lane = (wi / C::KWORDS_PER_LANE) % 32;
-    const int nt = wi / (C::KWORDS_PER_LANE * 32);
-    const int t = 8 * nt + (lane >> 2), i = lane & 3;
-    uint32_t word = 0;
+  const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
+  {
+    // A thread's key words (wi = tid + 128k) share one word index w and one
+    // lane, hence one set of channels: their (z, 1/s) are loaded once.
+    static_assert(128 % C::KWORDS_PER_LANE == 0 && (128 / C::KWORDS_PER_LANE) % 32 == 0,
+                  "key words of a thread share their channels");
+    const int w = tid % C::KWORDS_PER_LANE;
+    const int lane = (tid / C::KWORDS_PER_LANE) % 32;
+    const int i = lane & 3;
+    float zk[C::FK][2], rk[C::FK][2];
 #pragma unroll
-    for (int fp = 0; fp < 32 / KB; ++fp) {
-      const int e = fp / C::FK, f = fp % C::FK;
+    for (int f = 0; f < C::FK; ++f) {
       const int p = w * C::FK + f;
-      const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i + e;
-      word |= (uint32_t)kc[t * D + c] << (KB * fp);
+      const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4 pc = kp[c + e];
+        zk[f][e] = pc.x;
+        rk[f][e] = pc.y;
+      }
     }
-    kw[wi] = word;
+    for (int wi = tid; wi < C::KWORDS; wi += blockDim.x) {
+      const int nt = wi / (C::KWORDS_PER_LANE * 32);
+      const int t = 8 * nt + (lane >> 2);
+      uint32_t word = 0;
+      bool tie = false;
+#pragma unroll
+      for (int f = 0; f < C::FK; ++f) {
+        // field f of the low half and of the high half: channels c, c + 1
+        const int p = w * C::FK + f;
+        const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+        const float2 x = __half22float2(sk2[(t * D + c) >> 1]);
+        uint32_t c0, c1;
+        codes2(x.x, x.y, zk[f][0], zk[f][1], rk[f][0], rk[f][1], C::QK, c0, c1, tie);
+        word |= ((c0 & C::QK) << (KB * f)) | ((c1 & C::QK) << (KB * (C::FK + f)));
+      }
+      if (tie) {   // rare: IEEE division for the whole word
+        word = 0;
+#pragma unroll
+        for (int f = 0; f < C::FK; ++f) {
+          const int p = w * C::FK + f;
+          const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 pc = kp[c + e];
+            const uint32_t code =
+                (uint32_t)quant_code(__half2float(sk[t * D + c + e]), pc.x, pc.z, C::QK);
+            word |= code << (KB * (e * C::FK + f));
+          }
+        }
+      }
+      kw[wi] = word;
+    }
   }
   uint32_t* vw = reinterpret_cast<uint32_t*>(blk + g.sec_vcodes);
   for (int wi = tid; wi < C::VWORDS; wi += blockDim.x) {
@@ -282,15 +371,46 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     const int kv = wi / (C::VWORDS_PER_LANE * 32);
     const int gg = lane >> 2, i = lane & 3;
     uint32_t word = 0;
+    bool tie = false;
+    // the word's channels 16 mt .. 16 mt + 15 lie in one value group j; its
+    // four tokens (kh, e) have one (z, 1/s) each
+    const int jw = (16 * (w * (C::FV / 4))) / G;
+    float4 pv[2][2];
 #pragma unroll
-    for (int fp = 0; fp < 32 / VB; ++fp) {
-      const int e = fp / C::FV, fl = fp % C::FV;
+    for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) pv[kh][e] = vp[(16 * kv + 8 * kh + 2 * i + e) * C::J + jw];
+#pragma unroll
+    for (int fl = 0; fl < C::FV; ++fl) {
+      // field fl of the low half (token t) and of the high half (token t + 1)
       const int kh = fl / (C::FV / 2), rem = fl % (C::FV / 2);
       const int u = rem >> 1, hr = rem & 1;
       const int mt = w * (C::FV / 4) + u;
       const int c = 16 * mt + 8 * hr + gg;
-      const int t = 16 * kv + 8 * kh + 2 * i + e;
-      word |= (uint32_t)vc[t * D + c] << (VB * fp);
+      const int t = 16 * kv + 8 * kh + 2 * i;
+      const float4 p0 = pv[kh][0], p1 = pv[kh][1];
+      uint32_t c0, c1;
+      codes2(__half2float(sv[t * D + c]), __half2float(sv[(t + 1) * D + c]), p0.x, p1.x, p0.y,
+             p1.y, C::QV, c0, c1, tie);
+      word |= ((c0 & C::QV) << (VB * fl)) | ((c1 & C::QV) << (VB * (C::FV + fl)));
+    }
+    if (tie) {
+      word = 0;
+#pragma unroll
+      for (int fl = 0; fl < C::FV; ++fl) {
+        const int kh = fl / (C::FV / 2), rem = fl % (C::FV / 2);
+        const int u = rem >> 1, hr = rem & 1;
+        const int mt = w * (C::FV / 4) + u;
+        const int c = 16 * mt + 8 * hr + gg;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 16 * kv + 8 * kh + 2 * i + e;
+          const float4 pc = vp[t * C::J + c / G];
+          const uint32_t code =
+              (uint32_t)quant_code(__half2float(sv[t * D + c]), pc.x, pc.z, C::QV);
+          word |= code << (VB * (e * C::FV + fl));
+        }
+      }
     }
     vw[wi] = word;
   }
