@@ -1274,6 +1274,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Geom g, 
   }
 }
 
+#include "kvq_decode_tc.cuh"
+
 template <int D, int KB, int VB, int G, bool WIDE>
 size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
   return DecCfg<D, KB, VB, G, WIDE>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
@@ -1776,8 +1778,23 @@ cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
   KVQ_DECODE_DISPATCH(max_ctas_t, max_ctas);
 }
 
+// The tcgen05 kernel (kvq_decode_tc.cuh) is opt-in: KVQ_DECODE_TC=1 selects
+// it for the shapes it covers.  Measured on B200 it is about 2x slower than
+// the mma.sync kernel on these shapes (the contraction per group is too
+// small for the tensor core to matter; unpacking and the role hand-offs
+// dominate), so the mma.sync kernel is the default.
+bool decode_tc_eligible(const Geom& g) {
+  if (!(g.d == 128 && g.G == 32 && g.vb == 2 && (g.kb == 2 || g.kb == 4) && g.gqa <= 4 &&
+        g.slices == 1))
+    return false;
+  const char* env = std::getenv("KVQ_DECODE_TC");
+  return env && env[0] == '1';
+}
+
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
                           bool wide, cudaStream_t stream) {
+  if (wide && decode_tc_eligible(g))
+    return g.kb == 4 ? launch_tc_t<4>(g, w, a, grid, stream) : launch_tc_t<2>(g, w, a, grid, stream);
   KVQ_DECODE_DISPATCH(launch_t, g, w, a, grid, stream);
 }
 
