@@ -321,6 +321,7 @@ def run_ours(args, rank, world, device):
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, wl, caches, nk, nv, q, stream, device)
     fp16 = run_fp16_baseline(wl, ks, vs, q, stream, device)
+    long_ctx = run_long_context(stream, device) if args.long_context else None
 
     for cache in caches:
         if cache.workspace_status(stream) != 0:
@@ -343,7 +344,7 @@ def run_ours(args, rank, world, device):
     return {
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
         "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
-        "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K,
+        "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K, "long_ctx": long_ctx,
     }
 
 
@@ -383,6 +384,83 @@ def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
     return {"kernel": "kvq_decode_fp16 (f16_decode_kernel<128,packed> + combine)",
             "context": n, "bytes_per_launch": byts, "avg_launch_us": round(us, 3),
             "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
+
+
+def run_long_context(stream, device, iters=100):
+    """Decode alone on the 128k-token long-context workload (batch 1, 32 q /
+    8 kv heads, d 128, K2/V2, G 32): the configuration the HBM-roofline
+    target is stated on.  Copies of the cache (> 3x L2 in total) are
+    rotated so that every decode reads HBM; CUDA events on the launch
+    stream around `iters` decodes.  The unquantized comparison kernel runs
+    the same shape (fp16 K/V, two copies)."""
+    import torch
+    from asymmetric_kv_cache_b200 import inputs, kvq
+    w = inputs.WORKLOADS["long_ctx"]()
+    n = w.lens[0]
+    spec = kvq.CacheSpec(w.k_bits, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
+                         w.batch, n)
+    G, d = w.group, w.head_dim
+    blk = G * d * (w.k_bits + w.v_bits) // 8 + 8 * d
+    byts = w.n_kv_heads * ((n // G) * blk + (n % G) * 4 * d) + w.n_q_heads * d * 2
+    copies = max(2, math.ceil(3 * L2_BYTES / byts))
+    k = torch.from_numpy(np.concatenate(w.keys)).to(device)
+    v = torch.from_numpy(np.concatenate(w.values)).to(device)
+    q = torch.from_numpy(np.ascontiguousarray(w.q, np.float16)).to(device)
+    caches = []
+    with torch.cuda.stream(stream):
+        for _ in range(copies):
+            c = kvq.KVQCache(spec)
+            c.append(k, v, w.lens, stream=stream)
+            caches.append(c)
+        out = torch.empty_like(q)
+        for i in range(2 * copies):
+            caches[i % copies].decode(q, out=out, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(iters):
+            caches[i % copies].decode(q, out=out, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    for c in caches:
+        if c.workspace_status(stream) != 0:
+            raise RuntimeError("decode kernel reported a failed wait")
+    peak, peak_kind = _peaks()
+    res = {"workload": "long_ctx", "context": n, "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv",
+           "bits": f"K{w.k_bits}/V{w.v_bits}", "group": G, "copies": copies,
+           "bytes_per_launch": int(byts), "avg_launch_us": round(us, 3),
+           "achieved_gbs": round(byts / us / 1e3, 1), "peak": peak, "peak_kind": peak_kind,
+           "frac": round(byts / us / 1e3 / peak, 4), "launches": iters,
+           "kv_tokens_per_s": round(n * iters / (e0.elapsed_time(e1) / 1e3), 1),
+           "note": "decode + combine per launch, CUDA events around the launches"}
+    del caches
+    # the unquantized kernel on the same shape
+    kk = k.view(n, w.n_kv_heads, d).transpose(0, 1).unsqueeze(0).contiguous()
+    vv = v.view(n, w.n_kv_heads, d).transpose(0, 1).unsqueeze(0).contiguous()
+    del k, v
+    kc, vc = [kk, kk.clone()], [vv, vv.clone()]
+    lens = torch.full((1,), n, dtype=torch.int32, device=device)
+    import ctypes
+    nb = ctypes.c_size_t()
+    kvq.kvq_fp16_workspace_bytes(1, w.n_q_heads, w.n_kv_heads, d, ctypes.byref(nb))
+    ws = torch.zeros(nb.value, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        for i in range(4):
+            kvq.decode_fp16(kc[i % 2], vc[i % 2], lens, q, out=out, workspace=ws, stream=stream)
+        e0.record(stream)
+        for i in range(iters):
+            kvq.decode_fp16(kc[i % 2], vc[i % 2], lens, q, out=out, workspace=ws, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    f_us = e0.elapsed_time(e1) / iters * 1e3
+    f_bytes = w.n_kv_heads * n * d * 4 + w.n_q_heads * d * 2
+    res["fp16_baseline"] = {"avg_launch_us": round(f_us, 3), "bytes_per_launch": int(f_bytes),
+                            "achieved_gbs": round(f_bytes / f_us / 1e3, 1),
+                            "quantized_decode_speedup": round(f_us / us, 3)}
+    del kc, vc, kk, vv
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(args, wl, caches, nk, nv, q, stream, device):
@@ -591,6 +669,8 @@ def main():
     ap.add_argument("--copies", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--long-context", type=int, default=1,
+                    help="also time decode alone on the 128k-token workload (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -640,6 +720,8 @@ def main():
             fp16["quantized_decode_speedup"] = round(
                 fp16["avg_launch_us"] / res["roofline"]["avg_launch_us"], 3)
         line["fp16_baseline"] = fp16
+        if res["long_ctx"]:
+            line["long_context_decode"] = res["long_ctx"]
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as tdist
