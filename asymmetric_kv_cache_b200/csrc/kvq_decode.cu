@@ -767,6 +767,36 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
   auto piece = [&](int pc, int h) {
     return partials + (int64_t)(pc == 0 ? s0 : 2 * (kf + pc)) * w.slot_floats + h * (D + 4);
   };
+  if (npc <= 4) {
+    // few pieces: every thread loads its element's values and the pieces'
+    // (m, l) in one round of L2 loads and forms the weights itself
+    for (int idx = tid; idx < nh * D; idx += THREADS) {
+      const int h = idx / D, c = idx % D;
+      float2 ml[4];
+      float o[4];
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        if (pc < npc) {
+          ml[pc] = __ldcg(reinterpret_cast<const float2*>(piece(pc, h) + D));
+          o[pc] = __ldcg(piece(pc, h) + c);
+        } else {
+          ml[pc] = make_float2(-INFINITY, 0.f);
+          o[pc] = 0.f;
+        }
+      }
+      float M = fmaxf(fmaxf(ml[0].x, ml[1].x), fmaxf(ml[2].x, ml[3].x));
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        const float f = ml[pc].x == -INFINITY ? 0.f : fast_exp2(ml[pc].x - M);
+        L += f * ml[pc].y;
+        O += f * o[pc];
+      }
+      reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
+          __float2half_rn(O / L);
+    }
+    return;
+  }
   if (npc <= max_pieces) {
     // (m, l) of every (piece, head) in one round of loads, then the per-head
     // weights, then every element's pieces with all loads in flight

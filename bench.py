@@ -665,7 +665,8 @@ def main():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--workload", default="llama3_8b",
+                    help="llama3_8b (the step), or long_ctx (decode alone on the 128k context)")
     ap.add_argument("--copies", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -704,6 +705,18 @@ def main():
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device(device))
+    if args.workload == "long_ctx":
+        # decode alone on the 128k-token workload (the long-context leg of
+        # the default run on its own, `--steps` timed launches)
+        if rank == 0:
+            stream = torch.cuda.Stream(device=device)
+            lc = run_long_context(stream, device, iters=max(1, args.steps))
+            print(json.dumps({"metric": METRIC, "workload": "long_ctx",
+                              "long_context_decode": lc}))
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+        return 0
     res = run_ours(args, rank, world, device)
     wl = res["wl"]
     cb = cpu_oracle(args.cpu_budget) if (rank == 0 and world == 1) else None
