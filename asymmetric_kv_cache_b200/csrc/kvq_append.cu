@@ -38,12 +38,14 @@ struct AppCfg {
   static constexpr int VWORDS_PER_LANE = D * VB / 64;    // per 16-token tile
   static constexpr int KWORDS = G * D * KB / 32;
   static constexpr int VWORDS = G * D * VB / 32;
-  // dynamic shared memory: fp16 K and V of the group, the fp16 metadata in
-  // slot order, and per key channel / per (token, value group) the fp32
+  // dynamic shared memory: fp16 K and V of the group (token rows padded by
+  // 16 bytes, so that rows fall 4 banks apart), the fp16 metadata in slot
+  // order, and per key channel / per (token, value group) the fp32
   // parameters of the code computation {z, 1/s, s}
+  static constexpr int DP = D + 8;   // halves per staged row
   static constexpr int SM_K = 0;
-  static constexpr int SM_V = SM_K + 2 * G * D;
-  static constexpr int SM_KS = SM_V + 2 * G * D;
+  static constexpr int SM_V = SM_K + 2 * G * DP;
+  static constexpr int SM_KS = SM_V + 2 * G * DP;
   static constexpr int SM_KZ = SM_KS + 2 * D;
   static constexpr int SM_VS = SM_KZ + 2 * D;
   static constexpr int SM_VZ = SM_VS + 2 * G * J;
@@ -236,9 +238,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     }
 #pragma unroll
     for (int j = 0; j < NCH; ++j) {
-      const int ci = tid + 128 * j;
-      reinterpret_cast<uint4*>(sk)[ci] = kx[j];
-      reinterpret_cast<uint4*>(sv)[ci] = vx[j];
+      const int ci = tid + 128 * j, r = ci / CPR, cc = ci % CPR;
+      reinterpret_cast<uint4*>(sk + r * C::DP)[cc] = kx[j];
+      reinterpret_cast<uint4*>(sv + r * C::DP)[cc] = vx[j];
     }
   }
   __syncthreads();
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     for (int cp = tid; cp < D / 2; cp += 64) {
       __half2 mn = sk2[cp], mx = mn;
       for (int r = 1; r < G; ++r) {
-        const __half2 x = sk2[r * (D / 2) + cp];
+        const __half2 x = sk2[r * (C::DP / 2) + cp];
         mn = __hmin2(mn, x);
         mx = __hmax2(mx, x);
       }
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   } else {
     for (int q = tid - 64; q < G * C::J; q += 64) {
       const int r = q / C::J, j = q % C::J;
-      const uint4* row = reinterpret_cast<const uint4*>(sv + r * D + j * G);
+      const uint4* row = reinterpret_cast<const uint4*>(sv + r * C::DP + j * G);
       constexpr int NV = G / 8;
       uint4 w0 = row[r % NV];
       __half2 mn = *reinterpret_cast<__half2*>(&w0.x), mx = mn;
@@ -312,12 +314,14 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   uint32_t* kw = reinterpret_cast<uint32_t*>(blk + g.sec_kcodes);
   const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
   {
-    // A thread's key words (wi = tid + 128k) share one word index w and one
-    // lane, hence one set of channels: their (z, 1/s) are loaded once.
-    static_assert(128 % C::KWORDS_PER_LANE == 0 && (128 / C::KWORDS_PER_LANE) % 32 == 0,
-                  "key words of a thread share their channels");
-    const int w = tid % C::KWORDS_PER_LANE;
-    const int lane = (tid / C::KWORDS_PER_LANE) % 32;
+    // Thread items wi = tid + 128k: lane = wi % 32 varies fastest (a warp
+    // reads 8 tokens x 4 channel pairs: 32 distinct banks of the padded
+    // rows), then the word w of the lane, then the token tile.  A thread's
+    // items share w and the lane, hence one set of channels: their (z, 1/s)
+    // are loaded once.
+    static_assert(4 % C::KWORDS_PER_LANE == 0, "key words of a thread share their channels");
+    const int lane = tid % 32;
+    const int w = (tid / 32) % C::KWORDS_PER_LANE;
     const int i = lane & 3;
     float zk[C::FK][2], rk[C::FK][2];
 #pragma unroll
@@ -334,6 +338,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     for (int wi = tid; wi < C::KWORDS; wi += blockDim.x) {
       const int nt = wi / (C::KWORDS_PER_LANE * 32);
       const int t = 8 * nt + (lane >> 2);
+      const int widx = (nt * 32 + lane) * C::KWORDS_PER_LANE + w;   // layout word
       uint32_t word = 0;
       bool tie = false;
 #pragma unroll
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
         // field f of the low half and of the high half: channels c, c + 1
         const int p = w * C::FK + f;
         const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
-        const float2 x = __half22float2(sk2[(t * D + c) >> 1]);
+        const float2 x = __half22float2(sk2[(t * C::DP + c) >> 1]);
         uint32_t c0, c1;
         codes2(x.x, x.y, zk[f][0], zk[f][1], rk[f][0], rk[f][1], C::QK, c0, c1, tie);
         word |= ((c0 & C::QK) << (KB * f)) | ((c1 & C::QK) << (KB * (C::FK + f)));
@@ -356,19 +361,22 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
           for (int e = 0; e < 2; ++e) {
             const float4 pc = kp[c + e];
             const uint32_t code =
-                (uint32_t)quant_code(__half2float(sk[t * D + c + e]), pc.x, pc.z, C::QK);
+                (uint32_t)quant_code(__half2float(sk[t * C::DP + c + e]), pc.x, pc.z, C::QK);
             word |= code << (KB * (e * C::FK + f));
           }
         }
       }
-      kw[wi] = word;
+      kw[widx] = word;
     }
   }
   uint32_t* vw = reinterpret_cast<uint32_t*>(blk + g.sec_vcodes);
   for (int wi = tid; wi < C::VWORDS; wi += blockDim.x) {
-    const int w = wi % C::VWORDS_PER_LANE;
-    const int lane = (wi / C::VWORDS_PER_LANE) % 32;
+    // lane fastest (a warp reads 4 token pairs x 8 channels: distinct banks
+    // of the padded rows), then the lane's word w, then the token tile
+    const int lane = wi % 32;
+    const int w = (wi / 32) % C::VWORDS_PER_LANE;
     const int kv = wi / (C::VWORDS_PER_LANE * 32);
+    const int widx = (kv * 32 + lane) * C::VWORDS_PER_LANE + w;   // layout word
     const int gg = lane >> 2, i = lane & 3;
     uint32_t word = 0;
     bool tie = false;
@@ -390,8 +398,8 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
       const int t = 16 * kv + 8 * kh + 2 * i;
       const float4 p0 = pv[kh][0], p1 = pv[kh][1];
       uint32_t c0, c1;
-      codes2(__half2float(sv[t * D + c]), __half2float(sv[(t + 1) * D + c]), p0.x, p1.x, p0.y,
-             p1.y, C::QV, c0, c1, tie);
+      codes2(__half2float(sv[t * C::DP + c]), __half2float(sv[(t + 1) * C::DP + c]), p0.x, p1.x,
+             p0.y, p1.y, C::QV, c0, c1, tie);
       word |= ((c0 & C::QV) << (VB * fl)) | ((c1 & C::QV) << (VB * (C::FV + fl)));
     }
     if (tie) {
@@ -407,12 +415,12 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
           const int t = 16 * kv + 8 * kh + 2 * i + e;
           const float4 pc = vp[t * C::J + c / G];
           const uint32_t code =
-              (uint32_t)quant_code(__half2float(sv[t * D + c]), pc.x, pc.z, C::QV);
+              (uint32_t)quant_code(__half2float(sv[t * C::DP + c]), pc.x, pc.z, C::QV);
           word |= code << (VB * (e * C::FV + fl));
         }
       }
     }
-    vw[wi] = word;
+    vw[widx] = word;
   }
   // metadata sections are copied verbatim (already in slot order)
   {
