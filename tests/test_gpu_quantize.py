@@ -155,3 +155,49 @@ def test_prefill_workload_full_size_sampled():
     tl.append_chunks(cache, w.keys, w.values, "fp16")
     tl.check_cache_against_oracle(cache, w.keys, w.values,
                                   group_sample=lambda ng: np.arange(0, ng, 61))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_tail_conversion_is_rne_on_every_pattern(dtype):
+    """The cache's fp16 rounding on entry, bit for bit: stratified fp32 bit
+    patterns (every exponent, ties at the fp16 spacing, the subnormal range,
+    overflow; tests/fp16_rne.py) or every bf16 pattern go through appends
+    that stay in the fp16 tails; the stored halves must equal the binary16
+    round-to-nearest-even written from the format's definition."""
+    import torch
+    from tests.fp16_rne import fp16_bits_rne, stratified_fp32_patterns
+    K = tl.kvq()
+    G, d, T = 32, 128, 31   # 31 tokens per sequence: no group completes
+    if dtype == "fp32":
+        u = stratified_fp32_patterns(np.random.default_rng(11))
+    else:
+        b = np.arange(1 << 16, dtype=np.uint32) << 16
+        u = b[~np.isnan(b.view(np.float32))]
+    per_seq = 2 * T * d                    # K and V elements per sequence
+    n_seq = -(-len(u) // per_seq)
+    pad = n_seq * per_seq - len(u)
+    u = np.concatenate([u, np.zeros(pad, np.uint32)])
+    vals = u.view(np.float32).reshape(n_seq, 2, T, 1, d)
+    spec = K.CacheSpec(4, 2, G, d, 1, 1, n_seq, 64)
+    cache = K.KVQCache(spec)
+    ks = [vals[i, 0] for i in range(n_seq)]
+    vs = [vals[i, 1] for i in range(n_seq)]
+    if dtype == "fp32":
+        kd = torch.from_numpy(np.ascontiguousarray(np.concatenate(ks))).cuda()
+        vd = torch.from_numpy(np.ascontiguousarray(np.concatenate(vs))).cuda()
+    else:   # exact bf16 values: the high halves of the fp32 patterns
+        kd = torch.from_numpy(np.ascontiguousarray(np.concatenate(ks))).cuda().to(torch.bfloat16)
+        vd = torch.from_numpy(np.ascontiguousarray(np.concatenate(vs))).cuda().to(torch.bfloat16)
+    cache.append(kd, vd, [T] * n_seq)
+    torch.cuda.synchronize()
+    from oracle import kvq_oracle as o
+    want = fp16_bits_rne(u).reshape(n_seq, 2, T, d)
+    kidx = np.array([[o.tail_key_index(t, c, d) for c in range(d)] for t in range(T)])
+    vidx = np.array([[o.tail_value_index(t, c, d) for c in range(d)] for t in range(T)])
+    bad = 0
+    for i in range(n_seq):
+        tk, tv = cache.tail_halves(i, 0)
+        hk = tk.cpu().view(torch.int16).numpy().view(np.uint16)
+        hv = tv.cpu().view(torch.int16).numpy().view(np.uint16)
+        bad += int((hk[kidx] != want[i, 0]).sum()) + int((hv[vidx] != want[i, 1]).sum())
+    assert bad == 0, bad
