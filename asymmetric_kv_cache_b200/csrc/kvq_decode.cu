@@ -106,7 +106,10 @@ struct DecCfg {
   static_assert(kHeadsPerSlice * D * 4 <= QA_BYTES, "raw query rows fit the fragment area");
   // merge area (in the idle ring between pieces): the warps' (o, m, l) per
   // head, then the per-head weights of the NW warps, the max and the sum
-  static constexpr int MERGE_FLOATS = NW * kHeadsPerSlice * (D + 2);
+  // rows of D + 8 floats (o[D], m, l, pad): a warp's stores of its state
+  // then fall on 32 distinct banks
+  static constexpr int MRS = D + 8;
+  static constexpr int MERGE_FLOATS = NW * kHeadsPerSlice * MRS;
   static constexpr int WTS_OFF = MERGE_FLOATS;
   static_assert((MERGE_FLOATS + (NW + 2) * kHeadsPerSlice) * 4 <= RING,
                 "merge area must fit in the ring");
@@ -534,7 +537,7 @@ __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw
 // Per-head weights of the NW warps' pieces, (h, warp) per thread: the
 // head's max M and sum L over the warps, and each warp's factor
 // 2^(m_w - M) (divided by L when the piece is the whole unit).
-template <int D, int NW>
+template <int D, int NW, int RS = D + 2>
 __device__ __forceinline__ void merge_weights(const float* __restrict__ merge,
                                               float* __restrict__ wts, bool whole, int tid) {
   constexpr int NWP = NW <= 4 ? 4 : NW <= 8 ? 8 : 16;   // lanes per head
@@ -542,7 +545,7 @@ __device__ __forceinline__ void merge_weights(const float* __restrict__ merge,
   if (tid < kHeadsPerSlice * NWP) {   // whole warps: 8 * NWP is a multiple of 32
     const int h = tid / NWP, ww = tid % NWP;
     const bool v = ww < NW;
-    const float* mo = merge + (ww * kHeadsPerSlice + h) * (D + 2);
+    const float* mo = merge + (ww * kHeadsPerSlice + h) * RS;
     const float mw = v ? mo[D] : -INFINITY;
     const float lw = v ? mo[D + 1] : 0.f;
     float M = mw;
@@ -907,6 +910,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
   __shared__ int32_t wsum[NW];
   __shared__ int32_t claim;   // next unclaimed group of the current piece
   __shared__ int32_t ticket_flag[3];
+  __shared__ Piece piece_s;   // the current piece, for the merge after the group loop
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint4* qsm = reinterpret_cast<uint4*>(smem + C::QA_OFF);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + C::SMEM_FIXED);
@@ -1005,6 +1009,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     bool my_tail;        // this warp owns tail chunk `warp`
     {
       const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+      if (tid == 0) piece_s = p;   // published by the barriers below
       gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
       ngr = max(0, min(p.slot1, p.ng) - p.slot0);
       nh = p.nh;
@@ -1111,13 +1116,14 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     // waited on, except after a failed wait)
     fence_proxy_async_smem();
     __syncthreads();
-    // the piece again (rebuilt rather than kept through the group loop)
-    const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+    // the piece again (from shared memory rather than kept through the loop)
+    const Piece p = piece_s;
     const int b = p.b, slot0 = p.slot0, slot1 = p.slot1, wb = p.wb, unit = p.unit;
     const int hbase = p.hbase;
     if (tid == 0) claim = 0;   // for the next piece (published by the barriers below)
     {
-      float* mo = merge + (warp * kHeadsPerSlice) * (D + 2);
+      constexpr int RS = C::MRS;
+      float* mo = merge + (warp * kHeadsPerSlice) * RS;
       // value-min terms for channel group j and heads 2*i4, 2*i4+1 live in
       // lane 4j + i4; the denominators in lane 4J + i4
       float zl0[C::J], zl1[C::J];
@@ -1128,29 +1134,38 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       }
       const float l0 = __shfl_sync(0xffffffffu, st.z[0], 4 * C::J + i4);
       const float l1 = __shfl_sync(0xffffffffu, st.z[1], 4 * C::J + i4);
-      // (packed: columns 4-7 repeat heads 0-3 and are skipped)
-      if (!PK || i4 < 2) {
+      if constexpr (PK) {
+        // columns 4-7 repeat heads 0-3 bit for bit (the same B columns and
+        // rescale factors), so lanes i4 >= 2 store the channel + 8 half of
+        // lane i4 - 2's heads: every lane stores two values per m-tile
+        const int hh = 2 * (i4 & 1);
+        const int co = (i4 >= 2) ? 8 : 0;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int c = 16 * mt + g8 + co;
+          const int j = (16 * mt) / G;
+          mo[hh * RS + c] = ((i4 >= 2) ? st.o[mt][2] : st.o[mt][0]) + zl0[j];
+          mo[(hh + 1) * RS + c] = ((i4 >= 2) ? st.o[mt][3] : st.o[mt][1]) + zl1[j];
+        }
+        if (g8 == 0 && i4 < 2) {
+          mo[(2 * i4) * RS + D] = st.m[0];
+          mo[(2 * i4 + 1) * RS + D] = st.m[1];
+        }
+      } else {
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
           const int c0 = 16 * mt + g8, c1 = c0 + 8;
           const int j = (16 * mt) / G;
-          mo[(2 * i4) * (D + 2) + c0] = st.o[mt][0] + zl0[j];
-          mo[(2 * i4 + 1) * (D + 2) + c0] = st.o[mt][1] + zl1[j];
-          mo[(2 * i4) * (D + 2) + c1] = st.o[mt][2] + zl0[j];
-          mo[(2 * i4 + 1) * (D + 2) + c1] = st.o[mt][3] + zl1[j];
+          mo[(2 * i4) * RS + c0] = st.o[mt][0] + zl0[j];
+          mo[(2 * i4 + 1) * RS + c0] = st.o[mt][1] + zl1[j];
+          mo[(2 * i4) * RS + c1] = st.o[mt][2] + zl0[j];
+          mo[(2 * i4 + 1) * RS + c1] = st.o[mt][3] + zl1[j];
         }
-      }
-      if constexpr (PK) {
-        if (g8 == 0 && i4 < 2) {
-          mo[(2 * i4) * (D + 2) + D] = st.m[0];
-          mo[(2 * i4 + 1) * (D + 2) + D] = st.m[1];
-        }
-      } else {
-        if (i4 == 0) mo[g8 * (D + 2) + D] = st.m[0];
+        if (i4 == 0) mo[g8 * RS + D] = st.m[0];
       }
       if (g8 == 0) {
-        mo[(2 * i4) * (D + 2) + D + 1] = l0;
-        mo[(2 * i4 + 1) * (D + 2) + D + 1] = l1;
+        mo[(2 * i4) * RS + D + 1] = l0;
+        mo[(2 * i4 + 1) * RS + D + 1] = l1;
       }
     }
     __syncthreads();
@@ -1158,7 +1173,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     const bool whole = (slot0 == 0 && slot1 == wb);
     // [h][NW] weights of the warps' shares, then [h] max and [h] sum
     float* wts = merge + C::WTS_OFF;
-    merge_weights<D, NW>(merge, wts, whole, tid);
+    merge_weights<D, NW, C::MRS>(merge, wts, whole, tid);
     // Partial slots: a CTA holds at most two split pieces, its first (slot
     // 2k) and its last (2k + 1); pieces in between are whole units.
     const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
@@ -1173,8 +1188,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     for (int idx = tid; idx < nh * D; idx += C::THREADS) {
       const int h = idx / D, c = idx % D;
       const float* f = wts + h * NW;
-      const float* mo = merge + h * (D + 2) + c;
-      constexpr int WS = kHeadsPerSlice * (D + 2);   // stride between the warps' areas
+      const float* mo = merge + h * C::MRS + c;
+      constexpr int WS = kHeadsPerSlice * C::MRS;   // stride between the warps' areas
       float O = 0.f;
 #pragma unroll
       for (int ww = 0; ww < NW; ++ww) O += f[ww] * mo[ww * WS];
