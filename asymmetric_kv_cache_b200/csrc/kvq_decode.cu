@@ -879,19 +879,22 @@ struct Piece {
 
 // Built from the slot position alone, so that it can be rebuilt after the
 // group loop instead of holding registers through it.
+// (G: the group size when the caller knows it at compile time - a shift
+// instead of a division on the path to the piece's first copies - else 0)
+template <int G = 0>
 __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix,
                                             const int32_t* slen, int n_seq, int pos, int end) {
   Piece p;
   p.b = find_seq(prefix, n_seq, pos);
   p.L = slen[p.b];
-  p.ng = p.L / g.G;
-  p.Tb = p.L - p.ng * g.G;
+  p.ng = G ? p.L / G : p.L / g.G;
+  p.Tb = p.L - p.ng * (G ? G : g.G);
   p.wb = p.ng + (p.Tb ? 1 : 0);
   const int local = pos - prefix[p.b];
   const int uis = local / p.wb;
   p.slot0 = local - uis * p.wb;
   p.slot1 = min(p.wb, p.slot0 + (end - pos));
-  p.kvh = uis / g.slices;
+  p.kvh = g.slices == 1 ? uis : uis / g.slices;
   p.slice = uis - p.kvh * g.slices;
   p.unit = p.b * (g.hkv * g.slices) + uis;
   p.hbase = p.kvh * g.gqa + p.slice * kHeadsPerSlice;
@@ -1008,7 +1011,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     int64_t gb;          // global block index of the piece's first group
     bool my_tail;        // this warp owns tail chunk `warp`
     {
-      const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+      const Piece p = make_piece<G>(g, prefix, slen, n_seq, pos, end);
       if (tid == 0) piece_s = p;   // published by the barriers below
       gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
       ngr = max(0, min(p.slot1, p.ng) - p.slot0);
@@ -1069,7 +1072,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     if (my_tail) {
       cp_async_wait_all();
       __syncwarp();
-      const Piece p = make_piece(g, prefix, slen, n_seq, pos, end);
+      const Piece p = piece_s;
       const unsigned char* tb =
           C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
       if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
