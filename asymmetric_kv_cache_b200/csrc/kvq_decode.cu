@@ -1188,20 +1188,32 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
     __syncthreads();
-    for (int idx = tid; idx < nh * D; idx += C::THREADS) {
-      const int h = idx / D, c = idx % D;
+    // four channels per thread: 128-bit loads of the warps' rows, 128-bit
+    // partial stores (rows of D + 8 floats and partial rows of D + 4 keep
+    // every such address 16-byte aligned)
+    static_assert(C::MRS % 4 == 0 && (D + 4) % 4 == 0, "16-byte aligned merge rows");
+    for (int idx = tid; idx < nh * (D / 4); idx += C::THREADS) {
+      const int h = idx / (D / 4), c = 4 * (idx % (D / 4));
       const float* f = wts + h * NW;
       const float* mo = merge + h * C::MRS + c;
       constexpr int WS = kHeadsPerSlice * C::MRS;   // stride between the warps' areas
-      float O = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int ww = 0; ww < NW; ++ww) O += f[ww] * mo[ww * WS];
+      for (int ww = 0; ww < NW; ++ww) {
+        const float fw = f[ww];
+        const float4 x = *reinterpret_cast<const float4*>(mo + ww * WS);
+        O.x = fmaf(fw, x.x, O.x);
+        O.y = fmaf(fw, x.y, O.y);
+        O.z = fmaf(fw, x.z, O.z);
+        O.w = fmaf(fw, x.w, O.w);
+      }
       if (whole) {
-        reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-            __float2half_rn(O);
+        const uint2 hv = make_uint2(pack_h2(O.x, O.y), pack_h2(O.z, O.w));
+        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.out) +
+                                  ((int64_t)b * g.hq + hbase + h) * D + c) = hv;
       } else {
         float* ps = partials + myslot * w.slot_floats + h * (D + 4);
-        ps[c] = O;
+        *reinterpret_cast<float4*>(ps + c) = O;
         if (c == 0) {
           ps[D] = wts[NW * kHeadsPerSlice + h];
           ps[D + 1] = wts[(NW + 1) * kHeadsPerSlice + h];
