@@ -303,12 +303,12 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     a.ws = ws;
     a.n_seq = ns;
     a.seq0 = s0;
-    // wide CTAs (one unit piece each) with few pieces per split unit: the
-    // last CTA of each unit merges them (no combine kernel).  Otherwise the
-    // combine kernel: a narrow CTA moves on to its next piece, which an
-    // in-kernel merge would delay; many pieces merge faster spread out.
+    // wide CTAs (one unit piece each) with up to 32 pieces per split unit:
+    // the last CTA of each unit merges them in one round of L2 loads (no
+    // combine kernel).  Otherwise the combine kernel: a narrow CTA moves on
+    // to its next piece, which an in-kernel merge would delay.
     const int64_t units = (int64_t)ns * g.hkv * g.slices;
-    a.inline_merge = (wide && (grid / units + 1) <= 4) ? 1 : 0;
+    a.inline_merge = (wide && (grid / units + 1) <= 32) ? 1 : 0;
     cudaError_t e = kvq::launch_decode(g, w, a, (int)grid, wide, stream);
     if (e != cudaSuccess) return e;
   }

@@ -770,6 +770,61 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
   auto piece = [&](int pc, int h) {
     return partials + (int64_t)(pc == 0 ? s0 : 2 * (kf + pc)) * w.slot_floats + h * (D + 4);
   };
+  if (npc > 4 && npc <= 32) {
+    // up to 32 pieces: an item is (head, 4 channels); 4 threads share an
+    // item, each loading its pieces' 4 values and (m, l) (up to 8 pieces,
+    // every load in flight at once: one round of L2 latency), merging them
+    // in registers, then the 4 threads merge through shuffles
+    constexpr int TPI = 4;
+    const int sub = tid % TPI;
+    for (int it = tid / TPI; it < nh * (D / 4); it += THREADS / TPI) {
+      const int h = it / (D / 4), c = 4 * (it % (D / 4));
+      float2 ml[8];
+      float4 o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int pc = sub + TPI * k;
+        if (pc < npc) {
+          ml[k] = __ldcg(reinterpret_cast<const float2*>(piece(pc, h) + D));
+          o[k] = __ldcg(reinterpret_cast<const float4*>(piece(pc, h) + c));
+        } else {
+          ml[k] = make_float2(-INFINITY, 0.f);
+          o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float M = ml[0].x;
+#pragma unroll
+      for (int k = 1; k < 8; ++k) M = fmaxf(M, ml[k].x);
+      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+      M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float f = ml[k].x == -INFINITY ? 0.f : fast_exp2(ml[k].x - M);
+        L = fmaf(f, ml[k].y, L);
+        O.x = fmaf(f, o[k].x, O.x);
+        O.y = fmaf(f, o[k].y, O.y);
+        O.z = fmaf(f, o[k].z, O.z);
+        O.w = fmaf(f, o[k].w, O.w);
+      }
+#pragma unroll
+      for (int x = 1; x < TPI; x <<= 1) {
+        L += __shfl_xor_sync(0xffffffffu, L, x);
+        O.x += __shfl_xor_sync(0xffffffffu, O.x, x);
+        O.y += __shfl_xor_sync(0xffffffffu, O.y, x);
+        O.z += __shfl_xor_sync(0xffffffffu, O.z, x);
+        O.w += __shfl_xor_sync(0xffffffffu, O.w, x);
+      }
+      if (sub == 0) {
+        const float inv = 1.0f / L;
+        const uint2 hv = make_uint2(pack_h2(O.x * inv, O.y * inv), pack_h2(O.z * inv, O.w * inv));
+        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.out) +
+                                  ((int64_t)b * g.hq + hbase + h) * D + c) = hv;
+      }
+    }
+    return;
+  }
   if (npc <= 4) {
     // few pieces: every thread loads its element's values and the pieces'
     // (m, l) in one round of L2 loads and forms the weights itself
