@@ -1000,7 +1000,24 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     prefix[0] = 0;
     claim = 0;
   }
-  {
+  if (n_seq <= 32) {
+    // one warp: a lane per sequence and a shuffle scan (no block barrier on
+    // the way to the first copies)
+    if (warp == 0) {
+      const int L = lane < n_seq ? lens[lane] : 0;
+      const int32_t run = per_seq_units * (L / G + (L % G ? 1 : 0));
+      int32_t incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane < n_seq) {
+        prefix[lane + 1] = incl;
+        slen[lane] = L;
+      }
+    }
+  } else {
     const int chunk = (n_seq + C::THREADS - 1) / C::THREADS;
     const int b0 = tid * chunk, b1 = min(n_seq, b0 + chunk);
     int32_t run = 0;
