@@ -29,6 +29,12 @@ Readings where the pages are silent (each is listed in the design notes):
 * key groups: G consecutive tokens from position 0 of each sequence; value
   groups: G consecutive channels of one token; the tail holds the n mod G
   newest tokens of both K and V.
+* recent window R (same page, §III and §V: the most recent tokens, 32 to
+  128 of them, stay in FP16): with R > 0 a group is quantized only once R
+  newer tokens follow it, so the tail holds between R and R + G - 1 tokens
+  (all n tokens while n < R); R = 0 is the n mod G tail above.  The tail is a
+  ring of R + G token slots: token p sits in slot p mod (R + G), so tokens
+  never move while they wait (our layout; the pages do not store it).
 * GQA: query head h reads kv head floor(h / (Hq / Hkv)).
 * attention is evaluated in float64 on the dequantized cache
   x_hat = code * s + z (tail tokens exactly as stored in fp16).
@@ -63,6 +69,11 @@ class Config:
     n_kv_heads: int
     max_seqs: int = 1
     max_tokens: int = 0
+    window: int = 0      # R: recent tokens kept in fp16 beyond the partial group
+
+    @property
+    def tail_slots(self) -> int:   # W = R + G slots of the fp16 tail ring
+        return self.window + self.group
 
     @property
     def gqa(self) -> int:
@@ -432,10 +443,22 @@ def unpack_block(cfg: Config, blk: np.ndarray):
 # ---------------------------------------------------------------------------
 # the cache: groups + fp16 tail, as a function of the token history
 # ---------------------------------------------------------------------------
-def split_tokens(n: int, group: int):
-    """(N, T): tokens in full key groups, tokens in the fp16 tail (n mod G)."""
-    T = n % group
-    return n - T, T
+def split_tokens(n: int, group: int, window: int = 0):
+    """(N, T): tokens in quantized key groups, tokens in the fp16 tail.
+
+    Groups are cut from position 0 and one is quantized once ``window`` (R)
+    newer tokens follow it: N = G floor(max(0, n - R) / G), T = n - N, so T is
+    n mod G for R = 0 and lies in [R, R + G - 1] once n >= R ("[Framework] The
+    Asymmetric Key-Value Cache Compression", §III and §V).
+    """
+    N = group * (max(0, n - window) // group)
+    return N, n - N
+
+
+def tail_slot(cfg: Config, p: int) -> int:
+    """Slot of the fp16 tail ring that token position p occupies while it is
+    in the tail: p mod (R + G)."""
+    return p % cfg.tail_slots
 
 
 def quantize_group(cfg: Config, k16: np.ndarray, v16: np.ndarray):
@@ -447,9 +470,9 @@ def quantize_group(cfg: Config, k16: np.ndarray, v16: np.ndarray):
 
 
 def grouped(cfg: Config, x16: np.ndarray) -> np.ndarray:
-    """[n, Hkv, d] token history -> [Hkv, N/G, G, d] full groups."""
+    """[n, Hkv, d] token history -> [Hkv, N/G, G, d] quantized groups."""
     G = cfg.group
-    N, _ = split_tokens(x16.shape[0], G)
+    N, _ = split_tokens(x16.shape[0], G, cfg.window)
     x = np.asarray(x16[:N], np.float16).reshape(N // G, G, x16.shape[1], x16.shape[2])
     return x.transpose(2, 0, 1, 3)
 
@@ -460,10 +483,11 @@ def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True
     k16, v16: [n, Hkv, d] fp16 token history.  Returns a dict with
     ``groups``: (kc, ks, kz, vc, vs, vz) with a leading [Hkv, n_groups] shape,
     ``blocks``: [Hkv, n_groups, block_bytes] uint8 (if ``pack``),
-    ``tail_k``/``tail_v``: [Hkv, T, d] fp16 tail tokens, and N, T.
+    ``tail_k``/``tail_v``: [Hkv, T, d] fp16 tail tokens (positions N .. n-1 in
+    order), and N, T.
     """
     n = k16.shape[0]
-    N, T = split_tokens(n, cfg.group)
+    N, T = split_tokens(n, cfg.group, cfg.window)
     q = quantize_group(cfg, grouped(cfg, k16), grouped(cfg, v16))
     out = {"N": N, "T": T, "groups": q}
     if pack:
@@ -473,17 +497,19 @@ def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True
     return out
 
 
-def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray):
-    """Place T tail tokens [T, d] into the G-slot tail arrays (flat fp16,
-    LAYOUT v1); slots >= T are zero here (their device contents are
-    unspecified)."""
-    G, d = cfg.group, cfg.head_dim
-    tk = np.zeros(G * d, np.float16)
-    tv = np.zeros(G * d, np.float16)
-    for t in range(tail_k.shape[0]):
+def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray, first: int = 0):
+    """Place T tail tokens [T, d], the first at sequence position ``first``,
+    into the (R + G)-slot tail arrays (flat fp16, LAYOUT v1): token
+    first + i goes to slot tail_slot(first + i).  Slots holding no tail token
+    are zero here (their device contents are unspecified)."""
+    W, d = cfg.tail_slots, cfg.head_dim
+    tk = np.zeros(W * d, np.float16)
+    tv = np.zeros(W * d, np.float16)
+    for i in range(tail_k.shape[0]):
+        t = tail_slot(cfg, first + i)
         for c in range(d):
-            tk[tail_key_index(t, c, d)] = tail_k[t, c]
-            tv[tail_value_index(t, c, d)] = tail_v[t, c]
+            tk[tail_key_index(t, c, d)] = tail_k[i, c]
+            tv[tail_value_index(t, c, d)] = tail_v[i, c]
     return tk, tv
 
 
