@@ -75,6 +75,8 @@ kvq_status validate_config(const kvq_config* c) {
   if (c->max_seqs < 1 || c->max_tokens < 1)
     return fail(KVQ_ERR_CONFIG, "max_seqs and max_tokens must be >= 1 (got %d, %d)", c->max_seqs,
                 c->max_tokens);
+  if (c->window < 0 || c->window > 1024 || c->window % 16 != 0)
+    return fail(KVQ_ERR_CONFIG, "window must be a multiple of 16 in [0, 1024] (got %d)", c->window);
   // decode addresses slots (groups + tail) of all units with 32-bit prefixes
   const int64_t slices = (c->n_q_heads / c->n_kv_heads + kvq::kHeadsPerSlice - 1) / kvq::kHeadsPerSlice;
   const int64_t slots = (int64_t)c->max_seqs * c->n_kv_heads * slices * (c->max_tokens / c->group + 1);
@@ -98,6 +100,7 @@ void fill_layout(const kvq::Geom& g, kvq_layout* o) {
   o->max_groups = g.max_groups;
   o->tails_offset = g.tails_off;
   o->tail_bytes = g.tail_bytes;
+  o->tail_slots = (uint64_t)g.tail_slots;
   o->kcodes_offset = g.sec_kcodes;
   o->kscale_offset = g.sec_kscale;
   o->kmin_offset = g.sec_kmin;
@@ -232,8 +235,10 @@ kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype 
     for (int i = 0; i < n; ++i) {
       const int b = s0 + i;
       const int len0 = cache->lens[b], nn = n_new[b];
-      const int T0 = len0 % g.G;
-      const int F = (T0 + nn) / g.G;
+      // groups this append completes (the kernel recomputes them from the
+      // device lengths; for nn < G at most one, whatever the length)
+      const int F = kvq::quantized_groups(len0 + nn, g.G, g.window) -
+                    kvq::quantized_groups(len0, g.G, g.window);
       seqs.task_prefix[i] = tasks;
       seqs.row_off[i] = (int32_t)row;
       seqs.n_new[i] = nn;
@@ -259,9 +264,9 @@ namespace {
 int64_t choose_grid(const kvq::Geom& g, const int32_t* lens, int n_seq, int64_t slots, int cap) {
   int64_t grid = std::min<int64_t>(slots, cap);
   const int64_t units = (int64_t)n_seq * g.hkv * g.slices;
-  const int w0 = lens[0] / g.G + (lens[0] % g.G ? 1 : 0);
+  const int w0 = kvq::unit_slots(lens[0], g.G, g.window);
   bool equal = true;
-  for (int b = 1; b < n_seq && equal; ++b) equal = (lens[b] / g.G + (lens[b] % g.G ? 1 : 0)) == w0;
+  for (int b = 1; b < n_seq && equal; ++b) equal = kvq::unit_slots(lens[b], g.G, g.window) == w0;
   if (equal && units <= cap) {
     const int64_t alt = std::min<int64_t>(slots, units * (cap / units));
     if (alt * 5 >= (int64_t)cap * 4) grid = alt;
@@ -293,7 +298,7 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     if (env_cap > 0) cap = std::min(cap, env_cap);
     int64_t slots = 0;
     for (int b = s0; b < s0 + ns; ++b)
-      slots += (int64_t)g.hkv * g.slices * (lens[b] / g.G + (lens[b] % g.G ? 1 : 0));
+      slots += (int64_t)g.hkv * g.slices * kvq::unit_slots(lens[b], g.G, g.window);
     const int64_t grid = std::min(max_grid, choose_grid(g, lens + s0, ns, slots, cap));
     kvq::DecodeArgs a;
     a.cache = cache_buf;

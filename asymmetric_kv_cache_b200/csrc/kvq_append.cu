@@ -10,9 +10,13 @@
 // Grid: x = tasks (flattened over sequences), y = kv head; 128 threads.
 // A task is either one group to quantize (tokens taken from the old tail
 // and/or the input) or, when no group completes, the copy of the new tokens
-// into the tail.  The task that quantizes the first completed group of a
-// sequence also writes that sequence's new tail, after it has read the old
-// one, so no other CTA touches the tail concurrently.
+// into the tail.  With a recent window of R tokens a group is quantized once
+// R newer tokens follow it (same page, §III and §V), and the tail is a ring
+// of W = R + G token slots (token p in slot p mod W), so tokens that stay in
+// the tail never move.  A slot whose old token a group task reads is
+// rewritten, if a new tail token maps to it, by that same task after its
+// read; every other new tail token is written by the sequence's first task.
+// So no slot is read and written by two CTAs.
 //
 // Every CTA reads the sequence's current length from the device copy when
 // it starts; the last CTA of the sequence to finish (atomic ticket in the
@@ -178,14 +182,17 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   const int len0 = *reinterpret_cast<volatile int32_t*>(lens + seq);
   const int nn = s.n_new[b];
   const int seq_ctas = (s.task_prefix[b + 1] - s.task_prefix[b]) * gridDim.y;
-  const int T0 = len0 % G;
-  const int N0 = len0 - T0;
-  const int F = (T0 + nn) / G;     // groups completed by this append
-  const int T1 = (T0 + nn) % G;    // tail length afterwards
+  const int W = g.tail_slots;      // ring slots of the tail: R + G
+  const int N0 = G * quantized_groups(len0, G, g.window);
+  const int T0 = len0 - N0;        // tail length before
+  const int n1 = len0 + nn;
+  const int N1 = G * quantized_groups(n1, G, g.window);
+  const int F = (N1 - N0) / G;     // groups completed by this append
   const int64_t row0 = s.row_off[b];
   const int64_t unit = (int64_t)seq * g.hkv + kvh;
   __half* tailk = reinterpret_cast<__half*>(cache + g.tails_off + unit * g.tail_bytes);
-  __half* tailv = tailk + G * D;
+  __half* tailv = tailk + (int64_t)W * D;
+  const int base0 = N0 % W;        // ring slot of position N0
   auto in_idx = [&](int64_t r, int c) { return ((row0 + r) * g.hkv + kvh) * D + c; };
   // A replayed capture can ask for more than the capacity, which the host
   // could not check: such an append writes nothing and the length stays.
@@ -205,10 +212,14 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
 
   constexpr int CPR = D / 8;   // 16-byte fp16 chunks per token row
   if (F == 0) {
-    // no group completes: new tokens go to tail slots T0 .. T0 + nn - 1
+    // no group completes: new token len0 + j goes to ring slot
+    // (len0 + j) mod W, which holds no tail token (the tail stays below W)
+    const int sl0 = (base0 + T0) % W;
     for (int ci = tid; ci < nn * CPR; ci += blockDim.x) {
       const int j = ci / CPR, cc = ci % CPR;
-      store_tail8(tailk, tailv, T0 + j, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
+      int sl = sl0 + j;
+      sl -= (sl >= W) ? W : 0;
+      store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
                   load8_fp16(vin, in_idx(j, 8 * cc), dtype));
     }
     finish();
@@ -219,8 +230,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     return;
   }
 
-  // ---- load the group: virtual token u = tau*G + r of [old tail ++ input],
-  // 16-byte chunks, every load of a thread issued before its stores
+  // ---- load the group: position N0 + u (u = tau*G + r) is old tail
+  // token u (ring slot (N0 + u) mod W) or input row u - T0; 16-byte chunks,
+  // every load of a thread issued before its stores
   {
     constexpr int NCH = G * CPR / 128;   // chunks per thread (K and V each)
     uint4 kx[NCH], vx[NCH];
@@ -229,8 +241,10 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
       const int ci = tid + 128 * j, r = ci / CPR, cc = ci % CPR;
       const int u = tau * G + r;
       if (u < T0) {
-        kx[j] = *reinterpret_cast<const uint4*>(tailk + u * D + 8 * cc);
-        vx[j] = tail_v8(tailv, u, cc, D);
+        int sl = base0 + u;
+        sl -= (sl >= W) ? W : 0;
+        kx[j] = *reinterpret_cast<const uint4*>(tailk + sl * D + 8 * cc);
+        vx[j] = tail_v8(tailv, sl, cc, D);
       } else {
         kx[j] = load8_fp16(kin, in_idx(u - T0, 8 * cc), dtype);
         vx[j] = load8_fp16(vin, in_idx(u - T0, 8 * cc), dtype);
@@ -440,15 +454,34 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     for (int i = tid; i < G * C::J / 2; i += blockDim.x) dst[i] = src[i];
   }
 
-  if (tau == 0) {
-    // the new tail: virtual tokens F*G .. F*G + T1 - 1, all from the input
-    // (the old tail was fully read above, before the barrier)
-    for (int ci = tid; ci < T1 * CPR; ci += blockDim.x) {
-      const int t = ci / CPR, cc = ci % CPR;
-      const int64_t r = (int64_t)F * G + t - T0;
-      store_tail8(tailk, tailv, t, cc, D, load8_fp16(kin, in_idx(r, 8 * cc), dtype),
-                  load8_fp16(vin, in_idx(r, 8 * cc), dtype));
-    }
+  // ---- the new tail: positions [A, n1), all new tokens (input rows p -
+  // len0).  Ring residue rr = (p - N0) mod W: rr < T0 is the slot of old
+  // tail token N0 + rr, which this append quantizes in task rr / G (that
+  // task read it before the barrier above), so that task writes the slot;
+  // residues T0 .. W-1 hold no old tail token and task 0 writes them.  Each
+  // residue occurs at most once in [A, n1) (the new tail is shorter than W).
+  {
+    const int A = max(N1, len0);
+    const int r_lo = tau * G;
+    const int r_hi = min(T0, r_lo + G);
+    auto write_residues = [&](int lo, int hi) {
+      for (int ci = tid; ci < (hi - lo) * CPR; ci += blockDim.x) {
+        const int rr = lo + ci / CPR, cc = ci % CPR;
+        // the position p >= A with p = N0 + rr (mod W)
+        int off = (N0 + rr - A) % W;
+        off += (off < 0) ? W : 0;
+        const int p = A + off;
+        if (p < n1) {
+          int sl = base0 + rr;
+          sl -= (sl >= W) ? W : 0;
+          const int64_t r = (int64_t)p - len0;
+          store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(r, 8 * cc), dtype),
+                      load8_fp16(vin, in_idx(r, 8 * cc), dtype));
+        }
+      }
+    };
+    if (r_lo < r_hi) write_residues(r_lo, r_hi);
+    if (tau == 0) write_residues(T0, W);
   }
   finish();
 }

@@ -113,11 +113,13 @@ struct DecCfg {
   static constexpr int WTS_OFF = MERGE_FLOATS;
   static_assert((MERGE_FLOATS + (NW + 2) * kHeadsPerSlice) * 4 <= RING,
                 "merge area must fit in the ring");
-  // The tail (< G tokens, G/16 chunks of 16): chunk kv belongs to warp kv,
-  // which stages it when the piece starts (its copy latency hidden behind
-  // the query's) and processes it before claiming groups.  For 32-token
-  // groups the chunks get an area of their own, for larger ones they go
-  // through the warp's ring, which then starts its group copies late.
+  // The tail, in chunks of 16 tokens (< G/16 chunks without a recent
+  // window, up to (R + G - 1)/16 with one): chunk c belongs to warp
+  // c mod TAIL_CHUNKS, which stages its first chunk when the piece starts
+  // (its copy latency hidden behind the query's) and processes its chunks
+  // one after another before claiming groups.  For 32-token groups the
+  // chunks get an area of their own, for larger ones they go through the
+  // warp's ring, which then starts its group copies late.
   static constexpr int TAIL_CHUNKS = G / 16;
   static constexpr bool TAIL_EARLY = (G == 32);
   static_assert(TAIL_EARLY || TailStage<D>::BYTES <= NST * BLK, "tail chunk fits a warp's ring");
@@ -349,6 +351,22 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   softmax_update<D, NT, KB, VB, G>(st, s, *reinterpret_cast<uint32_t(*)[NT]>(&pt[0][0]),
                                    lane & 3);
   value_side<D, KB, VB, G, false>(st, sp, pt, lane);
+}
+
+// Decode slots of a unit with L tokens: its quantized groups plus one for a
+// non-empty tail (the window-free form when WIN is false).
+template <int G, bool WIN>
+__device__ __forceinline__ int dec_unit_slots(int L, int window) {
+  if constexpr (WIN) return unit_slots(L, G, window);
+  else return L / G + (L % G ? 1 : 0);
+}
+
+// Ring slot of the first token of tail chunk c (tokens 16c .. 16c + 15 of a
+// tail whose first token sits at sequence position `first`) in a tail ring
+// of W slots (token p in slot p mod W).  first and W are multiples of 16, so
+// a chunk never wraps.
+__device__ __forceinline__ int tail_chunk_slot(int first, int c, int W) {
+  return (first + 16 * c) % W;
 }
 
 // Issue the cp.async copies of tail chunk kv (16 tokens: key rows and
@@ -935,14 +953,20 @@ struct Piece {
 // Built from the slot position alone, so that it can be rebuilt after the
 // group loop instead of holding registers through it.
 // (G: the group size when the caller knows it at compile time - a shift
-// instead of a division on the path to the piece's first copies - else 0)
-template <int G = 0>
+// instead of a division on the path to the piece's first copies - else 0;
+// WIN: the cache has a recent window, g.window > 0)
+template <int G = 0, bool WIN = false>
 __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix,
                                             const int32_t* slen, int n_seq, int pos, int end) {
   Piece p;
   p.b = find_seq(prefix, n_seq, pos);
   p.L = slen[p.b];
-  p.ng = G ? p.L / G : p.L / g.G;
+  if constexpr (WIN) {
+    const int Lq = p.L - g.window;   // groups leave the newest `window` tokens in fp16
+    p.ng = Lq <= 0 ? 0 : G ? Lq / G : Lq / g.G;
+  } else {
+    p.ng = G ? p.L / G : p.L / g.G;
+  }
   p.Tb = p.L - p.ng * (G ? G : g.G);
   p.wb = p.ng + (p.Tb ? 1 : 0);
   const int local = pos - prefix[p.b];
@@ -957,7 +981,10 @@ __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix
   return p;
 }
 
-template <int D, int KB, int VB, int G, bool PK, bool WIDE>
+// WIN: compiled for caches with a recent window (tails of up to R + G - 1
+// tokens in a ring of R + G slots); the kernels without it keep the
+// single-chunk-per-warp tail and its register budget.
+template <int D, int KB, int VB, int G, bool PK, bool WIDE, bool WIN>
 __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
                                   DecCfg<D, KB, VB, G, WIDE>::MIN_BLOCKS)
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
@@ -1005,7 +1032,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     // the way to the first copies)
     if (warp == 0) {
       const int L = lane < n_seq ? lens[lane] : 0;
-      const int32_t run = per_seq_units * (L / G + (L % G ? 1 : 0));
+      const int32_t run = per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
       int32_t incl = run;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1023,7 +1050,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     int32_t run = 0;
     for (int bb = b0; bb < b1; ++bb) {
       const int L = lens[bb];
-      run += per_seq_units * (L / G + (L % G ? 1 : 0));
+      run += per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
     }
     // exclusive scan of the per-thread sums across the block
     int32_t incl = run;
@@ -1039,7 +1066,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     int32_t acc = base + incl - run;
     for (int bb = b0; bb < b1; ++bb) {
       const int L = lens[bb];
-      acc += per_seq_units * (L / G + (L % G ? 1 : 0));
+      acc += per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
       prefix[bb + 1] = acc;
       slen[bb] = L;
     }
@@ -1081,14 +1108,15 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
 
     int ngr, nh;         // groups in this piece, heads of the unit
     int64_t gb;          // global block index of the piece's first group
-    bool my_tail;        // this warp owns tail chunk `warp`
+    bool my_tail;        // this warp owns tail chunks warp, warp + TAIL_CHUNKS, ...
     {
-      const Piece p = make_piece<G>(g, prefix, slen, n_seq, pos, end);
+      const Piece p = make_piece<G, WIN>(g, prefix, slen, n_seq, pos, end);
       if (tid == 0) piece_s = p;   // published by the barriers below
       gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
       ngr = max(0, min(p.slot1, p.ng) - p.slot0);
       nh = p.nh;
       my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng && warp * 16 < p.Tb;
+      if constexpr (WIN) my_tail = my_tail && warp < C::TAIL_CHUNKS;
       // the unit's raw query rows first, so that they are not queued behind
       // the group blocks
       if (tid == 0) {
@@ -1104,9 +1132,14 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       if (my_tail) {
         const __half* tk = reinterpret_cast<const __half*>(
             a.cache + g.tails_off + ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.tail_bytes);
-        stage_tail_chunk<D>(C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES
-                                          : wring,
-                            tk, tk + G * D, p.Tb, warp, lane);
+        unsigned char* tb = C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
+        if constexpr (WIN) {
+          const int64_t so = tail_chunk_slot(p.ng * G, warp, g.tail_slots) * D;
+          stage_tail_chunk<D>(tb, tk + so, tk + (int64_t)g.tail_slots * D + so,
+                              min(16, p.Tb - 16 * warp), 0, lane);
+        } else {
+          stage_tail_chunk<D>(tb, tk, tk + G * D, p.Tb, warp, lane);
+        }
       }
     }
     // Claim a group (lane 0) and start its copy into stage `stg`; -1 once
@@ -1144,11 +1177,33 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     if (my_tail) {
       cp_async_wait_all();
       __syncwarp();
-      const Piece p = piece_s;
-      const unsigned char* tb =
-          C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
-      if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
-      else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+      unsigned char* tb = C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
+      if constexpr (!WIN) {
+        const Piece p = piece_s;
+        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+        else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+      } else {
+        const int Tc = min(16, piece_s.Tb - 16 * warp);
+        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+        else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+      }
+      // chunks warp + TAIL_CHUNKS, warp + 2 TAIL_CHUNKS, ... (a recent
+      // window only), each staged once the previous one is done
+      if constexpr (WIN)
+      for (int c = warp + C::TAIL_CHUNKS; 16 * c < piece_s.Tb; c += C::TAIL_CHUNKS) {
+        const Piece p = piece_s;
+        const __half* tk = reinterpret_cast<const __half*>(
+            a.cache + g.tails_off + ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.tail_bytes);
+        const int64_t so = tail_chunk_slot(p.ng * G, c, g.tail_slots) * D;
+        __syncwarp();   // every lane's reads of the stage are done
+        stage_tail_chunk<D>(tb, tk + so, tk + (int64_t)g.tail_slots * D + so,
+                            min(16, p.Tb - 16 * c), 0, lane);
+        cp_async_wait_all();
+        __syncwarp();
+        const int Tc = min(16, p.Tb - 16 * c);
+        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+        else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+      }
       if (!C::TAIL_EARLY) {   // the ring is free again: start its copies
         __syncwarp();
         cur = claim_into(head);
@@ -1416,14 +1471,21 @@ size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
 template <int D, int KB, int VB, int G, bool PK, bool WIDE>
 cudaError_t max_ctas_t(int* out) {
   using C = DecCfg<D, KB, VB, G, WIDE>;
-  auto kern = decode_kernel<D, KB, VB, G, PK, WIDE>;
   const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(64);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, sm);
-  if (e != cudaSuccess) return e;
+  // residency of the kernels with and without a recent window (the same
+  // launch bounds and shared memory: normally equal), the smaller one
+  int per_sm = 1 << 30;
+  for (auto kern : {decode_kernel<D, KB, VB, G, PK, WIDE, false>,
+                    decode_kernel<D, KB, VB, G, PK, WIDE, true>}) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, C::THREADS, sm);
+    if (e != cudaSuccess) return e;
+    per_sm = min(per_sm, n);
+  }
+  cudaError_t e;
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1439,14 +1501,16 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
   using C = DecCfg<D, KB, VB, G, WIDE>;
   if (g.block_bytes != C::BLK || g.sec_vmin != C::SEC_VMIN || g.sec_kscale != C::SEC_KSCALE)
     return cudaErrorInvalidValue;
-  auto kern = decode_kernel<D, KB, VB, G, PK, WIDE>;
+  const bool win = g.window > 0;
+  auto kern = win ? decode_kernel<D, KB, VB, G, PK, WIDE, true>
+                  : decode_kernel<D, KB, VB, G, PK, WIDE, false>;
   const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(a.n_seq);
-  static bool configured = false;   // attribute set once, before any capture
-  if (!configured) {
+  static bool configured[2] = {false, false};   // attribute set once, before any capture
+  if (!configured[win]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[win] = true;
   }
   {
     // a programmatic dependent of the previous kernel (it waits for it
@@ -1917,7 +1981,7 @@ cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
 // dominate), so the mma.sync kernel is the default.
 bool decode_tc_eligible(const Geom& g) {
   if (!(g.d == 128 && g.G == 32 && g.vb == 2 && (g.kb == 2 || g.kb == 4) && g.gqa <= 4 &&
-        g.slices == 1))
+        g.slices == 1 && g.window == 0))
     return false;
   const char* env = std::getenv("KVQ_DECODE_TC");
   return env && env[0] == '1';

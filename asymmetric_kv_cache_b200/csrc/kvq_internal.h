@@ -33,6 +33,7 @@ struct Geom {
   int32_t block_bytes;
   int32_t sec_kcodes, sec_kscale, sec_kmin, sec_vcodes, sec_vscale, sec_vmin;
   int64_t lens_off, counters_off, blocks_off, tails_off, tail_bytes, total_bytes;
+  int32_t window, tail_slots;   // R, and W = R + G slots of the fp16 tail ring
 };
 
 // Workspace of kvq_decode: [error word | per-unit split records | per-unit
@@ -46,6 +47,20 @@ struct WsLayout {
 };
 
 inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Groups of a sequence of L tokens that are quantized: those followed by at
+// least `window` newer tokens ("[Framework] The Asymmetric Key-Value Cache
+// Compression", §III and §V: the most recent tokens stay in fp16).  The
+// other L - G * groups tokens are the fp16 tail.
+__host__ __device__ inline int quantized_groups(int L, int G, int window) {
+  const int Lq = L - window;
+  return Lq > 0 ? Lq / G : 0;
+}
+// Decode slots of one unit: its groups plus one for a non-empty tail.
+__host__ __device__ inline int unit_slots(int L, int G, int window) {
+  const int ng = quantized_groups(L, G, window);
+  return ng + (L > ng * G ? 1 : 0);
+}
 
 // Fill g from a validated configuration (no checks here).
 inline void make_geom(const kvq_config& c, Geom* g) {
@@ -61,6 +76,8 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->max_seqs = c.max_seqs;
   g->max_tokens = c.max_tokens;
   g->max_groups = c.max_tokens / c.group;
+  g->window = c.window;
+  g->tail_slots = c.window + c.group;
   const int G = g->G, d = g->d, J = g->J;
   int off = 0;
   g->sec_kcodes = off; off += G * d * g->kb / 8;
@@ -78,7 +95,7 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->blocks_off = pos;
   pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->max_groups * g->block_bytes, 256);
   g->tails_off = pos;
-  g->tail_bytes = 4LL * G * d;  // K tail + V tail, fp16
+  g->tail_bytes = 4LL * g->tail_slots * d;  // K tail + V tail, fp16
   pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->tail_bytes, 256);
   g->total_bytes = pos;
 }

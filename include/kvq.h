@@ -24,9 +24,14 @@
  *              code = 0 when s == 0.
  * Key group: G consecutive tokens x one channel (G tokens from position 0 of
  * each sequence).  Value group: G consecutive channels of one token.
- * The n mod G newest tokens of each sequence (keys and values) sit in an
- * fp16 tail; when the tail reaches G tokens it is quantized as the next group
- * ("flush").  Query head h reads kv head h / (n_q_heads / n_kv_heads).
+ * The newest tokens of each sequence (keys and values) sit in an fp16 tail.
+ * With the recent window R = kvq_config.window (same page, §III and §V: the
+ * most recent 32 to 128 tokens stay in FP16), a group is quantized once R
+ * newer tokens follow it: N = G * floor(max(0, n - R) / G) tokens are
+ * quantized and the tail holds the other n - N, between R and R + G - 1 once
+ * n >= R; a tail that reaches R + G tokens has its oldest G quantized as the
+ * next group ("flush").  R = 0 gives the n mod G tail.  Query head h reads
+ * kv head h / (n_q_heads / n_kv_heads).
  *
  * Conventions
  * -----------
@@ -45,10 +50,12 @@
  *   lens   : int32 [max_seqs]                 device copy of the lengths
  *   tickets: int32 [max_seqs]                 append completion counters (0 at rest)
  *   blocks : [max_seqs][n_kv_heads][max_groups] group blocks of block_bytes
- *   tails  : [max_seqs][n_kv_heads] { K tail fp16 [G][d] token-major,
- *                                     V tail fp16 [G/2][d][2] token pairs }
- *            K tail slot (t, c) is element t*d + c; V tail slot (t, c) is
- *            element ((t/2)*d + c)*2 + t%2.
+ *   tails  : [max_seqs][n_kv_heads] { K tail fp16 [W][d] token-major,
+ *                                     V tail fp16 [W/2][d][2] token pairs }
+ *            a ring of W = R + G token slots: the token at sequence
+ *            position p sits in slot t = p mod W while it is in the tail
+ *            (t = p - N when R = 0).  K tail slot (t, c) is element t*d + c;
+ *            V tail slot (t, c) is element ((t/2)*d + c)*2 + t%2.
  * A group block holds, in this order (byte offsets in kvq_layout):
  *   key codes   G*d*kbits/8 bytes
  *   key scales  d fp16, key mins d fp16
@@ -117,6 +124,9 @@ typedef struct {
   int32_t max_seqs;        /* sequences the buffer holds, >= 1 */
   int32_t max_tokens;      /* capacity per sequence, >= 1 */
   int32_t layout_version;  /* must be KVQ_LAYOUT_VERSION (or 0 = current) */
+  int32_t window;          /* R: recent tokens kept in fp16 beyond the partial
+                              group; a multiple of 16 in [0, 1024]; 0 = the
+                              n mod G tail */
 } kvq_config;
 
 typedef struct {
@@ -127,9 +137,10 @@ typedef struct {
   uint64_t block_bytes;    /* one group block */
   uint64_t max_groups;     /* floor(max_tokens / G) blocks per (seq, kv head) */
   uint64_t tails_offset;   /* first tail */
-  uint64_t tail_bytes;     /* K tail + V tail of one (seq, kv head) = 4*G*d */
+  uint64_t tail_bytes;     /* K tail + V tail of one (seq, kv head) = 4*W*d */
   uint64_t kcodes_offset, kscale_offset, kmin_offset; /* within a block */
   uint64_t vcodes_offset, vscale_offset, vmin_offset; /* within a block */
+  uint64_t tail_slots;     /* W = window + G token slots per tail ring */
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache;
@@ -172,7 +183,7 @@ KVQ_API kvq_status kvq_reset(kvq_cache* cache, void* stream);
  * 16-byte aligned.  n_new: host array of n_seq non-negative counts.
  * Performs prefill quantization (whole groups straight from the input),
  * per-step appends into the fp16 tail and the flush of a tail that reaches
- * G tokens, all in one launch.  The kernel takes the current lengths from
+ * R + G tokens (its oldest G become a group), all in one launch.  The kernel takes the current lengths from
  * the device copy and advances it, so an append captured in a CUDA graph
  * may be replayed provided every n_new[b] < G (the launch shape then does
  * not depend on the lengths); after replays, kvq_sync_lengths refreshes the

@@ -18,7 +18,7 @@ def kvq():
 
 def oracle_cfg(spec) -> o.Config:
     return o.Config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim, spec.n_q_heads,
-                    spec.n_kv_heads)
+                    spec.n_kv_heads, window=getattr(spec, "window", 0))
 
 
 def to_device(x: np.ndarray, dtype: str) -> torch.Tensor:
@@ -51,12 +51,14 @@ def append_chunks(cache, chunks_k, chunks_v, dtype: str):
     cache.append(to_device(k, dtype), to_device(v, dtype), n_new)
 
 
-def expected_tail_mask(cfg: o.Config, T: int):
-    """Element masks of the defined slots of the fp16 tails (slots < T)."""
-    G, d = cfg.group, cfg.head_dim
-    mk = np.zeros(G * d, bool)
-    mv = np.zeros(G * d, bool)
-    for t in range(T):
+def expected_tail_mask(cfg: o.Config, N: int, T: int):
+    """Element masks of the defined slots of the fp16 tail rings: the slots of
+    positions N .. N + T - 1."""
+    W, d = cfg.tail_slots, cfg.head_dim
+    mk = np.zeros(W * d, bool)
+    mv = np.zeros(W * d, bool)
+    for p in range(N, N + T):
+        t = o.tail_slot(cfg, p)
         for c in range(d):
             mk[o.tail_key_index(t, c, d)] = True
             mv[o.tail_value_index(t, c, d)] = True
@@ -76,7 +78,7 @@ def check_cache_against_oracle(cache, hist_k, hist_v, seqs=None, group_sample=No
         n = hist_k[b].shape[0]
         assert lens[b] == n, (b, lens[b], n)
         assert dev_lens[b] == n, (b, dev_lens[b], n)
-        N, T = o.split_tokens(n, cfg.group)
+        N, T = o.split_tokens(n, cfg.group, cfg.window)
         ng = N // cfg.group
         gsel = np.arange(ng) if group_sample is None else np.asarray(group_sample(ng), np.int64)
         if len(gsel):
@@ -94,9 +96,9 @@ def check_cache_against_oracle(cache, hist_k, hist_v, seqs=None, group_sample=No
                         f"seq {b} head {h}: {len(bad)} bytes differ; first at group "
                         f"{gsel[g0]} byte {byte0}: got {got[g0, byte0]:#04x} want {want[h][g0, byte0]:#04x}")
         if T:
-            mk, mv = expected_tail_mask(cfg, T)
+            mk, mv = expected_tail_mask(cfg, N, T)
             for h in range(cfg.n_kv_heads):
-                tk, tv = o.tail_arrays(cfg, hist_k[b][N:, h], hist_v[b][N:, h])
+                tk, tv = o.tail_arrays(cfg, hist_k[b][N:, h], hist_v[b][N:, h], first=N)
                 gk, gv = cache.tail_halves(b, h)
                 gk = gk.cpu().numpy()
                 gv = gv.cpu().numpy()

@@ -63,6 +63,15 @@ def test_layout_matches_oracle_sections(kvq, kb, vb, G, d):
     assert ws > 0
 
 
+@pytest.mark.parametrize("G,R", [(32, 0), (32, 32), (32, 128), (64, 16), (64, 1024)])
+def test_tail_ring_size_from_library(kvq, G, R):
+    """The tail is a ring of R + G token slots (K and V fp16)."""
+    lay = kvq.layout_for(_cfg(kvq, group=G, window=R))
+    assert lay["tail_slots"] == o.Config(4, 2, G, 128, 32, 8, window=R).tail_slots == R + G
+    assert lay["tail_bytes"] == 4 * (R + G) * 128
+    assert lay["total_bytes"] >= lay["tails_offset"] + 8 * 8 * lay["tail_bytes"]
+
+
 def test_bytes_per_token_head_from_library(kvq):
     """128 B per token-head for K4/V2 G=32, 96 for K2/V2, 112 for K4/V2 G=64."""
     for kb, G, expect in ((4, 32, 128), (2, 32, 96), (4, 64, 112)):
@@ -74,6 +83,7 @@ def test_bytes_per_token_head_from_library(kvq):
     ("k_bits", 3), ("k_bits", 8), ("v_bits", 1), ("group", 16), ("group", 128),
     ("head_dim", 96), ("head_dim", 256), ("n_q_heads", 30), ("n_kv_heads", 0),
     ("max_seqs", 0), ("max_tokens", 0), ("layout_version", 2),
+    ("window", -16), ("window", 24), ("window", 1040),
 ])
 def test_bad_config_rejected(kvq, field, value):
     cfg = _cfg(kvq)
