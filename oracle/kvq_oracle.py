@@ -35,6 +35,11 @@ Readings where the pages are silent (each is listed in the design notes):
   (all n tokens while n < R); R = 0 is the n mod G tail above.  The tail is a
   ring of R + G token slots: token p sits in slot p mod (R + G), so tokens
   never move while they wait (our layout; the pages do not store it).
+* sink window S (InnerQ abstract, page "WUSH-KV: KV Cache Quantization with
+  Data-Adaptive Transforms", third abstract: high-precision windows for the
+  recent tokens and for the attention-sink tokens): the first S tokens of a
+  sequence stay in fp16; key groups are cut from position S on, and the
+  recent window applies to the tokens after the sink.
 * GQA: query head h reads kv head floor(h / (Hq / Hkv)).
 * attention is evaluated in float64 on the dequantized cache
   x_hat = code * s + z (tail tokens exactly as stored in fp16).
@@ -70,6 +75,7 @@ class Config:
     max_seqs: int = 1
     max_tokens: int = 0
     window: int = 0      # R: recent tokens kept in fp16 beyond the partial group
+    sink: int = 0        # S: first tokens of a sequence kept in fp16
 
     @property
     def tail_slots(self) -> int:   # W = R + G slots of the fp16 tail ring
@@ -455,6 +461,16 @@ def split_tokens(n: int, group: int, window: int = 0):
     return N, n - N
 
 
+def segments(cfg: Config, n: int):
+    """(Sb, Nq, T) for a sequence of n tokens: Sb = min(n, S) sink tokens
+    (positions 0 .. Sb-1, fp16), Nq quantized tokens (positions Sb ..
+    Sb+Nq-1, whole groups cut from position S), T tail tokens (the rest,
+    fp16).  The tokens after the sink split as in ``split_tokens``."""
+    Sb = min(n, cfg.sink)
+    Nq, T = split_tokens(n - Sb, cfg.group, cfg.window)
+    return Sb, Nq, T
+
+
 def tail_slot(cfg: Config, p: int) -> int:
     """Slot of the fp16 tail ring that token position p occupies while it is
     in the tail: p mod (R + G)."""
@@ -470,10 +486,10 @@ def quantize_group(cfg: Config, k16: np.ndarray, v16: np.ndarray):
 
 
 def grouped(cfg: Config, x16: np.ndarray) -> np.ndarray:
-    """[n, Hkv, d] token history -> [Hkv, N/G, G, d] quantized groups."""
+    """[n, Hkv, d] token history -> [Hkv, Nq/G, G, d] quantized groups."""
     G = cfg.group
-    N, _ = split_tokens(x16.shape[0], G, cfg.window)
-    x = np.asarray(x16[:N], np.float16).reshape(N // G, G, x16.shape[1], x16.shape[2])
+    Sb, Nq, _ = segments(cfg, x16.shape[0])
+    x = np.asarray(x16[Sb:Sb + Nq], np.float16).reshape(Nq // G, G, x16.shape[1], x16.shape[2])
     return x.transpose(2, 0, 1, 3)
 
 
@@ -484,16 +500,20 @@ def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True
     ``groups``: (kc, ks, kz, vc, vs, vz) with a leading [Hkv, n_groups] shape,
     ``blocks``: [Hkv, n_groups, block_bytes] uint8 (if ``pack``),
     ``tail_k``/``tail_v``: [Hkv, T, d] fp16 tail tokens (positions N .. n-1 in
-    order), and N, T.
+    order), ``sink_k``/``sink_v``: [Hkv, Sb, d] fp16 sink tokens (positions
+    0 .. Sb-1), N (the first tail position, Sb + Nq), T, Sb and Nq.
     """
     n = k16.shape[0]
-    N, T = split_tokens(n, cfg.group, cfg.window)
+    Sb, Nq, T = segments(cfg, n)
+    N = Sb + Nq
     q = quantize_group(cfg, grouped(cfg, k16), grouped(cfg, v16))
-    out = {"N": N, "T": T, "groups": q}
+    out = {"N": N, "T": T, "Sb": Sb, "Nq": Nq, "groups": q}
     if pack:
         out["blocks"] = pack_blocks(cfg, *q)
     out["tail_k"] = np.ascontiguousarray(np.asarray(k16[N:], np.float16).transpose(1, 0, 2))
     out["tail_v"] = np.ascontiguousarray(np.asarray(v16[N:], np.float16).transpose(1, 0, 2))
+    out["sink_k"] = np.ascontiguousarray(np.asarray(k16[:Sb], np.float16).transpose(1, 0, 2))
+    out["sink_v"] = np.ascontiguousarray(np.asarray(v16[:Sb], np.float16).transpose(1, 0, 2))
     return out
 
 
@@ -515,18 +535,16 @@ def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray, first: int 
 
 def dequantized_cache(cfg: Config, k16: np.ndarray, v16: np.ndarray):
     """K_hat, V_hat [n, Hkv, d] float64: quantized groups dequantized, the
-    tail exactly as stored (fp16)."""
+    sink and the tail exactly as stored (fp16)."""
     n, hkv, d = k16.shape
     img = cache_image(cfg, k16, v16, pack=False)
-    N = img["N"]
+    Sb, Nq, N = img["Sb"], img["Nq"], img["N"]
     kc, ks, kz, vc, vs, vz = img["groups"]
-    kh = np.zeros((n, hkv, d))
-    vh = np.zeros((n, hkv, d))
-    # [Hkv, ng, G, d] -> [N, Hkv, d]
-    kh[:N] = dequantize_keys(kc, ks, kz).transpose(1, 2, 0, 3).reshape(N, hkv, d)
-    vh[:N] = dequantize_values(vc, vs, vz, cfg.group).transpose(1, 2, 0, 3).reshape(N, hkv, d)
-    kh[N:] = np.asarray(k16[N:], np.float64)
-    vh[N:] = np.asarray(v16[N:], np.float64)
+    kh = np.asarray(k16, np.float64).copy()   # sink and tail: the fp16 values
+    vh = np.asarray(v16, np.float64).copy()
+    # [Hkv, ng, G, d] -> [Nq, Hkv, d]
+    kh[Sb:N] = dequantize_keys(kc, ks, kz).transpose(1, 2, 0, 3).reshape(Nq, hkv, d)
+    vh[Sb:N] = dequantize_values(vc, vs, vz, cfg.group).transpose(1, 2, 0, 3).reshape(Nq, hkv, d)
     return kh, vh
 
 
