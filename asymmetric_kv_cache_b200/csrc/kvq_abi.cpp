@@ -77,6 +77,8 @@ kvq_status validate_config(const kvq_config* c) {
                 c->max_tokens);
   if (c->window < 0 || c->window > 1024 || c->window % 16 != 0)
     return fail(KVQ_ERR_CONFIG, "window must be a multiple of 16 in [0, 1024] (got %d)", c->window);
+  if (c->sink < 0 || c->sink > 1024)
+    return fail(KVQ_ERR_CONFIG, "sink must be in [0, 1024] (got %d)", c->sink);
   // decode addresses slots (groups + tail) of all units with 32-bit prefixes
   const int64_t slices = (c->n_q_heads / c->n_kv_heads + kvq::kHeadsPerSlice - 1) / kvq::kHeadsPerSlice;
   const int64_t slots = (int64_t)c->max_seqs * c->n_kv_heads * slices * (c->max_tokens / c->group + 1);
@@ -101,6 +103,9 @@ void fill_layout(const kvq::Geom& g, kvq_layout* o) {
   o->tails_offset = g.tails_off;
   o->tail_bytes = g.tail_bytes;
   o->tail_slots = (uint64_t)g.tail_slots;
+  o->sinks_offset = (uint64_t)g.sinks_off;
+  o->sink_bytes = (uint64_t)g.sink_bytes;
+  o->sink_slots = (uint64_t)g.sink_slots;
   o->kcodes_offset = g.sec_kcodes;
   o->kscale_offset = g.sec_kscale;
   o->kmin_offset = g.sec_kmin;
@@ -237,8 +242,8 @@ kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype 
       const int len0 = cache->lens[b], nn = n_new[b];
       // groups this append completes (the kernel recomputes them from the
       // device lengths; for nn < G at most one, whatever the length)
-      const int F = kvq::quantized_groups(len0 + nn, g.G, g.window) -
-                    kvq::quantized_groups(len0, g.G, g.window);
+      const int F = kvq::quantized_groups_s(len0 + nn, g.G, g.window, g.sink) -
+                    kvq::quantized_groups_s(len0, g.G, g.window, g.sink);
       seqs.task_prefix[i] = tasks;
       seqs.row_off[i] = (int32_t)row;
       seqs.n_new[i] = nn;
@@ -264,9 +269,10 @@ namespace {
 int64_t choose_grid(const kvq::Geom& g, const int32_t* lens, int n_seq, int64_t slots, int cap) {
   int64_t grid = std::min<int64_t>(slots, cap);
   const int64_t units = (int64_t)n_seq * g.hkv * g.slices;
-  const int w0 = kvq::unit_slots(lens[0], g.G, g.window);
+  const int w0 = kvq::unit_slots_s(lens[0], g.G, g.window, g.sink);
   bool equal = true;
-  for (int b = 1; b < n_seq && equal; ++b) equal = kvq::unit_slots(lens[b], g.G, g.window) == w0;
+  for (int b = 1; b < n_seq && equal; ++b)
+    equal = kvq::unit_slots_s(lens[b], g.G, g.window, g.sink) == w0;
   if (equal && units <= cap) {
     const int64_t alt = std::min<int64_t>(slots, units * (cap / units));
     if (alt * 5 >= (int64_t)cap * 4) grid = alt;
@@ -298,7 +304,7 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     if (env_cap > 0) cap = std::min(cap, env_cap);
     int64_t slots = 0;
     for (int b = s0; b < s0 + ns; ++b)
-      slots += (int64_t)g.hkv * g.slices * kvq::unit_slots(lens[b], g.G, g.window);
+      slots += (int64_t)g.hkv * g.slices * kvq::unit_slots_s(lens[b], g.G, g.window, g.sink);
     const int64_t grid = std::min(max_grid, choose_grid(g, lens + s0, ns, slots, cap));
     kvq::DecodeArgs a;
     a.cache = cache_buf;

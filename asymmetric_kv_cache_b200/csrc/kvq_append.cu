@@ -16,7 +16,11 @@
 // the tail never move.  A slot whose old token a group task reads is
 // rewritten, if a new tail token maps to it, by that same task after its
 // read; every other new tail token is written by the sequence's first task.
-// So no slot is read and written by two CTAs.
+// So no slot is read and written by two CTAs.  With a sink window of S
+// tokens (InnerQ abstract, page "WUSH-KV: KV Cache Quantization with
+// Data-Adaptive Transforms") the first S tokens of a sequence go to an fp16
+// sink area instead, and all of the above applies to the positions after
+// it (q = p - S).
 //
 // Every CTA reads the sequence's current length from the device copy when
 // it starts; the last CTA of the sequence to finish (atomic ticket in the
@@ -183,16 +187,21 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   const int nn = s.n_new[b];
   const int seq_ctas = (s.task_prefix[b + 1] - s.task_prefix[b]) * gridDim.y;
   const int W = g.tail_slots;      // ring slots of the tail: R + G
-  const int N0 = G * quantized_groups(len0, G, g.window);
-  const int T0 = len0 - N0;        // tail length before
   const int n1 = len0 + nn;
-  const int N1 = G * quantized_groups(n1, G, g.window);
+  // positions after the sink (q = p - S): a0 before, a1 after this append;
+  // the first nsink new tokens (input rows 0 .. nsink-1) go to the sink
+  const int a0 = max(len0 - g.sink, 0);
+  const int a1 = max(n1 - g.sink, 0);
+  const int nsink = max(min(n1, g.sink) - len0, 0);
+  const int N0 = G * quantized_groups(a0, G, g.window);
+  const int T0 = a0 - N0;          // tail length before
+  const int N1 = G * quantized_groups(a1, G, g.window);
   const int F = (N1 - N0) / G;     // groups completed by this append
   const int64_t row0 = s.row_off[b];
   const int64_t unit = (int64_t)seq * g.hkv + kvh;
   __half* tailk = reinterpret_cast<__half*>(cache + g.tails_off + unit * g.tail_bytes);
   __half* tailv = tailk + (int64_t)W * D;
-  const int base0 = N0 % W;        // ring slot of position N0
+  const int base0 = N0 % W;        // ring slot of post-sink position N0
   auto in_idx = [&](int64_t r, int c) { return ((row0 + r) * g.hkv + kvh) * D + c; };
   // A replayed capture can ask for more than the capacity, which the host
   // could not check: such an append writes nothing and the length stays.
@@ -211,16 +220,28 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   }
 
   constexpr int CPR = D / 8;   // 16-byte fp16 chunks per token row
+  // new sink tokens: input row j -> sink slot len0 + j (nobody reads them here)
+  auto write_sink = [&]() {
+    __half* sinkk = reinterpret_cast<__half*>(cache + g.sinks_off + unit * g.sink_bytes);
+    __half* sinkv = sinkk + (int64_t)g.sink_slots * D;
+    for (int ci = tid; ci < nsink * CPR; ci += blockDim.x) {
+      const int j = ci / CPR, cc = ci % CPR;
+      store_tail8(sinkk, sinkv, len0 + j, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
+                  load8_fp16(vin, in_idx(j, 8 * cc), dtype));
+    }
+  };
   if (F == 0) {
-    // no group completes: new token len0 + j goes to ring slot
-    // (len0 + j) mod W, which holds no tail token (the tail stays below W)
+    // no group completes: post-sink position a0 + j (input row nsink + j) goes
+    // to ring slot (a0 + j) mod W, which holds no tail token (the tail
+    // stays below W)
+    write_sink();
     const int sl0 = (base0 + T0) % W;
-    for (int ci = tid; ci < nn * CPR; ci += blockDim.x) {
+    for (int ci = tid; ci < (a1 - a0) * CPR; ci += blockDim.x) {
       const int j = ci / CPR, cc = ci % CPR;
       int sl = sl0 + j;
       sl -= (sl >= W) ? W : 0;
-      store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
-                  load8_fp16(vin, in_idx(j, 8 * cc), dtype));
+      store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(nsink + j, 8 * cc), dtype),
+                  load8_fp16(vin, in_idx(nsink + j, 8 * cc), dtype));
     }
     finish();
     return;
@@ -230,9 +251,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     return;
   }
 
-  // ---- load the group: position N0 + u (u = tau*G + r) is old tail
-  // token u (ring slot (N0 + u) mod W) or input row u - T0; 16-byte chunks,
-  // every load of a thread issued before its stores
+  // ---- load the group: post-sink position N0 + u (u = tau*G + r) is old
+  // tail token u (ring slot (N0 + u) mod W) or input row nsink + u - T0;
+  // 16-byte chunks, every load of a thread issued before its stores
   {
     constexpr int NCH = G * CPR / 128;   // chunks per thread (K and V each)
     uint4 kx[NCH], vx[NCH];
@@ -246,8 +267,8 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
         kx[j] = *reinterpret_cast<const uint4*>(tailk + sl * D + 8 * cc);
         vx[j] = tail_v8(tailv, sl, cc, D);
       } else {
-        kx[j] = load8_fp16(kin, in_idx(u - T0, 8 * cc), dtype);
-        vx[j] = load8_fp16(vin, in_idx(u - T0, 8 * cc), dtype);
+        kx[j] = load8_fp16(kin, in_idx(nsink + u - T0, 8 * cc), dtype);
+        vx[j] = load8_fp16(vin, in_idx(nsink + u - T0, 8 * cc), dtype);
       }
     }
 #pragma unroll
@@ -454,27 +475,29 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     for (int i = tid; i < G * C::J / 2; i += blockDim.x) dst[i] = src[i];
   }
 
-  // ---- the new tail: positions [A, n1), all new tokens (input rows p -
-  // len0).  Ring residue rr = (p - N0) mod W: rr < T0 is the slot of old
-  // tail token N0 + rr, which this append quantizes in task rr / G (that
-  // task read it before the barrier above), so that task writes the slot;
-  // residues T0 .. W-1 hold no old tail token and task 0 writes them.  Each
-  // residue occurs at most once in [A, n1) (the new tail is shorter than W).
+  // ---- the new tail: post-sink positions [A, a1), all new tokens (input
+  // rows nsink + q - a0).  Ring residue rr = (q - N0) mod W: rr < T0 is the
+  // slot of old tail token N0 + rr, which this append quantizes in task
+  // rr / G (that task read it before the barrier above), so that task
+  // writes the slot; residues T0 .. W-1 hold no old tail token and task 0
+  // writes them.  Each residue occurs at most once in [A, a1) (the new tail
+  // is shorter than W).  Task 0 also writes the new sink tokens.
+  if (tau == 0) write_sink();
   {
-    const int A = max(N1, len0);
+    const int A = max(N1, a0);
     const int r_lo = tau * G;
     const int r_hi = min(T0, r_lo + G);
     auto write_residues = [&](int lo, int hi) {
       for (int ci = tid; ci < (hi - lo) * CPR; ci += blockDim.x) {
         const int rr = lo + ci / CPR, cc = ci % CPR;
-        // the position p >= A with p = N0 + rr (mod W)
+        // the post-sink position q >= A with q = N0 + rr (mod W)
         int off = (N0 + rr - A) % W;
         off += (off < 0) ? W : 0;
-        const int p = A + off;
-        if (p < n1) {
+        const int q = A + off;
+        if (q < a1) {
           int sl = base0 + rr;
           sl -= (sl >= W) ? W : 0;
-          const int64_t r = (int64_t)p - len0;
+          const int64_t r = (int64_t)nsink + q - a0;
           store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(r, 8 * cc), dtype),
                       load8_fp16(vin, in_idx(r, 8 * cc), dtype));
         }

@@ -114,7 +114,8 @@ struct DecCfg {
   static_assert((MERGE_FLOATS + (NW + 2) * kHeadsPerSlice) * 4 <= RING,
                 "merge area must fit in the ring");
   // The tail, in chunks of 16 tokens (< G/16 chunks without a recent
-  // window, up to (R + G - 1)/16 with one): chunk c belongs to warp
+  // window, up to (R + G - 1)/16 with one, after the sink's chunks when
+  // there is a sink window): chunk c belongs to warp
   // c mod TAIL_CHUNKS, which stages its first chunk when the piece starts
   // (its copy latency hidden behind the query's) and processes its chunks
   // one after another before claiming groups.  For 32-token groups the
@@ -356,8 +357,8 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
 // Decode slots of a unit with L tokens: its quantized groups plus one for a
 // non-empty tail (the window-free form when WIN is false).
 template <int G, bool WIN>
-__device__ __forceinline__ int dec_unit_slots(int L, int window) {
-  if constexpr (WIN) return unit_slots(L, G, window);
+__device__ __forceinline__ int dec_unit_slots(int L, const Geom& g) {
+  if constexpr (WIN) return unit_slots_s(L, G, g.window, g.sink);
   else return L / G + (L % G ? 1 : 0);
 }
 
@@ -367,6 +368,36 @@ __device__ __forceinline__ int dec_unit_slots(int L, int window) {
 // a chunk never wraps.
 __device__ __forceinline__ int tail_chunk_slot(int first, int c, int W) {
   return (first + 16 * c) % W;
+}
+
+// Where fp16 chunk c (16 tokens) of a unit lives, for caches with a sink
+// and/or a recent window: chunks 0 .. ns-1 are the sink (tokens 16c ..,
+// ns = ceil(min(L, sink) / 16)), the rest the tail ring's chunks (tail chunk
+// c - ns starts at ring slot (ng G + 16 (c - ns)) mod W, positions counted
+// after the sink).  Returns the key and value base pointers and the chunk's
+// token count.
+template <int D, int G>
+__device__ __forceinline__ int fp16_chunk_src(const Geom& g, const unsigned char* cache,
+                                              int64_t ui, int L, int ng, int Tb, int c,
+                                              const __half*& k, const __half*& v) {
+  const int Sb = min(L, g.sink);
+  const int ns = (Sb + 15) / 16;
+  if (c < ns) {
+    const __half* sk = reinterpret_cast<const __half*>(cache + g.sinks_off + ui * g.sink_bytes);
+    k = sk + (int64_t)16 * c * D;
+    v = sk + (int64_t)g.sink_slots * D + (int64_t)16 * c * D;
+    return min(16, Sb - 16 * c);
+  }
+  const int ct = c - ns;
+  const __half* tk = reinterpret_cast<const __half*>(cache + g.tails_off + ui * g.tail_bytes);
+  const int64_t so = (int64_t)tail_chunk_slot(ng * G, ct, g.tail_slots) * D;
+  k = tk + so;
+  v = tk + (int64_t)g.tail_slots * D + so;
+  return min(16, Tb - 16 * ct);
+}
+// Chunks of the fp16 slot: the sink's, then the tail's.
+__device__ __forceinline__ int fp16_chunks(const Geom& g, int L, int Tb) {
+  return (min(L, g.sink) + 15) / 16 + (Tb + 15) / 16;
 }
 
 // Issue the cp.async copies of tail chunk kv (16 tokens: key rows and
@@ -962,13 +993,19 @@ __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix
   p.b = find_seq(prefix, n_seq, pos);
   p.L = slen[p.b];
   if constexpr (WIN) {
-    const int Lq = p.L - g.window;   // groups leave the newest `window` tokens in fp16
+    // the first min(L, sink) tokens stay in fp16; groups after them leave
+    // the newest `window` tokens in fp16; the sink and the tail share the
+    // unit's last (fp16) slot, Tb counts the tail alone
+    const int Sb = min(p.L, g.sink);
+    const int Lq = p.L - Sb - g.window;
     p.ng = Lq <= 0 ? 0 : G ? Lq / G : Lq / g.G;
+    p.Tb = p.L - Sb - p.ng * (G ? G : g.G);
+    p.wb = p.ng + (p.L > p.ng * (G ? G : g.G) ? 1 : 0);
   } else {
     p.ng = G ? p.L / G : p.L / g.G;
+    p.Tb = p.L - p.ng * (G ? G : g.G);
+    p.wb = p.ng + (p.Tb ? 1 : 0);
   }
-  p.Tb = p.L - p.ng * (G ? G : g.G);
-  p.wb = p.ng + (p.Tb ? 1 : 0);
   const int local = pos - prefix[p.b];
   const int uis = local / p.wb;
   p.slot0 = local - uis * p.wb;
@@ -982,8 +1019,9 @@ __device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix
 }
 
 // WIN: compiled for caches with a recent window (tails of up to R + G - 1
-// tokens in a ring of R + G slots); the kernels without it keep the
-// single-chunk-per-warp tail and its register budget.
+// tokens in a ring of R + G slots) and/or a sink window (the first S tokens
+// in an fp16 area, folded in with the tail); the kernels without it keep
+// the single-chunk-per-warp tail and its register budget.
 template <int D, int KB, int VB, int G, bool PK, bool WIDE, bool WIN>
 __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
                                   DecCfg<D, KB, VB, G, WIDE>::MIN_BLOCKS)
@@ -1032,7 +1070,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     // the way to the first copies)
     if (warp == 0) {
       const int L = lane < n_seq ? lens[lane] : 0;
-      const int32_t run = per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
+      const int32_t run = per_seq_units * dec_unit_slots<G, WIN>(L, g);
       int32_t incl = run;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1050,7 +1088,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     int32_t run = 0;
     for (int bb = b0; bb < b1; ++bb) {
       const int L = lens[bb];
-      run += per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
+      run += per_seq_units * dec_unit_slots<G, WIN>(L, g);
     }
     // exclusive scan of the per-thread sums across the block
     int32_t incl = run;
@@ -1066,7 +1104,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     int32_t acc = base + incl - run;
     for (int bb = b0; bb < b1; ++bb) {
       const int L = lens[bb];
-      acc += per_seq_units * dec_unit_slots<G, WIN>(L, g.window);
+      acc += per_seq_units * dec_unit_slots<G, WIN>(L, g);
       prefix[bb + 1] = acc;
       slen[bb] = L;
     }
@@ -1115,8 +1153,11 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
       ngr = max(0, min(p.slot1, p.ng) - p.slot0);
       nh = p.nh;
-      my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng && warp * 16 < p.Tb;
-      if constexpr (WIN) my_tail = my_tail && warp < C::TAIL_CHUNKS;
+      if constexpr (WIN)
+        my_tail = ok && p.slot1 == p.wb && p.slot0 <= p.ng && warp < C::TAIL_CHUNKS &&
+                  warp < fp16_chunks(g, p.L, p.Tb);
+      else
+        my_tail = ok && p.Tb > 0 && p.slot1 == p.wb && p.slot0 <= p.ng && warp * 16 < p.Tb;
       // the unit's raw query rows first, so that they are not queued behind
       // the group blocks
       if (tid == 0) {
@@ -1134,9 +1175,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
             a.cache + g.tails_off + ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.tail_bytes);
         unsigned char* tb = C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
         if constexpr (WIN) {
-          const int64_t so = tail_chunk_slot(p.ng * G, warp, g.tail_slots) * D;
-          stage_tail_chunk<D>(tb, tk + so, tk + (int64_t)g.tail_slots * D + so,
-                              min(16, p.Tb - 16 * warp), 0, lane);
+          const __half *ck, *cv;
+          const int Tc = fp16_chunk_src<D, G>(g, a.cache, (int64_t)(a.seq0 + p.b) * g.hkv + p.kvh,
+                                              p.L, p.ng, p.Tb, warp, ck, cv);
+          stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
         } else {
           stage_tail_chunk<D>(tb, tk, tk + G * D, p.Tb, warp, lane);
         }
@@ -1183,26 +1225,25 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
         else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
       } else {
-        const int Tc = min(16, piece_s.Tb - 16 * warp);
-        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
-        else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
-      }
-      // chunks warp + TAIL_CHUNKS, warp + 2 TAIL_CHUNKS, ... (a recent
-      // window only), each staged once the previous one is done
-      if constexpr (WIN)
-      for (int c = warp + C::TAIL_CHUNKS; 16 * c < piece_s.Tb; c += C::TAIL_CHUNKS) {
+        // fp16 chunks warp, warp + TAIL_CHUNKS, ... (sink chunks first, then
+        // the tail ring's), each staged once the previous one is done
         const Piece p = piece_s;
-        const __half* tk = reinterpret_cast<const __half*>(
-            a.cache + g.tails_off + ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.tail_bytes);
-        const int64_t so = tail_chunk_slot(p.ng * G, c, g.tail_slots) * D;
-        __syncwarp();   // every lane's reads of the stage are done
-        stage_tail_chunk<D>(tb, tk + so, tk + (int64_t)g.tail_slots * D + so,
-                            min(16, p.Tb - 16 * c), 0, lane);
-        cp_async_wait_all();
-        __syncwarp();
-        const int Tc = min(16, p.Tb - 16 * c);
-        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
-        else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+        const int64_t ui = (int64_t)(a.seq0 + p.b) * g.hkv + p.kvh;
+        const int nck = fp16_chunks(g, p.L, p.Tb);
+        for (int c = warp;;) {
+          const __half *ck, *cv;
+          const int Tc = fp16_chunk_src<D, G>(g, a.cache, ui, p.L, p.ng, p.Tb, c, ck, cv);
+          if (c != warp) {
+            __syncwarp();   // every lane's reads of the stage are done
+            stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
+            cp_async_wait_all();
+            __syncwarp();
+          }
+          if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+          else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+          c += C::TAIL_CHUNKS;
+          if (c >= nck) break;
+        }
       }
       if (!C::TAIL_EARLY) {   // the ring is free again: start its copies
         __syncwarp();
@@ -1501,7 +1542,7 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
   using C = DecCfg<D, KB, VB, G, WIDE>;
   if (g.block_bytes != C::BLK || g.sec_vmin != C::SEC_VMIN || g.sec_kscale != C::SEC_KSCALE)
     return cudaErrorInvalidValue;
-  const bool win = g.window > 0;
+  const bool win = g.window > 0 || g.sink > 0;
   auto kern = win ? decode_kernel<D, KB, VB, G, PK, WIDE, true>
                   : decode_kernel<D, KB, VB, G, PK, WIDE, false>;
   const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(a.n_seq);
@@ -1981,7 +2022,7 @@ cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
 // dominate), so the mma.sync kernel is the default.
 bool decode_tc_eligible(const Geom& g) {
   if (!(g.d == 128 && g.G == 32 && g.vb == 2 && (g.kb == 2 || g.kb == 4) && g.gqa <= 4 &&
-        g.slices == 1 && g.window == 0))
+        g.slices == 1 && g.window == 0 && g.sink == 0))
     return false;
   const char* env = std::getenv("KVQ_DECODE_TC");
   return env && env[0] == '1';

@@ -34,6 +34,8 @@ struct Geom {
   int32_t sec_kcodes, sec_kscale, sec_kmin, sec_vcodes, sec_vscale, sec_vmin;
   int64_t lens_off, counters_off, blocks_off, tails_off, tail_bytes, total_bytes;
   int32_t window, tail_slots;   // R, and W = R + G slots of the fp16 tail ring
+  int32_t sink, sink_slots;     // S, and SW = S rounded up to 16 sink slots
+  int64_t sinks_off, sink_bytes;
 };
 
 // Workspace of kvq_decode: [error word | per-unit split records | per-unit
@@ -61,6 +63,15 @@ __host__ __device__ inline int unit_slots(int L, int G, int window) {
   const int ng = quantized_groups(L, G, window);
   return ng + (L > ng * G ? 1 : 0);
 }
+// With a sink window of S tokens: the first min(L, S) tokens stay in fp16,
+// the rule above applies to the rest; the sink shares the tail's slot.
+__host__ __device__ inline int quantized_groups_s(int L, int G, int window, int sink) {
+  return quantized_groups(L > sink ? L - sink : 0, G, window);
+}
+__host__ __device__ inline int unit_slots_s(int L, int G, int window, int sink) {
+  const int ng = quantized_groups_s(L, G, window, sink);
+  return ng + (L > ng * G ? 1 : 0);
+}
 
 // Fill g from a validated configuration (no checks here).
 inline void make_geom(const kvq_config& c, Geom* g) {
@@ -78,6 +89,8 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->max_groups = c.max_tokens / c.group;
   g->window = c.window;
   g->tail_slots = c.window + c.group;
+  g->sink = c.sink;
+  g->sink_slots = (c.sink + 15) / 16 * 16;
   const int G = g->G, d = g->d, J = g->J;
   int off = 0;
   g->sec_kcodes = off; off += G * d * g->kb / 8;
@@ -97,6 +110,9 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->tails_off = pos;
   g->tail_bytes = 4LL * g->tail_slots * d;  // K tail + V tail, fp16
   pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->tail_bytes, 256);
+  g->sinks_off = pos;
+  g->sink_bytes = 4LL * g->sink_slots * d;  // K sink + V sink, fp16
+  pos = align_up(pos + (int64_t)c.max_seqs * c.n_kv_heads * g->sink_bytes, 256);
   g->total_bytes = pos;
 }
 

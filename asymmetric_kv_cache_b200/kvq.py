@@ -34,14 +34,15 @@ LAYOUT_VERSION = 1
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "k_bits", "v_bits", "group", "head_dim", "n_q_heads", "n_kv_heads",
-        "max_seqs", "max_tokens", "layout_version", "window")]
+        "max_seqs", "max_tokens", "layout_version", "window", "sink")]
 
 
 class KvqLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "total_bytes", "lens_offset", "counters_offset", "blocks_offset", "block_bytes", "max_groups",
         "tails_offset", "tail_bytes", "kcodes_offset", "kscale_offset", "kmin_offset",
-        "vcodes_offset", "vscale_offset", "vmin_offset", "tail_slots")]
+        "vcodes_offset", "vscale_offset", "vmin_offset", "tail_slots", "sinks_offset",
+        "sink_bytes", "sink_slots")]
 
 
 _c_status = ctypes.c_int32
@@ -103,9 +104,9 @@ def check(status: int, where: str) -> None:
 
 
 def make_config(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                max_tokens, window=0) -> KvqConfig:
+                max_tokens, window=0, sink=0) -> KvqConfig:
     return KvqConfig(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                     max_tokens, LAYOUT_VERSION, window)
+                     max_tokens, LAYOUT_VERSION, window, sink)
 
 
 def required_bytes(cfg: KvqConfig) -> tuple[int, int]:
@@ -146,6 +147,7 @@ class CacheSpec:
     max_seqs: int
     max_tokens: int
     window: int = 0     # R: recent tokens kept in fp16 beyond the partial group
+    sink: int = 0       # S: first tokens of each sequence kept in fp16
 
 
 class KVQCache:
@@ -159,7 +161,7 @@ class KVQCache:
         self.spec = spec
         self.cfg = make_config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim,
                                spec.n_q_heads, spec.n_kv_heads, spec.max_seqs, spec.max_tokens,
-                               spec.window)
+                               spec.window, spec.sink)
         cache_bytes, ws_bytes = required_bytes(self.cfg)
         self.buffer = torch.empty(cache_bytes, dtype=torch.uint8, device=device)
         self.workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
@@ -259,6 +261,13 @@ class KVQCache:
         base = L["tails_offset"] + (seq * self.spec.n_kv_heads + kv_head) * L["tail_bytes"]
         raw = self.buffer[base: base + L["tail_bytes"]].view(torch.float16)
         return raw[: W * d], raw[W * d: 2 * W * d]
+
+    def sink_halves(self, seq: int, kv_head: int) -> tuple[torch.Tensor, torch.Tensor]:
+        L = self.layout
+        SW, d = L["sink_slots"], self.spec.head_dim
+        base = L["sinks_offset"] + (seq * self.spec.n_kv_heads + kv_head) * L["sink_bytes"]
+        raw = self.buffer[base: base + L["sink_bytes"]].view(torch.float16)
+        return raw[: SW * d], raw[SW * d: 2 * SW * d]
 
     def device_lengths(self) -> torch.Tensor:
         L = self.layout

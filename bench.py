@@ -324,6 +324,8 @@ def run_ours(args, rank, world, device):
     long_ctx = run_long_context(stream, device) if args.long_context else None
     window = (run_long_context(stream, device, window=args.window, fp16=False)
               if args.long_context and args.window else None)
+    sinkw = (run_long_context(stream, device, window=args.window, sink=args.sink, fp16=False)
+             if args.long_context and args.sink else None)
 
     for cache in caches:
         if cache.workspace_status(stream) != 0:
@@ -347,7 +349,7 @@ def run_ours(args, rank, world, device):
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
         "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K, "long_ctx": long_ctx,
-        "window": window,
+        "window": window, "sink": sinkw,
     }
 
 
@@ -389,24 +391,26 @@ def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
             "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
 
 
-def run_long_context(stream, device, iters=100, window=0, fp16=True):
+def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0):
     """Decode alone on the 128k-token long-context workload (batch 1, 32 q /
     8 kv heads, d 128, K2/V2, G 32): the configuration the HBM-roofline
     target is stated on.  Copies of the cache (> 3x L2 in total) are
     rotated so that every decode reads HBM; CUDA events on the launch
     stream around `iters` decodes.  The unquantized comparison kernel runs
     the same shape (fp16 K/V, two copies) when `fp16`.  `window` > 0 keeps
-    that many recent tokens in fp16 beyond the partial group (their bytes
-    counted at 4d per token-head)."""
+    that many recent tokens in fp16 beyond the partial group, `sink` > 0 the
+    first tokens of the sequence (their bytes counted at 4d per
+    token-head)."""
     import torch
     from asymmetric_kv_cache_b200 import inputs, kvq
     w = inputs.WORKLOADS["long_ctx"]()
     n = w.lens[0]
     spec = kvq.CacheSpec(w.k_bits, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
-                         w.batch, n, window=window)
+                         w.batch, n, window=window, sink=sink)
     G, d = w.group, w.head_dim
     blk = G * d * (w.k_bits + w.v_bits) // 8 + 8 * d
-    nq = G * ((n - window) // G) if n > window else 0   # quantized tokens
+    after = n - min(n, sink)                                  # tokens after the sink
+    nq = G * ((after - window) // G) if after > window else 0   # quantized tokens
     byts = w.n_kv_heads * ((nq // G) * blk + (n - nq) * 4 * d) + w.n_q_heads * d * 2
     copies = max(2, math.ceil(3 * L2_BYTES / byts))
     k = torch.from_numpy(np.concatenate(w.keys)).to(device)
@@ -434,8 +438,8 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True):
             raise RuntimeError("decode kernel reported a failed wait")
     peak, peak_kind = _peaks()
     res = {"workload": "long_ctx", "context": n, "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv",
-           "bits": f"K{w.k_bits}/V{w.v_bits}", "group": G, "window": window,
-           "fp16_tail_tokens": n - nq, "copies": copies,
+           "bits": f"K{w.k_bits}/V{w.v_bits}", "group": G, "window": window, "sink": sink,
+           "fp16_tokens": n - nq, "copies": copies,
            "bytes_per_launch": int(byts), "avg_launch_us": round(us, 3),
            "achieved_gbs": round(byts / us / 1e3, 1), "peak": peak, "peak_kind": peak_kind,
            "frac": round(byts / us / 1e3 / peak, 4), "launches": iters,
@@ -685,6 +689,8 @@ def main():
                     help="also time decode alone on the 128k-token workload (0: skip)")
     ap.add_argument("--window", type=int, default=128,
                     help="recent fp16 window of the extra 128k-token decode leg (0: skip it)")
+    ap.add_argument("--sink", type=int, default=32,
+                    help="fp16 sink window of one more 128k-token leg, with --window (0: skip it)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -728,6 +734,10 @@ def main():
             if args.window:
                 out["recent_window_decode"] = run_long_context(
                     stream, device, iters=max(1, args.steps), window=args.window, fp16=False)
+            if args.sink:
+                out["sink_window_decode"] = run_long_context(
+                    stream, device, iters=max(1, args.steps), window=args.window, fp16=False,
+                    sink=args.sink)
             print(json.dumps(out))
         if world > 1:
             import torch.distributed as tdist
@@ -753,6 +763,8 @@ def main():
             line["long_context_decode"] = res["long_ctx"]
         if res["window"]:
             line["recent_window_decode"] = res["window"]
+        if res["sink"]:
+            line["sink_window_decode"] = res["sink"]
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as tdist

@@ -30,8 +30,13 @@
  * newer tokens follow it: N = G * floor(max(0, n - R) / G) tokens are
  * quantized and the tail holds the other n - N, between R and R + G - 1 once
  * n >= R; a tail that reaches R + G tokens has its oldest G quantized as the
- * next group ("flush").  R = 0 gives the n mod G tail.  Query head h reads
- * kv head h / (n_q_heads / n_kv_heads).
+ * next group ("flush").  R = 0 gives the n mod G tail.  With the sink window
+ * S = kvq_config.sink (InnerQ abstract, page "WUSH-KV: KV Cache Quantization
+ * with Data-Adaptive Transforms": high-precision windows for recent and for
+ * attention-sink tokens) the first S tokens of a sequence stay in fp16 as
+ * well; groups are cut from position S on and the rule above applies to the
+ * tokens after the sink.  Query head h reads kv head h / (n_q_heads /
+ * n_kv_heads).
  *
  * Conventions
  * -----------
@@ -53,9 +58,12 @@
  *   tails  : [max_seqs][n_kv_heads] { K tail fp16 [W][d] token-major,
  *                                     V tail fp16 [W/2][d][2] token pairs }
  *            a ring of W = R + G token slots: the token at sequence
- *            position p sits in slot t = p mod W while it is in the tail
- *            (t = p - N when R = 0).  K tail slot (t, c) is element t*d + c;
- *            V tail slot (t, c) is element ((t/2)*d + c)*2 + t%2.
+ *            position p sits in slot t = (p - S) mod W while it is in the
+ *            tail (t = p - N when R = S = 0).  K tail slot (t, c) is element
+ *            t*d + c; V tail slot (t, c) is element ((t/2)*d + c)*2 + t%2.
+ *   sinks  : [max_seqs][n_kv_heads] { K fp16 [SW][d], V fp16 [SW/2][d][2] }
+ *            SW = S rounded up to a multiple of 16; token p < S in slot p,
+ *            same element order as the tail (absent when S = 0).
  * A group block holds, in this order (byte offsets in kvq_layout):
  *   key codes   G*d*kbits/8 bytes
  *   key scales  d fp16, key mins d fp16
@@ -127,6 +135,8 @@ typedef struct {
   int32_t window;          /* R: recent tokens kept in fp16 beyond the partial
                               group; a multiple of 16 in [0, 1024]; 0 = the
                               n mod G tail */
+  int32_t sink;            /* S: first tokens of each sequence kept in fp16,
+                              in [0, 1024]; 0 = none */
 } kvq_config;
 
 typedef struct {
@@ -141,6 +151,9 @@ typedef struct {
   uint64_t kcodes_offset, kscale_offset, kmin_offset; /* within a block */
   uint64_t vcodes_offset, vscale_offset, vmin_offset; /* within a block */
   uint64_t tail_slots;     /* W = window + G token slots per tail ring */
+  uint64_t sinks_offset;   /* first sink area (0 bytes each when sink = 0) */
+  uint64_t sink_bytes;     /* K + V sink of one (seq, kv head) = 4*SW*d */
+  uint64_t sink_slots;     /* SW: sink rounded up to a multiple of 16 */
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache;

@@ -33,8 +33,9 @@ Readings where the pages are silent (each is listed in the design notes):
   128 of them, stay in FP16): with R > 0 a group is quantized only once R
   newer tokens follow it, so the tail holds between R and R + G - 1 tokens
   (all n tokens while n < R); R = 0 is the n mod G tail above.  The tail is a
-  ring of R + G token slots: token p sits in slot p mod (R + G), so tokens
-  never move while they wait (our layout; the pages do not store it).
+  ring of R + G token slots: token p sits in slot (p - S) mod (R + G), S the
+  sink window below, so tokens never move while they wait (our layout; the
+  pages do not store it).
 * sink window S (InnerQ abstract, page "WUSH-KV: KV Cache Quantization with
   Data-Adaptive Transforms", third abstract: high-precision windows for the
   recent tokens and for the attention-sink tokens): the first S tokens of a
@@ -472,9 +473,15 @@ def segments(cfg: Config, n: int):
 
 
 def tail_slot(cfg: Config, p: int) -> int:
-    """Slot of the fp16 tail ring that token position p occupies while it is
-    in the tail: p mod (R + G)."""
-    return p % cfg.tail_slots
+    """Slot of the fp16 tail ring that token position p (>= S) occupies
+    while it is in the tail: (p - S) mod (R + G)."""
+    return (p - cfg.sink) % cfg.tail_slots
+
+
+def sink_slots(cfg: Config) -> int:
+    """Token slots of the fp16 sink area: S rounded up to a multiple of 16
+    (token s < S in slot s)."""
+    return (cfg.sink + 15) // 16 * 16
 
 
 def quantize_group(cfg: Config, k16: np.ndarray, v16: np.ndarray):
@@ -531,6 +538,20 @@ def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray, first: int 
             tk[tail_key_index(t, c, d)] = tail_k[i, c]
             tv[tail_value_index(t, c, d)] = tail_v[i, c]
     return tk, tv
+
+
+def sink_arrays(cfg: Config, sink_k: np.ndarray, sink_v: np.ndarray):
+    """Place the Sb sink tokens [Sb, d] into the sink arrays (flat fp16 of
+    sink_slots(cfg) token slots, the tail's element order): token s in slot
+    s.  Slots past Sb are zero here (their device contents are unspecified)."""
+    SW, d = sink_slots(cfg), cfg.head_dim
+    sk = np.zeros(SW * d, np.float16)
+    sv = np.zeros(SW * d, np.float16)
+    for t in range(sink_k.shape[0]):
+        for c in range(d):
+            sk[tail_key_index(t, c, d)] = sink_k[t, c]
+            sv[tail_value_index(t, c, d)] = sink_v[t, c]
+    return sk, sv
 
 
 def dequantized_cache(cfg: Config, k16: np.ndarray, v16: np.ndarray):

@@ -18,7 +18,8 @@ def kvq():
 
 def oracle_cfg(spec) -> o.Config:
     return o.Config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim, spec.n_q_heads,
-                    spec.n_kv_heads, window=getattr(spec, "window", 0))
+                    spec.n_kv_heads, window=getattr(spec, "window", 0),
+                    sink=getattr(spec, "sink", 0))
 
 
 def to_device(x: np.ndarray, dtype: str) -> torch.Tensor:
@@ -78,11 +79,12 @@ def check_cache_against_oracle(cache, hist_k, hist_v, seqs=None, group_sample=No
         n = hist_k[b].shape[0]
         assert lens[b] == n, (b, lens[b], n)
         assert dev_lens[b] == n, (b, dev_lens[b], n)
-        N, T = o.split_tokens(n, cfg.group, cfg.window)
-        ng = N // cfg.group
+        Sb, Nq, T = o.segments(cfg, n)
+        N = Sb + Nq                      # first tail position
+        ng = Nq // cfg.group
         gsel = np.arange(ng) if group_sample is None else np.asarray(group_sample(ng), np.int64)
         if len(gsel):
-            toks = (gsel[:, None] * cfg.group + np.arange(cfg.group)[None, :]).reshape(-1)
+            toks = (Sb + gsel[:, None] * cfg.group + np.arange(cfg.group)[None, :]).reshape(-1)
             kk = hist_k[b][toks].reshape(len(gsel), cfg.group, cfg.n_kv_heads, cfg.head_dim)
             vv = hist_v[b][toks].reshape(len(gsel), cfg.group, cfg.n_kv_heads, cfg.head_dim)
             q = o.quantize_group(cfg, kk.transpose(2, 0, 1, 3), vv.transpose(2, 0, 1, 3))
@@ -104,6 +106,21 @@ def check_cache_against_oracle(cache, hist_k, hist_v, seqs=None, group_sample=No
                 gv = gv.cpu().numpy()
                 assert np.array_equal(gk[mk].view(np.uint16), tk[mk].view(np.uint16)), (b, h, "tail K")
                 assert np.array_equal(gv[mv].view(np.uint16), tv[mv].view(np.uint16)), (b, h, "tail V")
+        if Sb:
+            d = cfg.head_dim
+            mk = np.zeros(o.sink_slots(cfg) * d, bool)
+            mv = np.zeros(o.sink_slots(cfg) * d, bool)
+            for t in range(Sb):
+                for c in range(d):
+                    mk[o.tail_key_index(t, c, d)] = True
+                    mv[o.tail_value_index(t, c, d)] = True
+            for h in range(cfg.n_kv_heads):
+                sk, sv = o.sink_arrays(cfg, hist_k[b][:Sb, h], hist_v[b][:Sb, h])
+                gk, gv = cache.sink_halves(b, h)
+                gk = gk.cpu().numpy()
+                gv = gv.cpu().numpy()
+                assert np.array_equal(gk[mk].view(np.uint16), sk[mk].view(np.uint16)), (b, h, "sink K")
+                assert np.array_equal(gv[mv].view(np.uint16), sv[mv].view(np.uint16)), (b, h, "sink V")
 
 
 def oracle_decode(spec, hist_k, hist_v, q: np.ndarray) -> np.ndarray:

@@ -72,6 +72,17 @@ def test_tail_ring_size_from_library(kvq, G, R):
     assert lay["total_bytes"] >= lay["tails_offset"] + 8 * 8 * lay["tail_bytes"]
 
 
+@pytest.mark.parametrize("S", [0, 4, 16, 33, 1024])
+def test_sink_area_size_from_library(kvq, S):
+    """The sink area holds S rounded up to 16 token slots (K and V fp16)."""
+    lay = kvq.layout_for(_cfg(kvq, sink=S, window=64))
+    sw = o.sink_slots(o.Config(4, 2, 32, 128, 32, 8, window=64, sink=S))
+    assert lay["sink_slots"] == sw and lay["sink_bytes"] == 4 * sw * 128
+    assert lay["sinks_offset"] % 256 == 0
+    assert lay["sinks_offset"] >= lay["tails_offset"] + 8 * 8 * lay["tail_bytes"]
+    assert lay["total_bytes"] >= lay["sinks_offset"] + 8 * 8 * lay["sink_bytes"]
+
+
 def test_bytes_per_token_head_from_library(kvq):
     """128 B per token-head for K4/V2 G=32, 96 for K2/V2, 112 for K4/V2 G=64."""
     for kb, G, expect in ((4, 32, 128), (2, 32, 96), (4, 64, 112)):
@@ -83,7 +94,7 @@ def test_bytes_per_token_head_from_library(kvq):
     ("k_bits", 3), ("k_bits", 8), ("v_bits", 1), ("group", 16), ("group", 128),
     ("head_dim", 96), ("head_dim", 256), ("n_q_heads", 30), ("n_kv_heads", 0),
     ("max_seqs", 0), ("max_tokens", 0), ("layout_version", 2),
-    ("window", -16), ("window", 24), ("window", 1040),
+    ("window", -16), ("window", 24), ("window", 1040), ("sink", -1), ("sink", 1025),
 ])
 def test_bad_config_rejected(kvq, field, value):
     cfg = _cfg(kvq)

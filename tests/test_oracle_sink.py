@@ -147,3 +147,18 @@ def test_sink_covering_the_context_is_plain_fp16_attention():
     q = rng.standard_normal((2, d))
     assert o.segments(cfg, n) == (n, 0, 0)
     assert np.abs(o.decode(cfg, k, v, q) - _plain_attention(q, k, v, 2)).max() <= 1e-12
+
+
+@pytest.mark.parametrize("S", [4, 16, 33])
+def test_sink_shifts_the_tail_ring(S):
+    """With a sink the tail ring holds the tokens after it exactly as the
+    sink-free ring holds the shifted sequence; slots stay distinct."""
+    G, R = 32, 64
+    cs = o.Config(4, 2, G, 64, 1, 1, window=R, sink=S)
+    c0 = o.Config(4, 2, G, 64, 1, 1, window=R)
+    for n in range(S, S + R + 4 * G):
+        Sb, Nq, T = o.segments(cs, n)
+        slots = [o.tail_slot(cs, p) for p in range(Sb + Nq, n)]
+        assert slots == [o.tail_slot(c0, p - S) for p in range(Sb + Nq, n)]
+        assert len(set(slots)) == T and all(0 <= x < R + G for x in slots)
+    assert o.sink_slots(cs) % 16 == 0 and S <= o.sink_slots(cs) < S + 16
