@@ -36,6 +36,16 @@ Readings where the pages are silent (each is listed in the design notes):
   ring of R + G token slots: token p sits in slot (p - S) mod (R + G), S the
   sink window below, so tokens never move while they wait (our layout; the
   pages do not store it).
+* rotation (optional; "[Framework] The Asymmetric Key-Value Cache
+  Compression", §IV stage 1: Y = X H with an orthogonal +-1 Hadamard matrix
+  computed by the fast Walsh-Hadamard transform; "Asymmetric Key-Value
+  Quantization ...", §3.1: keys and values quantized after an FWHT
+  rotation): every K and V token entering the cache is rotated over its d
+  channels - converted to fp32, the radix-2 butterfly in fp32 in the fixed
+  order of ``fwht_fp32``, times fp32(1/sqrt(d)) - and then rounded to
+  fp16, so the whole cache (groups, tail, sink) holds rotated tokens; the
+  decode rotates q the same way (in fp64 here) and rotates its output
+  back (H is symmetric and H H = d I).
 * sink window S (InnerQ abstract, page "WUSH-KV: KV Cache Quantization with
   Data-Adaptive Transforms", third abstract: high-precision windows for the
   recent tokens and for the attention-sink tokens): the first S tokens of a
@@ -77,6 +87,7 @@ class Config:
     max_tokens: int = 0
     window: int = 0      # R: recent tokens kept in fp16 beyond the partial group
     sink: int = 0        # S: first tokens of a sequence kept in fp16
+    rotate: bool = False # cache holds Hadamard-rotated tokens
 
     @property
     def tail_slots(self) -> int:   # W = R + G slots of the fp16 tail ring
@@ -448,6 +459,56 @@ def unpack_block(cfg: Config, blk: np.ndarray):
 
 
 # ---------------------------------------------------------------------------
+# Hadamard rotation (fast Walsh-Hadamard transform)
+# ---------------------------------------------------------------------------
+def fwht_fp32(x) -> np.ndarray:
+    """Unnormalized Walsh-Hadamard transform over the last axis (a power of
+    two), in IEEE fp32: stages h = 1, 2, 4, ..., d/2; in each, every pair
+    (j, j + h) of a block of 2h entries becomes (a + b, a - b).  Equals
+    x H with H[i, j] = (-1)^popcount(i & j) (Sylvester order)."""
+    y = np.array(x, dtype=np.float32)
+    d = y.shape[-1]
+    h = 1
+    while h < d:
+        y = y.reshape(y.shape[:-1] + (d // (2 * h), 2, h))
+        a, b = y[..., 0, :], y[..., 1, :]
+        y = np.stack([a + b, a - b], axis=-2).reshape(y.shape[:-3] + (d,))
+        h *= 2
+    return y
+
+
+def rotate_fp16(x) -> np.ndarray:
+    """The cache's rotation of tokens x [..., d] (fp16, bf16 or fp32 values):
+    fp16( fwht_fp32(x) * fp32(1 / sqrt(d)) ), every step rounded to nearest
+    even."""
+    x32 = np.asarray(x, dtype=np.float32)
+    d = x32.shape[-1]
+    scale = np.float32(1.0 / math.sqrt(d))
+    return (fwht_fp32(x32) * scale).astype(np.float16)
+
+
+def rotate_fp64(x) -> np.ndarray:
+    """x H / sqrt(d) over the last axis in float64 (the query's rotation,
+    and the inverse rotation of the output: the map is its own inverse)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    y = x.copy()
+    h = 1
+    while h < d:
+        y = y.reshape(y.shape[:-1] + (d // (2 * h), 2, h))
+        a, b = y[..., 0, :], y[..., 1, :]
+        y = np.stack([a + b, a - b], axis=-2).reshape(y.shape[:-3] + (d,))
+        h *= 2
+    return y / math.sqrt(d)
+
+
+def cache_tokens(cfg: Config, x) -> np.ndarray:
+    """What the cache stores for input tokens x [n, Hkv, d]: the fp16
+    values, rotated first when ``cfg.rotate``."""
+    return rotate_fp16(x) if cfg.rotate else np.asarray(x).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------
 # the cache: groups + fp16 tail, as a function of the token history
 # ---------------------------------------------------------------------------
 def split_tokens(n: int, group: int, window: int = 0):
@@ -503,7 +564,8 @@ def grouped(cfg: Config, x16: np.ndarray) -> np.ndarray:
 def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True):
     """Expected cache contents for one sequence.
 
-    k16, v16: [n, Hkv, d] fp16 token history.  Returns a dict with
+    k16, v16: [n, Hkv, d] fp16 tokens as the cache stores them (for a
+    rotating cache, ``cache_tokens(cfg, x)`` of the inputs).  Returns a dict with
     ``groups``: (kc, ks, kz, vc, vs, vz) with a leading [Hkv, n_groups] shape,
     ``blocks``: [Hkv, n_groups, block_bytes] uint8 (if ``pack``),
     ``tail_k``/``tail_v``: [Hkv, T, d] fp16 tail tokens (positions N .. n-1 in
@@ -608,6 +670,15 @@ def attention_weights(q_h: np.ndarray, k_kv: np.ndarray) -> np.ndarray:
 
 
 def decode(cfg: Config, k16: np.ndarray, v16: np.ndarray, q: np.ndarray) -> np.ndarray:
-    """Decode output for one sequence on the quantized cache, float64 [Hq, d]."""
+    """Decode output for one sequence on the quantized cache, float64 [Hq, d].
+
+    k16, v16: the input token history [n, Hkv, d] (fp16 values; with
+    ``cfg.rotate`` any fp16/bf16/fp32 values, rotated as the cache stores
+    them).  With rotation the attention runs in the rotated domain on the
+    rotated query (dot products are preserved) and its output is rotated
+    back."""
+    if cfg.rotate:
+        kh, vh = dequantized_cache(cfg, rotate_fp16(k16), rotate_fp16(v16))
+        return rotate_fp64(attention(rotate_fp64(q), kh, vh, cfg.gqa))
     kh, vh = dequantized_cache(cfg, k16, v16)
     return attention(q, kh, vh, cfg.gqa)
