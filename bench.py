@@ -632,6 +632,45 @@ def cpu_oracle(budget_s: float):
                       f"1 thread, {el:.1f} s"}
 
 
+def _oracle_worker(budget_s: float):
+    """One process of the all-cores CPU baseline: whole oracle units, one
+    thread, until budget_s seconds have passed; returns (units, seconds,
+    tokens per unit)."""
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    from threadpoolctl import threadpool_limits
+    k, v, q = _oracle_unit_inputs()
+    n = k.shape[0]
+    done = 0
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        while True:
+            oracle_unit(k, v, q, n)
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+    return done, el, n
+
+
+def cpu_oracle_all_cores(budget_s: float):
+    """The same oracle units on every host core at once (up to 64): one
+    single-threaded process per core (a spawn pool, safe after CUDA is
+    initialised), each for budget_s seconds; the rate is the sum of the
+    processes' rates."""
+    import multiprocessing as mp
+    cores = min(os.cpu_count() or 1, 64)   # bounded memory and start-up time
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(processes=cores) as pool:
+        # bounded: a pool whose workers cannot start would otherwise wait forever
+        res = pool.map_async(_oracle_worker, [budget_s] * cores).get(timeout=budget_s + 300)
+    rate = sum(done * n / 8 / el for done, el, n in res)
+    units = sum(done for done, _, _ in res)
+    return {"value": rate, "unit": UNIT, "cores": cores,
+            "sample": f"{units} (sequence, kv-head) units at context {res[0][2]} over {cores} "
+                      f"single-threaded processes, {budget_s:.1f} s each"}
+
+
 def reference_arm(args):
     """--impl reference: W warm-up and K timed steps of the oracle; each step
     is a bounded sample of the workload (one unit, its context cut to fit the
@@ -685,6 +724,8 @@ def main():
     ap.add_argument("--copies", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--cpu-all-cores", type=int, default=1,
+                    help="also time the oracle on every host core (0: one thread only)")
     ap.add_argument("--long-context", type=int, default=1,
                     help="also time decode alone on the 128k-token workload (0: skip)")
     ap.add_argument("--window", type=int, default=128,
@@ -746,6 +787,8 @@ def main():
     res = run_ours(args, rank, world, device)
     wl = res["wl"]
     cb = cpu_oracle(args.cpu_budget) if (rank == 0 and world == 1) else None
+    if cb is not None and args.cpu_all_cores:
+        cb["all_cores"] = cpu_oracle_all_cores(args.cpu_budget)
     if rank == 0:
         line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
