@@ -1,5 +1,5 @@
 // Host side of the libkvq C ABI: argument validation (before any launch),
-// LAYOUT v1 geometry, the host mirror of sequence lengths and launch
+// LAYOUT v2 geometry, the host mirror of sequence lengths and launch
 // planning.  Every numeric step of the method runs in the CUDA kernels.
 #include <cuda_runtime.h>
 
@@ -371,22 +371,30 @@ kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype
   const kvq::Geom& g = cache->geom;
   for (int b = 0; b < n_seq; ++b)
     if (cache->lens[b] <= 0) return fail(KVQ_ERR_EMPTY, "sequence %d is empty", b);
-  // The fixed scratch holds [error word | per-unit split records | two
-  // partial slots per CTA]; the CTA count is lowered until the partials fit.
+  // The fixed scratch holds [error word | split records and tickets of the
+  // units of one launch (at most kSeqsPerLaunch sequences) | two partial
+  // slots per CTA]; the CTA count is lowered until the partials fit.
   kvq::WsLayout w = cache->ws;
+  const int64_t units = (int64_t)std::min(n_seq, kvq::kSeqsPerLaunch) * g.hkv * g.slices;
+  w.units = (int32_t)units;
+  w.err_off = 0;
+  w.units_off = 256;
+  w.tickets_off = kvq::align_up(w.units_off + 8LL * units, 256);
+  w.partials_off = kvq::align_up(w.tickets_off + 4LL * units, 256);
   const int64_t slot_bytes = 2LL * w.slot_floats * 4;
   const int64_t room = kvq::kNoAllocScratchBytes - w.partials_off;
   if (room < slot_bytes)
     return fail(KVQ_ERR_CAPACITY,
-                "kvq_decode_noalloc: %d (sequence, kv head, head slice) units need more than the "
-                "%lld-byte fixed scratch; use kvq_decode with a workspace",
-                w.units, (long long)kvq::kNoAllocScratchBytes);
+                "kvq_decode_noalloc: the %lld (sequence, kv head, head slice) units of one launch "
+                "need more than the %lld-byte fixed scratch; use kvq_decode with a workspace",
+                (long long)units, (long long)kvq::kNoAllocScratchBytes);
   const int64_t max_grid = std::min<int64_t>(kvq::kMaxDecodeCtas, room / slot_bytes);
   void* scratch = nullptr;
   cudaError_t e = kvq::noalloc_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed decode scratch");
-  // the error word must start at zero; the array keeps whatever the previous
-  // call left (the split records are rewritten by every launch)
+  // the error word and the tickets must start at zero; the array keeps
+  // whatever the previous call left (split records are rewritten by every
+  // launch, and the last CTA of a unit puts its ticket back to zero)
   e = cudaMemsetAsync(scratch, 0, (size_t)w.partials_off, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed decode scratch");
   w.total = w.partials_off + max_grid * slot_bytes;

@@ -1,5 +1,5 @@
 // Append kernel of libkvq: per-channel key quantization, per-token value
-// quantization, bit packing into LAYOUT v1, the fp16 tail and its flush.
+// quantization, bit packing into LAYOUT v2, the fp16 tail and its flush.
 //
 // "[Framework] The Asymmetric Key-Value Cache Compression", §III: keys are
 // quantized per channel (outliers stay in their column), values per token,

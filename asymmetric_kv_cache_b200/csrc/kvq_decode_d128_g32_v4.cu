@@ -1,0 +1,8 @@
+// Instantiations of the quantized decode kernels for head_dim 128, group
+// 32, 4-bit values (2- and 4-bit keys).
+#include "kvq_decode_kernels.cuh"
+
+namespace kvq {
+KVQ_DECODE_DEFINE(128, 4, 4, 32)
+KVQ_DECODE_DEFINE(128, 2, 4, 32)
+}  // namespace kvq

@@ -1,5 +1,5 @@
 // Internal declarations shared by the host side of libkvq (kvq_abi.cpp) and
-// its CUDA kernels.  Geometry only: the offsets of LAYOUT v1 (documented in
+// its CUDA kernels.  Geometry only: the offsets of LAYOUT v2 (documented in
 // include/kvq.h) and the launch entry points of each kernel family.
 #pragma once
 
@@ -159,6 +159,21 @@ struct DecodeArgs {
 cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas);
 cudaError_t launch_decode(const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid,
                           bool wide, cudaStream_t stream);
+// The same two entry points per (head dim, key bits, value bits, group),
+// defined in the kvq_decode_d*_g*_v*.cu translation units.
+#define KVQ_DECODE_DECLARE(D_, KB_, VB_, G_)                                              \
+  cudaError_t decode_max_ctas_##D_##_##KB_##_##VB_##_##G_(const Geom& g, bool wide,       \
+                                                          int* out);                      \
+  cudaError_t launch_decode_##D_##_##KB_##_##VB_##_##G_(                                  \
+      const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid, bool wide,         \
+      cudaStream_t stream);
+#define KVQ_DECODE_FOR_EACH(X) \
+  X(128, 4, 2, 32) X(128, 2, 2, 32) X(128, 4, 2, 64) X(128, 2, 2, 64) \
+  X(128, 4, 4, 32) X(128, 2, 4, 32) X(128, 4, 4, 64) X(128, 2, 4, 64) \
+  X(64, 4, 2, 32) X(64, 2, 2, 32) X(64, 4, 2, 64) X(64, 2, 2, 64)     \
+  X(64, 4, 4, 32) X(64, 2, 4, 32) X(64, 4, 4, 64) X(64, 2, 4, 64)
+KVQ_DECODE_FOR_EACH(KVQ_DECODE_DECLARE)
+
 // fp16 decode baseline over K, V [n_seq][Hkv][max_tokens][d] (a.seq0 and the
 // device lengths `lens` index the cache; q and out start at a.seq0).
 cudaError_t launch_decode_fp16(const Geom& g, const WsLayout& w, const DecodeArgs& a,

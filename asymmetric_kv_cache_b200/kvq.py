@@ -28,7 +28,7 @@ STATUS_NAMES = {
     8: "KVQ_ERR_ALIGN", 9: "KVQ_ERR_ARG", 10: "KVQ_ERR_DEVICE",
 }
 DTYPE_CODES = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
-LAYOUT_VERSION = 1
+LAYOUT_VERSION = 2
 
 
 class KvqConfig(ctypes.Structure):

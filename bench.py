@@ -12,10 +12,12 @@ total) so every decode reads its cache from HBM; each copy's contexts start
 below 4113 so that over the timed steps their mean is 4113.
 
 Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA
-graphs (one graph = one round over the copies; two instances alternate so
-that CUDA events around every decode can be read while the next round
-runs), bracketed by barrier + synchronize, CUDA events on the launch
-stream, max over ranks.  Under torchrun every rank runs its own replica
+graphs (one graph = one round over the copies, two instances alternating,
+plus one graph for the remaining K mod C steps), every graph uploaded to
+the device before the timed region, no host synchronisation inside it,
+bracketed by barrier + synchronize, CUDA events on the launch stream, max
+over ranks.  CUDA events around every 4th decode of the last replay of
+each graph give the decode kernel's own time (read after the region).  Under torchrun every rank runs its own replica
 (weak scaling, no collective on the data path).
 
 `--impl reference` times the CPU oracle (test infrastructure) on the same
@@ -225,7 +227,7 @@ def run_ours(args, rank, world, device):
     # recorded between the append and the decode keeps the decode from
     # launching as a programmatic dependent of the append, so the other
     # steps run as a user's loop would
-    EV = 8
+    EV = 4
 
     def capture(n_steps, first_step):
         evs = [(torch.cuda.Event(enable_timing=True, external=True),
@@ -253,6 +255,12 @@ def run_ours(args, rank, world, device):
     gR = capture(rem, wl.W + rounds * C) if rem else None
     for cache in caches:          # capture advanced the host mirrors only
         cache.sync_lengths(stream)
+    # upload every instance now, so that no first-replay cost (the graph's
+    # upload to the device) falls inside the timed region
+    for x in (gA, gB, gR):
+        if x is not None:
+            _graph_upload(x[0], stream)
+    stream.synchronize()
 
     # host view of every copy's length at each timed step (for the metric)
     lens_at = []
@@ -263,9 +271,7 @@ def run_ours(args, rank, world, device):
         lens_at.append(cur[c])
     kv_tokens = sum(L * wl.batch for L in lens_at)
     alg_bytes = sum(wl.algorithmic_bytes([L] * wl.batch) for L in lens_at)
-    # bytes of the decodes that carry events (step i of each round, i % EV == 0)
-    ev_steps = [j for j in range(wl.K) if (j % C if C <= wl.K else j) % EV == 0]
-    ev_bytes = statistics.fmean(wl.algorithmic_bytes([lens_at[j]] * wl.batch) for j in ev_steps)
+    ev_bytes = None
 
     dist = world > 1
     if dist:
@@ -291,28 +297,28 @@ def run_ours(args, rank, world, device):
     insts = [x for x in (gA, gB) if x is not None]
     with torch.cuda.stream(stream):
         t0.record(stream)
-        pending = None
+        # every graph was uploaded before t0; no host synchronisation in here
         for r in range(rounds):
-            g, evs = insts[r % len(insts)]
-            g.replay()
-            if len(insts) == 1:
-                # one instance: its events must be read before it is replayed again
-                evs[-1][1].synchronize()
-                collect(evs)
-            else:
-                # two instances: read the previous round while this one runs
-                if pending is not None:
-                    pending[-1][1].synchronize()
-                    collect(pending)
-                pending = evs
+            insts[r % len(insts)][0].replay()
         if gR is not None:
             gR[0].replay()
         t1.record(stream)
     t1.synchronize()
-    if pending is not None and len(insts) > 1:
-        collect(pending)
+    # the decode events of the last replay of every instance (a replay
+    # overwrites its events, so these are read only after t1)
+    ev_idx = []
+    for ii, (gx, evs) in enumerate(insts):
+        last = max((r for r in range(rounds) if r % len(insts) == ii), default=None)
+        if last is None:
+            continue
+        collect(evs)
+        ev_idx += [last * C + i for i in range(steps_in_round) if i % EV == 0]
     if gR is not None:
         collect(gR[1])
+        ev_idx += [rounds * C + i for i in range(rem) if i % EV == 0]
+    if ev_idx:
+        ev_bytes = statistics.fmean(wl.algorithmic_bytes([lens_at[j]] * wl.batch)
+                                    for j in ev_idx)
     clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
     if dist:
@@ -326,6 +332,8 @@ def run_ours(args, rank, world, device):
               if args.long_context and args.window else None)
     sinkw = (run_long_context(stream, device, window=args.window, sink=args.sink, fp16=False)
              if args.long_context and args.sink else None)
+    qa = run_quant_append(stream, device) if args.other_legs else None
+    c70 = run_concurrent_70b(stream, device) if args.other_legs else None
 
     for cache in caches:
         if cache.workspace_status(stream) != 0:
@@ -335,7 +343,7 @@ def run_ours(args, rank, world, device):
     dec_avg_ms = statistics.fmean(decode_ms) if decode_ms and elapsed_ok else None
     peak, peak_kind = _peaks()
     roof = None
-    if dec_avg_ms:
+    if dec_avg_ms and ev_bytes:
         achieved = ev_bytes / (dec_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": _traffic(),
@@ -344,12 +352,13 @@ def run_ours(args, rank, world, device):
                 "bytes_per_launch": int(ev_bytes),
                 "avg_launch_us": round(dec_avg_ms * 1e3, 3),
                 "timed_launches": len(decode_ms),
-                "note": "decode + combine of every 8th step bracketed by CUDA events"}
+                "note": "decode (+ combine when launched) of every 4th step of the last replay "
+                        "of each graph, bracketed by CUDA events, read after the timed region"}
     return {
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
         "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K, "long_ctx": long_ctx,
-        "window": window, "sink": sinkw,
+        "window": window, "sink": sinkw, "quant_append": qa, "conc70b": c70,
     }
 
 
@@ -476,6 +485,154 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0):
     del kc, vc, kk, vv
     torch.cuda.empty_cache()
     return res
+
+
+def _graph_upload(g, stream):
+    """Upload an instantiated torch CUDA graph to the device on `stream`
+    (cudaGraphUpload) without running it."""
+    from cuda.bindings import runtime as rt
+    err, = rt.cudaGraphUpload(rt.cudaGraphExec_t(init_value=g.raw_cuda_graph_exec()),
+                              rt.cudaStream_t(init_value=stream.cuda_stream))
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphUpload failed: {err}")
+
+
+def run_quant_append(stream, device, reps=8):
+    """The quantize/append workload (4 x 32768 tokens x 8 kv heads x d 128,
+    fp16 K/V, K4/V2, G 32): (i) prefill quantization of the whole batch in
+    one kvq_append call, CUDA events around `reps` calls on a cache reset
+    between calls (537 MB read, 134 MB written per call: larger than L2);
+    (ii) 64 sequences starting empty, 256 steps appending one token to each
+    (a key group flushed every 32 steps), timed eagerly (host launch
+    included) and replayed from a CUDA graph."""
+    import torch
+    from asymmetric_kv_cache_b200 import inputs, kvq
+    w = inputs.WORKLOADS["quant_append"]()
+    n, B, hkv, d = w.lens[0], w.batch, w.n_kv_heads, w.head_dim
+    spec = kvq.CacheSpec(w.k_bits, w.v_bits, w.group, d, hkv, hkv, B, n)
+    k = torch.from_numpy(np.concatenate(w.keys)).to(device)
+    v = torch.from_numpy(np.concatenate(w.values)).to(device)
+    del w
+    cache = kvq.KVQCache(spec, device=device)
+    rd = 2 * k.numel() * 2
+    wr = B * hkv * (n // 32) * (32 * d * (4 + 2) // 8 + 8 * d)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ms = []
+    with torch.cuda.stream(stream):
+        for r in range(reps + 2):
+            cache.reset(stream)
+            # keep the GPU busy while the host plans and launches the call,
+            # so that the events time the kernel and not the host
+            torch.cuda._sleep(2_000_000)
+            e0.record(stream)
+            cache.append(k, v, [n] * B, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            if r >= 2:
+                ms.append(e0.elapsed_time(e1))
+    del k, v, cache
+    us = statistics.median(ms) * 1e3
+    peak, peak_kind = _peaks()
+    prefill = {"tokens": B * n, "kv_heads": hkv, "head_dim": d, "bits": "K4/V2", "group": 32,
+               "read_bytes": rd, "write_bytes": wr, "median_us": round(us, 2), "calls": reps,
+               "achieved_gbs": round((rd + wr) / us / 1e3, 1), "peak": peak,
+               "peak_kind": peak_kind, "frac": round((rd + wr) / us / 1e3 / peak, 4)}
+    # (ii) one-token appends to 64 sequences, 256 steps from empty
+    S, steps = 64, 256
+    nk, nv = inputs.append_stream(inputs.SEED_BASE + 3 + 7, S, steps, hkv, d)
+    nk_dev = [torch.from_numpy(x).to(device) for x in nk]
+    nv_dev = [torch.from_numpy(x).to(device) for x in nv]
+    spec2 = kvq.CacheSpec(4, 2, 32, d, hkv, hkv, S, steps + 32)
+    c2 = kvq.KVQCache(spec2, device=device)
+    with torch.cuda.stream(stream):
+        c2.reset(stream)
+        for s in range(steps):                     # warm-up (launch attributes set)
+            c2.append(nk_dev[s], nv_dev[s], [1] * S, stream=stream)
+        c2.reset(stream)
+        stream.synchronize()
+        e0.record(stream)
+        for s in range(steps):
+            c2.append(nk_dev[s], nv_dev[s], [1] * S, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        eager_us = e0.elapsed_time(e1) * 1e3 / steps
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            c2.reset(stream)
+            for s in range(steps):
+                c2.append(nk_dev[s], nv_dev[s], [1] * S, stream=stream)
+        _graph_upload(g, stream)
+        g.replay()
+        stream.synchronize()
+        e0.record(stream)
+        for _ in range(4):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        graph_us = e0.elapsed_time(e1) * 1e3 / (4 * steps)
+    c2.sync_lengths(stream)
+    if c2.lengths(S) != [steps] * S:
+        raise RuntimeError("append stream: unexpected lengths after the replays")
+    del g, c2
+    torch.cuda.empty_cache()
+    return {"workload": "quant_append", "prefill": prefill,
+            "append_stream": {"sequences": S, "steps": steps, "flush_every": 32,
+                              "eager_us_per_step": round(eager_us, 2),
+                              "graph_us_per_step": round(graph_us, 2),
+                              "note": "one kvq_append per step (one token per sequence), "
+                                      "CUDA events; graph: 256 steps + reset per replay"}}
+
+
+def run_concurrent_70b(stream, device, iters=100):
+    """Decode alone on the 70B-shaped high-concurrency batch (64 sequences,
+    64 q / 8 kv heads, d 128, contexts ~ U{1024..8192}, K4/V2, G 64, bf16
+    queries), two cache copies alternated (each larger than L2)."""
+    import torch
+    from asymmetric_kv_cache_b200 import inputs, kvq
+    w = inputs.WORKLOADS["llama70b_conc"]()
+    G, d = w.group, w.head_dim
+    blk = G * d * (w.k_bits + w.v_bits) // 8 + 8 * d
+    byts = sum(w.n_kv_heads * ((L // G) * blk + (L % G) * 4 * d) for L in w.lens)
+    byts += w.batch * w.n_q_heads * d * 2
+    spec = kvq.CacheSpec(w.k_bits, w.v_bits, G, d, w.n_q_heads, w.n_kv_heads, w.batch,
+                         max(w.lens))
+    k = torch.from_numpy(np.concatenate(w.keys)).to(device)
+    v = torch.from_numpy(np.concatenate(w.values)).to(device)
+    q = torch.from_numpy(w.q_bits.view(np.int16)).to(device).view(torch.bfloat16)
+    copies = max(2, math.ceil(2 * L2_BYTES / byts))
+    caches = []
+    with torch.cuda.stream(stream):
+        for _ in range(copies):
+            c = kvq.KVQCache(spec, device=device)
+            c.append(k, v, w.lens, stream=stream)
+            caches.append(c)
+        del k, v
+        out = torch.empty(q.shape, dtype=torch.float16, device=device)
+        for i in range(2 * copies):
+            caches[i % copies].decode(q, out=out, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(iters):
+            caches[i % copies].decode(q, out=out, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    for c in caches:
+        if c.workspace_status(stream) != 0:
+            raise RuntimeError("decode kernel reported a failed wait")
+    del caches
+    torch.cuda.empty_cache()
+    peak, peak_kind = _peaks()
+    return {"workload": "llama70b_conc", "batch": w.batch, "context_sum": int(sum(w.lens)),
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "bits": f"K{w.k_bits}/V{w.v_bits}",
+            "group": G, "q_dtype": "bf16", "copies": copies, "bytes_per_launch": int(byts),
+            "avg_launch_us": round(us, 3), "achieved_gbs": round(byts / us / 1e3, 1),
+            "peak": peak, "peak_kind": peak_kind, "frac": round(byts / us / 1e3 / peak, 4),
+            "launches": iters,
+            "kv_tokens_per_s": round(sum(w.lens) * iters / (e0.elapsed_time(e1) / 1e3), 1),
+            "note": "decode (+ combine when launched) per call, CUDA events around the calls"}
 
 
 def run_e2e(args, wl, caches, nk, nv, q, stream, device):
@@ -632,10 +789,11 @@ def cpu_oracle(budget_s: float):
                       f"1 thread, {el:.1f} s"}
 
 
-def _oracle_worker(budget_s: float):
-    """One process of the all-cores CPU baseline: whole oracle units, one
-    thread, until budget_s seconds have passed; returns (units, seconds,
-    tokens per unit)."""
+def _oracle_worker(budget_s: float, t_start: float):
+    """One process of the all-cores CPU baseline: waits until wall time
+    t_start (so that every process runs at the same time), then whole oracle
+    units, one thread, until budget_s seconds have passed; returns (units,
+    start, end, tokens per unit)."""
     if ROOT not in sys.path:
         sys.path.insert(0, ROOT)
     from threadpoolctl import threadpool_limits
@@ -643,32 +801,37 @@ def _oracle_worker(budget_s: float):
     n = k.shape[0]
     done = 0
     with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
+        while time.time() < t_start:
+            time.sleep(0.01)
+        t0 = time.time()
         while True:
             oracle_unit(k, v, q, n)
             done += 1
-            el = time.perf_counter() - t0
-            if el >= budget_s:
+            if time.time() - t0 >= budget_s:
                 break
-    return done, el, n
+    return done, t0, time.time(), n
 
 
 def cpu_oracle_all_cores(budget_s: float):
-    """The same oracle units on every host core at once (up to 64): one
-    single-threaded process per core (a spawn pool, safe after CUDA is
-    initialised), each for budget_s seconds; the rate is the sum of the
-    processes' rates."""
+    """The same oracle units on every host core this process may use (its
+    CPU affinity, up to 64): one single-threaded process per core (a spawn
+    pool, safe after CUDA is initialised), all started at one common wall
+    time; the rate is all units over the window from the first start to the
+    last end."""
     import multiprocessing as mp
-    cores = min(os.cpu_count() or 1, 64)   # bounded memory and start-up time
+    cores = max(1, min(len(os.sched_getaffinity(0)), 64))   # bounded memory and start-up
     ctx = mp.get_context("spawn")
+    t_start = time.time() + 20.0 + 0.25 * cores             # after every worker has started
     with ctx.Pool(processes=cores) as pool:
         # bounded: a pool whose workers cannot start would otherwise wait forever
-        res = pool.map_async(_oracle_worker, [budget_s] * cores).get(timeout=budget_s + 300)
-    rate = sum(done * n / 8 / el for done, el, n in res)
-    units = sum(done for done, _, _ in res)
-    return {"value": rate, "unit": UNIT, "cores": cores,
-            "sample": f"{units} (sequence, kv-head) units at context {res[0][2]} over {cores} "
-                      f"single-threaded processes, {budget_s:.1f} s each"}
+        res = pool.starmap_async(_oracle_worker, [(budget_s, t_start)] * cores).get(
+            timeout=budget_s + 300)
+    units = sum(r[0] for r in res)
+    n = res[0][3]
+    window = max(r[2] for r in res) - min(r[1] for r in res)
+    return {"value": units * n / 8 / window, "unit": UNIT, "cores": cores,
+            "sample": f"{units} (sequence, kv-head) units at context {n} over {cores} "
+                      f"single-threaded processes started together, {window:.1f} s window"}
 
 
 def reference_arm(args):
@@ -720,7 +883,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3_8b",
-                    help="llama3_8b (the step), or long_ctx (decode alone on the 128k context)")
+                    choices=["llama3_8b", "long_ctx", "quant_append", "llama70b_conc"],
+                    help="llama3_8b (the step, default), or one leg alone: long_ctx (decode "
+                         "on the 128k context), quant_append (prefill + append stream), "
+                         "llama70b_conc (decode on the 64-sequence ragged batch)")
     ap.add_argument("--copies", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -732,6 +898,9 @@ def main():
                     help="recent fp16 window of the extra 128k-token decode leg (0: skip it)")
     ap.add_argument("--sink", type=int, default=32,
                     help="fp16 sink window of one more 128k-token leg, with --window (0: skip it)")
+    ap.add_argument("--other-legs", type=int, default=1,
+                    help="also time the quantize/append workload and the 70B-shaped batch "
+                         "(0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -765,6 +934,20 @@ def main():
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device(device))
+    if args.workload in ("quant_append", "llama70b_conc"):
+        if rank == 0:
+            stream = torch.cuda.Stream(device=device)
+            if args.workload == "quant_append":
+                out = {"metric": METRIC, "quant_append": run_quant_append(stream, device)}
+            else:
+                out = {"metric": METRIC,
+                       "concurrent_70b_decode": run_concurrent_70b(stream, device,
+                                                                   iters=max(1, args.steps))}
+            print(json.dumps(out))
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+        return 0
     if args.workload == "long_ctx":
         # decode alone on the 128k-token workload (the long-context leg of
         # the default run on its own, `--steps` timed launches)
@@ -787,8 +970,8 @@ def main():
     res = run_ours(args, rank, world, device)
     wl = res["wl"]
     cb = cpu_oracle(args.cpu_budget) if (rank == 0 and world == 1) else None
-    if cb is not None and args.cpu_all_cores:
-        cb["all_cores"] = cpu_oracle_all_cores(args.cpu_budget)
+    cb_all = (cpu_oracle_all_cores(args.cpu_budget)
+              if (cb is not None and args.cpu_all_cores) else None)
     if rank == 0:
         line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
@@ -808,6 +991,12 @@ def main():
             line["recent_window_decode"] = res["window"]
         if res["sink"]:
             line["sink_window_decode"] = res["sink"]
+        if res.get("quant_append"):
+            line["quant_append"] = res["quant_append"]
+        if res.get("conc70b"):
+            line["concurrent_70b_decode"] = res["conc70b"]
+        if cb_all is not None:
+            line["cpu_baseline_all_cores"] = cb_all
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as tdist

@@ -50,8 +50,15 @@
  *    cache unchanged.
  *  - A handle is not thread-safe; distinct handles are independent.
  *
- * LAYOUT v1 of the cache buffer (all region offsets 256-byte aligned; see
- * kvq_layout for the numbers):
+ * LAYOUT v2 of the cache buffer (all region offsets 256-byte aligned; see
+ * kvq_layout for the numbers).  Version 1 was a plain layout: separate
+ * regions for key codes, key (scale, min) pairs, value codes and value
+ * pairs, codes packed little-endian in element order.  Version 2 (the only
+ * one this library reads or writes; a configuration asking for 1 is refused
+ * with KVQ_ERR_CONFIG) keeps the same bytes per token but interleaves each
+ * group's sections into one contiguous block, so that a single bulk copy
+ * brings a whole group on chip, and stores the codes in tensor-core fragment
+ * order, so that one 128-bit shared-memory load gives a lane its operand.
  *   lens   : int32 [max_seqs]                 device copy of the lengths
  *   tickets: int32 [max_seqs]                 append completion counters (0 at rest)
  *   blocks : [max_seqs][n_kv_heads][max_groups] group blocks of block_bytes
@@ -96,7 +103,7 @@
 extern "C" {
 #endif
 
-#define KVQ_LAYOUT_VERSION 1
+#define KVQ_LAYOUT_VERSION 2
 
 /* Exported entry points (the library is built with hidden visibility). */
 #if defined(__GNUC__)
@@ -165,7 +172,7 @@ KVQ_API const char* kvq_status_string(kvq_status s);
  * string stays valid until the next call on that thread. */
 KVQ_API const char* kvq_last_error(void);
 
-/* LAYOUT v1 offsets for a configuration (host only, no device work).
+/* LAYOUT v2 offsets for a configuration (host only, no device work).
  * Errors: KVQ_ERR_NULL, KVQ_ERR_CONFIG. */
 KVQ_API kvq_status kvq_layout_for(const kvq_config* cfg, kvq_layout* out);
 
@@ -191,31 +198,47 @@ KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
 KVQ_API kvq_status kvq_reset(kvq_cache* cache, void* stream);
 
 /* Append n_new[b] tokens to sequence b, for b in [0, n_seq).
+ * Defining passages: "[Framework] The Asymmetric Key-Value Cache
+ * Compression", §III (Pillar I: keys grouped per channel along the token
+ * axis, values per token, the most recent tokens in FP16), and the InnerQ
+ * abstract on the "WUSH-KV: KV Cache Quantization with Data-Adaptive
+ * Transforms" page (group-wise quantization of the cache); the quantizer is
+ * the bit-exact contract in the header comment above.
  * k, v: device arrays [sum_b n_new[b], n_kv_heads, head_dim] of dtype
  * (fp16, bf16 or fp32), token-major, sequences concatenated in order b;
- * 16-byte aligned.  n_new: host array of n_seq non-negative counts.
+ * 16-byte aligned; read only.  n_new: host array of n_seq non-negative
+ * counts, read before the call returns.
  * Performs prefill quantization (whole groups straight from the input),
  * per-step appends into the fp16 tail and the flush of a tail that reaches
- * R + G tokens (its oldest G become a group), all in one launch.  The kernel takes the current lengths from
- * the device copy and advances it, so an append captured in a CUDA graph
- * may be replayed provided every n_new[b] < G (the launch shape then does
- * not depend on the lengths); after replays, kvq_sync_lengths refreshes the
- * host mirror.  Values outside the fp16 range are not representable by the
- * cache (their codes are unspecified).
+ * R + G tokens (its oldest G become a group), all in one launch.  The kernel
+ * takes the current lengths from the device copy and advances it, so an
+ * append captured in a CUDA graph may be replayed provided every n_new[b] <
+ * G (the launch shape then does not depend on the lengths); after replays,
+ * kvq_sync_lengths refreshes the host mirror.  Values outside the fp16 range
+ * are not representable by the cache (their codes are unspecified).
  * Errors (host side, cache unchanged): KVQ_ERR_NULL, KVQ_ERR_ARG,
  * KVQ_ERR_CAPACITY (n_seq > max_seqs or a length would pass max_tokens),
  * KVQ_ERR_DTYPE, KVQ_ERR_ALIGN; KVQ_ERR_CUDA if the launch fails. */
 KVQ_API kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype dtype,
                       const int32_t* n_new, int32_t n_seq, void* stream);
 
-/* Decode attention for sequences [0, n_seq): q device [n_seq, n_q_heads, d]
- * (fp16, bf16 or fp32, 16-byte aligned); out device [n_seq, n_q_heads, d]
- * fp16.  workspace: device buffer of at least the workspace_bytes reported
- * by kvq_cache_required_bytes, 256-byte aligned, zero-filled before its
- * first use (kvq_workspace_init).  Calls that share a workspace must not
- * overlap on the GPU.  For each chunk of up to 2048 sequences the call
- * launches the split-K decode kernel (one CTA per SM) and a small combine
- * kernel that merges the units split across CTAs (launched as a
+/* Decode attention for sequences [0, n_seq): for every query head h,
+ * out_h = sum_t alpha_t v_t with alpha = softmax(q_h . k_t / sqrt(d)) over
+ * all tokens of the sequence ("Asymmetric Key-Value Quantization: 2-Bit
+ * Values and 4-Bit Keys under Long-Context Drift", §1 and §2.1), the keys
+ * and values dequantized from their groups (s * code + z) or read from the
+ * fp16 tail and sink.
+ * q: device [n_seq, n_q_heads, d] (fp16, bf16 or fp32, 16-byte aligned),
+ * read only; out: device [n_seq, n_q_heads, d] fp16, written.  n_seq: the
+ * first n_seq sequences of the cache are decoded (any count up to
+ * max_seqs; the survey's interface left it implicit, this library takes it
+ * as an argument so that a batch may use fewer slots than the cache holds).
+ * workspace: device buffer of at least the workspace_bytes reported by
+ * kvq_cache_required_bytes, 256-byte aligned, zero-filled before its first
+ * use (kvq_workspace_init).  Calls that share a workspace must not overlap
+ * on the GPU.  For each chunk of up to 2048 sequences the call launches the
+ * split-K decode kernel (one CTA per SM) and, when units are split across
+ * many CTAs, a small combine kernel that merges them (launched as a
  * programmatic dependent of the first).  Inside a CTA the warps claim key
  * groups dynamically, so repeated calls are not bit-identical: the fp16
  * attention weights are rounded relative to a running max that depends on
@@ -234,29 +257,30 @@ KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype
                       int32_t n_seq, void* workspace, size_t ws_bytes, void* stream);
 
 /* kvq_decode for callers that cannot allocate device memory when they
- * decode: code running while a CUDA graph is being captured (an allocation
- * there is not allowed in the capture), plugins whose host framework owns
- * every device allocation and has no workspace hook, and deployments that
- * forbid allocation after start-up.  The pages have no counterpart of this
- * call: it only changes where the decode scratch lives.
+ * decode: plugins whose host framework owns every device allocation and
+ * offers no workspace hook, and deployments that forbid allocation after
+ * start-up (a fixed memory footprint, no allocator on the serving path).
+ * The pages have no counterpart of this call: it only changes where the
+ * decode scratch lives.
  * Instead of a caller workspace, the scratch (error word, per-unit split
- * records, split partials) is a fixed 8 MiB device array inside the library
- * (kvq_noalloc_scratch_bytes()); every GPU that loads the library holds it
- * until exit.  The call allocates nothing: it clears the error word and the
- * split records with cudaMemsetAsync, lowers the number of CTAs until the
- * partials fit, and launches the same decode kernel.  All calls share the
- * array, which keeps the last call's contents, so calls that overlap on the
- * GPU (other streams, other threads) race: serialize them.  The first call on
- * each device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before any stream capture.  Arguments and errors as
- * kvq_decode; KVQ_ERR_CAPACITY if the cache has so many (sequence, kv head,
- * head slice) units that their split records leave no room for even one
- * CTA's partials.  A failed
- * internal wait (never expected) is recorded only in the array's error
- * word, which the next call clears; use kvq_decode with a workspace where
- * that report matters.  Bit-for-bit
- * results may differ from kvq_decode's when the CTA count differs (split
- * order); both are within the same tolerance of exact attention. */
+ * records and tickets, split partials) is a fixed 8 MiB device array inside
+ * the library (kvq_noalloc_scratch_bytes()); every GPU that loads the
+ * library holds it until exit.  The call allocates nothing: it clears the
+ * error word, split records and tickets with cudaMemsetAsync, lowers the
+ * number of CTAs until the partials fit, and launches the same decode
+ * kernel.  All calls share the array, which keeps the last call's contents,
+ * so calls that overlap on the GPU (other streams, other threads) race:
+ * serialize them.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  Arguments and errors as kvq_decode; KVQ_ERR_CAPACITY
+ * (nothing launched) when the units of one launch - min(n_seq, 2048)
+ * sequences x n_kv_heads x head slices of 8 query heads - need more split
+ * records than the array holds (about 690,000 units).  A failed internal
+ * wait (never expected) is recorded only in the array's error word, which
+ * the next call clears; use kvq_decode with a workspace where that report
+ * matters.  Bit-for-bit results may differ from kvq_decode's when the CTA
+ * count differs (split order); both are within the same tolerance of exact
+ * attention. */
 KVQ_API kvq_status kvq_decode_noalloc(kvq_cache* cache, const void* q, kvq_dtype q_dtype,
                                       void* out, int32_t n_seq, void* stream);
 

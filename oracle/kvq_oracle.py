@@ -55,7 +55,7 @@ Readings where the pages are silent (each is listed in the design notes):
 * attention is evaluated in float64 on the dequantized cache
   x_hat = code * s + z (tail tokens exactly as stored in fp16).
 
-The byte layout (``LAYOUT v1``) is a fixed per-group permutation of the codes
+The byte layout (``LAYOUT v2``) is a fixed per-group permutation of the codes
 and metadata; ``key_code_position``/``value_code_position`` and the
 ``*_meta_index`` functions state it element by element.
 
@@ -69,7 +69,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-LAYOUT_VERSION = 1
+LAYOUT_VERSION = 2
 
 
 # ---------------------------------------------------------------------------
@@ -103,7 +103,7 @@ class Config:
 
 
 def block_sections(cfg: Config) -> dict:
-    """Byte offsets and sizes of the sections of one group block (LAYOUT v1).
+    """Byte offsets and sizes of the sections of one group block (LAYOUT v2).
 
     Order: key codes, key scales, key mins, value codes, value scales,
     value mins.  All scales/mins are IEEE binary16.
@@ -246,7 +246,7 @@ def dequantize_values(codes, s16, z16, group) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# LAYOUT v1: element positions inside a group block
+# LAYOUT v2: element positions inside a group block
 # ---------------------------------------------------------------------------
 def key_code_position(t: int, c: int, d: int, bits: int):
     """(byte, bit) of key code (token t, channel c) inside the key-code section.
@@ -588,7 +588,7 @@ def cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, pack: bool = True
 
 def tail_arrays(cfg: Config, tail_k: np.ndarray, tail_v: np.ndarray, first: int = 0):
     """Place T tail tokens [T, d], the first at sequence position ``first``,
-    into the (R + G)-slot tail arrays (flat fp16, LAYOUT v1): token
+    into the (R + G)-slot tail arrays (flat fp16, LAYOUT v2): token
     first + i goes to slot tail_slot(first + i).  Slots holding no tail token
     are zero here (their device contents are unspecified)."""
     W, d = cfg.tail_slots, cfg.head_dim

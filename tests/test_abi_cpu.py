@@ -93,7 +93,7 @@ def test_bytes_per_token_head_from_library(kvq):
 @pytest.mark.parametrize("field,value", [
     ("k_bits", 3), ("k_bits", 8), ("v_bits", 1), ("group", 16), ("group", 128),
     ("head_dim", 96), ("head_dim", 256), ("n_q_heads", 30), ("n_kv_heads", 0),
-    ("max_seqs", 0), ("max_tokens", 0), ("layout_version", 2),
+    ("max_seqs", 0), ("max_tokens", 0), ("layout_version", 1), ("layout_version", 3),
     ("window", -16), ("window", 24), ("window", 1040), ("sink", -1), ("sink", 1025),
 ])
 def test_bad_config_rejected(kvq, field, value):

@@ -1,7 +1,7 @@
 """GPU parity of the quantize / pack / append / flush path (bit-exact).
 
 The CUDA append kernel must write exactly the oracle's group blocks
-(codes, fp16 scales and mins in LAYOUT v1) and fp16 tails, for prefill,
+(codes, fp16 scales and mins in LAYOUT v2) and fp16 tails, for prefill,
 per-step appends with flushes, mixed chunk sizes and every supported
 (key bits, value bits, group, head_dim), from fp16, bf16 and fp32 inputs.
 """

@@ -29,7 +29,7 @@ def test_seven_b_model_at_262k():
 @pytest.mark.parametrize("kb,vb,G,ratio", [(4, 2, 32, 4.0), (2, 2, 32, 16 / 3), (4, 2, 64, 512 / 112)])
 def test_ratio_with_fp16_metadata(kb, vb, G, ratio):
     """With one fp16 (scale, min) pair per group the real ratio is lower than
-    the pages' figure; it must agree with the block size of LAYOUT v1."""
+    the pages' figure; it must agree with the block size of LAYOUT v2."""
     assert o.compression_vs_fp16(kb, vb, G, with_metadata=True) == pytest.approx(ratio)
     cfg = o.Config(kb, vb, G, 128, 1, 1)
     assert o.fp16_bytes_per_token_head(128) / o.bytes_per_token_head(cfg) == pytest.approx(ratio)

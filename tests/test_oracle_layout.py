@@ -1,4 +1,4 @@
-"""Pins for LAYOUT v1 as the oracle states it (CPU only).
+"""Pins for LAYOUT v2 as the oracle states it (CPU only).
 
 The pages only ask for a fixed-width layout ("avoids irregular memory
 layouts", summary page; "a fixed per-token bit count", NOVA-KV abstract on
