@@ -20,6 +20,10 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libkvq.so")
+# the same library with the decode kernels' range checks compiled in
+# (-DKVQ_DEBUG): every cache, workspace, query and output index is checked
+# before its access and a failure is recorded in the workspace error word
+DEBUG_LIB = os.path.join(HERE, "libkvq_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -38,9 +42,9 @@ def _sources():
                   if f.endswith((".cu", ".cpp")))
 
 
-def _compile(src: str, verbose_ptxas: bool) -> tuple[str, str]:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [_nvcc(), *ARCH, *COMMON, "-c", src, "-o", obj]
+def _compile(src: str, verbose_ptxas: bool, debug: bool = False) -> tuple[str, str]:
+    obj = os.path.join(BUILD, os.path.basename(src) + (".debug.o" if debug else ".o"))
+    cmd = [_nvcc(), *ARCH, *COMMON, *(["-DKVQ_DEBUG"] if debug else []), "-c", src, "-o", obj]
     if verbose_ptxas and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -50,33 +54,40 @@ def _compile(src: str, verbose_ptxas: bool) -> tuple[str, str]:
 
 
 def _up_to_date(srcs) -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(DEBUG_LIB):
         return False
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(DEBUG_LIB))
     deps = list(srcs) + [os.path.join(INCLUDE, "kvq.h"), __file__]
     deps += [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile every CUDA/C++ source of the library and link libkvq.so."""
-    srcs = _sources()
-    if not force and not verbose_ptxas and _up_to_date(srcs):
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
-    with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    objs = [o for o, _ in results]
-    if verbose_ptxas:
-        with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
-            for _, log in results:
-                f.write(log)
-    tmp = LIB + ".tmp"
+def _link(objs, out: str) -> None:
+    tmp = out + ".tmp"
     cmd = [_nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, out)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    """Compile every CUDA/C++ source of the library and link libkvq.so and
+    its range-checked twin libkvq_debug.so."""
+    srcs = _sources()
+    if not force and not verbose_ptxas and _up_to_date(srcs):
+        return LIB
+    os.makedirs(BUILD, exist_ok=True)
+    jobs = [(s, False) for s in srcs] + [(s, True) for s in srcs]
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        results = list(ex.map(lambda j: _compile(j[0], verbose_ptxas and not j[1], j[1]), jobs))
+    if verbose_ptxas:
+        with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+            for (_, dbg), (_, log) in zip(jobs, results):
+                if not dbg:
+                    f.write(log)
+    _link([o for (_, dbg), (o, _) in zip(jobs, results) if not dbg], LIB)
+    _link([o for (_, dbg), (o, _) in zip(jobs, results) if dbg], DEBUG_LIB)
     return LIB
 
 

@@ -15,6 +15,7 @@
 
 #include "kvq.h"
 #include "kvq_internal.h"
+#include "kvq_split.h"
 
 struct kvq_cache {
   kvq_config cfg;
@@ -79,6 +80,8 @@ kvq_status validate_config(const kvq_config* c) {
     return fail(KVQ_ERR_CONFIG, "window must be a multiple of 16 in [0, 1024] (got %d)", c->window);
   if (c->sink < 0 || c->sink > 1024)
     return fail(KVQ_ERR_CONFIG, "sink must be in [0, 1024] (got %d)", c->sink);
+  if (c->rotate != 0 && c->rotate != 1)
+    return fail(KVQ_ERR_CONFIG, "rotate must be 0 or 1 (got %d)", c->rotate);
   // decode addresses slots (groups + tail) of all units with 32-bit prefixes
   const int64_t slices = (c->n_q_heads / c->n_kv_heads + kvq::kHeadsPerSlice - 1) / kvq::kHeadsPerSlice;
   const int64_t slots = (int64_t)c->max_seqs * c->n_kv_heads * slices * (c->max_tokens / c->group + 1);
@@ -261,25 +264,6 @@ kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype 
 }
 
 namespace {
-// Decode grid: one CTA per resident slot up to the cap.  When every
-// sequence has the same number of slots and the units fit the cap, a
-// multiple of the unit count (if it keeps >= 80% of the cap) makes every
-// CTA range end on a unit boundary: one piece per CTA, no CTA pays a
-// second prologue and merge.
-int64_t choose_grid(const kvq::Geom& g, const int32_t* lens, int n_seq, int64_t slots, int cap) {
-  int64_t grid = std::min<int64_t>(slots, cap);
-  const int64_t units = (int64_t)n_seq * g.hkv * g.slices;
-  const int w0 = kvq::unit_slots_s(lens[0], g.G, g.window, g.sink);
-  bool equal = true;
-  for (int b = 1; b < n_seq && equal; ++b)
-    equal = kvq::unit_slots_s(lens[b], g.G, g.window, g.sink) == w0;
-  if (equal && units <= cap) {
-    const int64_t alt = std::min<int64_t>(slots, units * (cap / units));
-    if (alt * 5 >= (int64_t)cap * 4) grid = alt;
-  }
-  return grid;
-}
-
 // One decode + combine pair per chunk of at most kSeqsPerLaunch sequences
 // (stream order keeps the chunks from overlapping on the workspace).
 cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
@@ -305,7 +289,7 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     int64_t slots = 0;
     for (int b = s0; b < s0 + ns; ++b)
       slots += (int64_t)g.hkv * g.slices * kvq::unit_slots_s(lens[b], g.G, g.window, g.sink);
-    const int64_t grid = std::min(max_grid, choose_grid(g, lens + s0, ns, slots, cap));
+    const int64_t grid = std::min(max_grid, kvq::choose_grid(g, lens + s0, ns, slots, cap));
     kvq::DecodeArgs a;
     a.cache = cache_buf;
     a.q = static_cast<const unsigned char*>(q) + s0 * qrow;
@@ -319,7 +303,7 @@ cudaError_t launch_decode_chunks(const kvq::Geom& g, const kvq::WsLayout& w,
     // combine kernel).  Otherwise the combine kernel: a narrow CTA moves on
     // to its next piece, which an in-kernel merge would delay.
     const int64_t units = (int64_t)ns * g.hkv * g.slices;
-    a.inline_merge = (wide && (grid / units + 1) <= 32) ? 1 : 0;
+    a.inline_merge = kvq::use_inline_merge(wide, grid, units) ? 1 : 0;
     cudaError_t e = kvq::launch_decode(g, w, a, (int)grid, wide, stream);
     if (e != cudaSuccess) return e;
   }
@@ -497,7 +481,10 @@ kvq_status kvq_workspace_status(const void* workspace, void* stream) {
   cudaError_t e = cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "reading the workspace error word");
-  if (word != 0) return fail(KVQ_ERR_DEVICE, "a decode kernel gave up a bounded wait");
+  if (word != 0)
+    return fail(KVQ_ERR_DEVICE,
+                "a decode kernel gave up a bounded wait or failed range check %d (word %#x)",
+                word >> 8, (unsigned)word);
   return ok();
 }
 

@@ -89,6 +89,61 @@ __device__ __forceinline__ uint4 load8_fp16(const void* base, int64_t idx, int d
   return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
+// Eight consecutive input elements as fp32 (exact for fp16 / bf16 / fp32).
+__device__ __forceinline__ void load8_f32(const void* base, int64_t idx, int dtype, float (&y)[8]) {
+  if (dtype == KVQ_FP32) {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+    y[0] = a.x; y[1] = a.y; y[2] = a.z; y[3] = a.w; y[4] = b.x; y[5] = b.y; y[6] = b.z; y[7] = b.w;
+    return;
+  }
+  const uint4 r = dtype == KVQ_FP16
+                      ? *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(base) + idx)
+                      : *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = dtype == KVQ_FP16
+                         ? __half22float2(*reinterpret_cast<const __half2*>(&w[i]))
+                         : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    y[2 * i] = f.x;
+    y[2 * i + 1] = f.y;
+  }
+}
+
+// Sixteen-byte chunk cc (channels 8cc .. 8cc + 7) of an input token row as
+// the cache stores it: rounded to fp16, after the rotation when `rot`.
+// Rotation ("[Framework] The Asymmetric Key-Value Cache Compression", §IV
+// stage 1: Y = X H, fast Walsh-Hadamard transform): the unnormalized
+// transform in fp32, stages h = 1, 2, ..., D/2 in that order, each pair
+// (j, j + h) of a block of 2h channels becoming (a + b, a - b), then times
+// fp32(1 / sqrt(D)) and rounded to fp16 - every step an IEEE fp32 operation
+// on the same operands in the same order for every element, so the result
+// is reproducible bit for bit.  A row is spread over D / 8 consecutive
+// lanes (chunk cc in lane cc of its lane group); stages h < 8 run inside a
+// lane, h >= 8 exchange with lane cc ^ (h / 8).  Every lane of the warp
+// must call this together (the exchanges are warp-wide); `use` = false
+// lanes load nothing and return zeros.
+template <int D>
+__device__ __forceinline__ uint4 row_chunk16(const void* base, int64_t idx, int dtype, int cc,
+                                             bool use, bool rot) {
+  if (!rot) return use ? load8_fp16(base, idx, dtype) : make_uint4(0u, 0u, 0u, 0u);
+  float y[8];
+  if (use) {
+    load8_f32(base, idx, dtype, y);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = 0.f;
+  }
+  fwht_lanes<D, 8>(y, cc);
+  const float sc = rot_scale<D>();
+  uint32_t h2[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    h2[i] = h2_as_u32(__floats2half2_rn(__fmul_rn(y[2 * i], sc), __fmul_rn(y[2 * i + 1], sc)));
+  return make_uint4(h2[0], h2[1], h2[2], h2[3]);
+}
+
 // Channels 8cc .. 8cc+7 of tail token u from the value tail, whose token
 // pairs are interleaved ([u/2][c][u%2]).
 __device__ __forceinline__ uint4 tail_v8(const __half* tailv, int u, int cc, int D) {
@@ -221,13 +276,19 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
 
   constexpr int CPR = D / 8;   // 16-byte fp16 chunks per token row
   // new sink tokens: input row j -> sink slot len0 + j (nobody reads them here)
+  const bool rot = g.rotate != 0;
+  // The loops over input rows below run whole warps (row_chunk16 exchanges
+  // across a warp when the cache rotates); a lane past the end loads nothing.
   auto write_sink = [&]() {
     __half* sinkk = reinterpret_cast<__half*>(cache + g.sinks_off + unit * g.sink_bytes);
     __half* sinkv = sinkk + (int64_t)g.sink_slots * D;
-    for (int ci = tid; ci < nsink * CPR; ci += blockDim.x) {
-      const int j = ci / CPR, cc = ci % CPR;
-      store_tail8(sinkk, sinkv, len0 + j, cc, D, load8_fp16(kin, in_idx(j, 8 * cc), dtype),
-                  load8_fp16(vin, in_idx(j, 8 * cc), dtype));
+    for (int c0 = tid - tid % 32; c0 < nsink * CPR; c0 += blockDim.x) {
+      const int ci = c0 + tid % 32;
+      const bool act = ci < nsink * CPR;
+      const int j = act ? ci / CPR : 0, cc = ci % CPR;
+      const uint4 k8 = row_chunk16<D>(kin, in_idx(j, 8 * cc), dtype, cc, act, rot);
+      const uint4 v8 = row_chunk16<D>(vin, in_idx(j, 8 * cc), dtype, cc, act, rot);
+      if (act) store_tail8(sinkk, sinkv, len0 + j, cc, D, k8, v8);
     }
   };
   if (F == 0) {
@@ -236,12 +297,15 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     // stays below W)
     write_sink();
     const int sl0 = (base0 + T0) % W;
-    for (int ci = tid; ci < (a1 - a0) * CPR; ci += blockDim.x) {
-      const int j = ci / CPR, cc = ci % CPR;
+    for (int c0 = tid - tid % 32; c0 < (a1 - a0) * CPR; c0 += blockDim.x) {
+      const int ci = c0 + tid % 32;
+      const bool act = ci < (a1 - a0) * CPR;
+      const int j = act ? ci / CPR : 0, cc = ci % CPR;
+      const uint4 k8 = row_chunk16<D>(kin, in_idx(nsink + j, 8 * cc), dtype, cc, act, rot);
+      const uint4 v8 = row_chunk16<D>(vin, in_idx(nsink + j, 8 * cc), dtype, cc, act, rot);
       int sl = sl0 + j;
       sl -= (sl >= W) ? W : 0;
-      store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(nsink + j, 8 * cc), dtype),
-                  load8_fp16(vin, in_idx(nsink + j, 8 * cc), dtype));
+      if (act) store_tail8(tailk, tailv, sl, cc, D, k8, v8);
     }
     finish();
     return;
@@ -261,14 +325,17 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     for (int j = 0; j < NCH; ++j) {
       const int ci = tid + 128 * j, r = ci / CPR, cc = ci % CPR;
       const int u = tau * G + r;
-      if (u < T0) {
+      const bool from_tail = u < T0;   // the same for the D / 8 lanes of the row
+      // every lane takes part in the (possibly rotating) input load
+      kx[j] = row_chunk16<D>(kin, in_idx(nsink + (from_tail ? 0 : u - T0), 8 * cc), dtype, cc,
+                             !from_tail, rot);
+      vx[j] = row_chunk16<D>(vin, in_idx(nsink + (from_tail ? 0 : u - T0), 8 * cc), dtype, cc,
+                             !from_tail, rot);
+      if (from_tail) {   // the old tail already holds cache tokens
         int sl = base0 + u;
         sl -= (sl >= W) ? W : 0;
         kx[j] = *reinterpret_cast<const uint4*>(tailk + sl * D + 8 * cc);
         vx[j] = tail_v8(tailv, sl, cc, D);
-      } else {
-        kx[j] = load8_fp16(kin, in_idx(nsink + u - T0, 8 * cc), dtype);
-        vx[j] = load8_fp16(vin, in_idx(nsink + u - T0, 8 * cc), dtype);
       }
     }
 #pragma unroll
@@ -488,18 +555,21 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
     const int r_lo = tau * G;
     const int r_hi = min(T0, r_lo + G);
     auto write_residues = [&](int lo, int hi) {
-      for (int ci = tid; ci < (hi - lo) * CPR; ci += blockDim.x) {
-        const int rr = lo + ci / CPR, cc = ci % CPR;
+      for (int c0 = tid - tid % 32; c0 < (hi - lo) * CPR; c0 += blockDim.x) {
+        const int ci = c0 + tid % 32;
+        const int rr = lo + (ci < (hi - lo) * CPR ? ci / CPR : 0), cc = ci % CPR;
         // the post-sink position q >= A with q = N0 + rr (mod W)
         int off = (N0 + rr - A) % W;
         off += (off < 0) ? W : 0;
         const int q = A + off;
-        if (q < a1) {
+        const bool act = ci < (hi - lo) * CPR && q < a1;
+        const int64_t r = act ? (int64_t)nsink + q - a0 : 0;
+        const uint4 k8 = row_chunk16<D>(kin, in_idx(r, 8 * cc), dtype, cc, act, rot);
+        const uint4 v8 = row_chunk16<D>(vin, in_idx(r, 8 * cc), dtype, cc, act, rot);
+        if (act) {
           int sl = base0 + rr;
           sl -= (sl >= W) ? W : 0;
-          const int64_t r = (int64_t)nsink + q - a0;
-          store_tail8(tailk, tailv, sl, cc, D, load8_fp16(kin, in_idx(r, 8 * cc), dtype),
-                      load8_fp16(vin, in_idx(r, 8 * cc), dtype));
+          store_tail8(tailk, tailv, sl, cc, D, k8, v8);
         }
       }
     };

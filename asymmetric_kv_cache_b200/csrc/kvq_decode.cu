@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
   const int T = prefix[n_seq];
   const int grid = gridDim.x;
   const int k = blockIdx.x;
-  const int start = (int)((int64_t)k * T / grid), end = (int)((int64_t)(k + 1) * T / grid);
+  int start, end;
+  cta_range(k, T, grid, &start, &end);
   if (start == end && tid < kHeadsPerSlice) {
     // an empty range (more CTAs than slots): the split record of a unit
     // counts every CTA between its first and its last slot, so publish an
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
 #pragma unroll
     for (int r = 0; r < (PK ? 2 : 1); ++r) st.m[r] = -INFINITY;
+    st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;   // unused here
     // the piece: slots [s0, s1) of unit (b, kvh, slice), slot = 16 tokens
     const int b = find_seq(prefix, n_seq, pos);
     const int L = slen[b];
@@ -305,7 +307,8 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
         bool got = mbar_wait_bounded(qbar, qphase & 1);
         got = __all_sync(0xffffffffu, got);
         if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-        convert_query<D, PK, NCW>(a.q_dtype, nh, got, warp, lane, qsm);
+        convert_query<D, PK, NCW>(a.q_dtype, nh, got, warp, lane, qsm,
+                                  reinterpret_cast<const unsigned char*>(qsm));
       }
     }
     ++qphase;
@@ -356,10 +359,9 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
     const bool whole = (s0 == 0 && s1 == wb);
     float* wts = merge + F::WTS_OFF;
     merge_weights<D, NW>(merge, wts, whole, tid);
-    const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
+    const int myslot = piece_partial_slot(k, pos, start);
     if (s0 == 0 && tid == 0) {
-      const int64_t last = (int64_t)pos + wb - 1;
-      const int kl = (int)(((last + 1) * grid - 1) / T);
+      const int kl = cta_of_slot((int64_t)pos + wb - 1, T, grid);
       const int unit = b * per_seq_units + uis;
       *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
@@ -458,7 +460,7 @@ cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
 // dominate), so the mma.sync kernel is the default.
 bool decode_tc_eligible(const Geom& g) {
   if (!(g.d == 128 && g.G == 32 && g.vb == 2 && (g.kb == 2 || g.kb == 4) && g.gqa <= 4 &&
-        g.slices == 1 && g.window == 0 && g.sink == 0))
+        g.slices == 1 && g.window == 0 && g.sink == 0 && g.rotate == 0))
     return false;
   const char* env = std::getenv("KVQ_DECODE_TC");
   return env && env[0] == '1';

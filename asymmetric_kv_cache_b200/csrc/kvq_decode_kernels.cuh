@@ -12,6 +12,7 @@
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
+#include "kvq_split.h"
 
 namespace kvq {
 namespace {
@@ -57,7 +58,10 @@ struct DecCfg {
   // 4 CTAs per SM (3 above 4 KB blocks), for calls with more units, whose
   // CTAs cross many unit boundaries: the prologue and merge of one CTA's
   // piece then overlap the other CTAs' groups.
-  static constexpr int NW = !WIDE ? 4 : (BLK <= 4096) ? 16 : (BLK <= 7680) ? 12 : 8;
+#ifndef KVQ_WIDE_WARPS_4K
+#define KVQ_WIDE_WARPS_4K 16
+#endif
+  static constexpr int NW = !WIDE ? 4 : (BLK <= 4096) ? KVQ_WIDE_WARPS_4K : (BLK <= 7680) ? 12 : 8;
   static constexpr int THREADS = NW * 32;
   static constexpr int MIN_BLOCKS = WIDE ? 1 : (BLK <= 4096) ? 4 : 3;
   // Ring stages per warp.  Two keep more bytes in flight than the HBM
@@ -94,7 +98,13 @@ struct DecCfg {
   static_assert(TAIL_EARLY || TailStage<D>::BYTES <= NST * BLK, "tail chunk fits a warp's ring");
   static_assert(TAIL_CHUNKS <= NW, "a warp per tail chunk");
   static constexpr int TAIL_OFF = QA_OFF + QA_BYTES;
-  static constexpr int BAR_OFF = TAIL_OFF + (TAIL_EARLY ? TAIL_CHUNKS * TailStage<D>::BYTES : 0);
+  // the unit's query rows rotated by H / sqrt(d), fp32 (rotating caches)
+  static constexpr int QR_OFF = TAIL_OFF + (TAIL_EARLY ? TAIL_CHUNKS * TailStage<D>::BYTES : 0);
+  static constexpr int QR_BYTES = kHeadsPerSlice * D * 4;
+  static constexpr int BAR_OFF = QR_OFF + QR_BYTES;
+  // the merge's fp32 output rows before the back-rotation (at the end of the ring)
+  static constexpr int OSCR_FLOATS = kHeadsPerSlice * D;
+  static constexpr int MAX_MERGE_PIECES = (RING / 4 - OSCR_FLOATS) / (3 * kHeadsPerSlice);
   static constexpr int SMEM_FIXED = BAR_OFF + (NW * NST + 1) * 8 + 56;
 };
 
@@ -107,6 +117,14 @@ struct WarpState {
   float z[4];           // rows: value-min terms (j < J) and sum p (row J); cols heads
   float m[PK ? 2 : 1];  // running max, log2 domain: head lane/4, or (PK) heads
                         // 2(i&1), 2(i&1)+1
+  // (PK) sums of the value product's B operands, sum_t fp16(p_t s_tj): lane
+  // (g, i) holds, in vb[0] + vb[2], the sum for head g mod 4 and channel
+  // group j = 2 (g >= 4) + (i >= 2)  (groups 2 and 3 only when d / G = 4;
+  // with d / G = 1 group 0 twice)
+  float vb[4];
+#ifdef KVQ_VB_TWO
+  float vb2[4];
+#endif
 };
 
 // Query fragments of head g = lane/4 (zeros for a padding head), channels
@@ -368,6 +386,26 @@ __device__ __forceinline__ int fp16_chunks(const Geom& g, int L, int Tb) {
   return (min(L, g.sink) + 15) / 16 + (Tb + 15) / 16;
 }
 
+// Debug builds: the key rows and value token-pair rows that staging chunk
+// kv (T tokens) reads from k and v must lie inside the cache's fp16 tail and
+// sink regions (check 4).  Always true in release builds.
+template <int D>
+__device__ __forceinline__ bool debug_fp16_rows(const Geom& g, const unsigned char* cache,
+                                                const __half* k, const __half* v, int T, int kv,
+                                                int32_t* err) {
+  if (!kDebug) return true;
+  const int rows = min(16, T - 16 * kv);
+  if (rows <= 0) return true;
+  const unsigned char* lo = cache + g.tails_off;
+  const unsigned char* hi = cache + g.total_bytes;
+  const unsigned char* k0 = reinterpret_cast<const unsigned char*>(k + (int64_t)16 * kv * D);
+  const unsigned char* k1 = reinterpret_cast<const unsigned char*>(k + (int64_t)(16 * kv + rows) * D);
+  const unsigned char* v0 = reinterpret_cast<const unsigned char*>(v + (int64_t)16 * kv * D);
+  const unsigned char* v1 = reinterpret_cast<const unsigned char*>(
+      v + (int64_t)(16 * kv + ((rows + 1) & ~1)) * D);
+  return debug_ok(k0 >= lo && k1 <= hi && v0 >= lo && v1 <= hi, err, 4);
+}
+
 // Issue the cp.async copies of tail chunk kv (16 tokens: key rows and
 // value token-pair rows) into `buf`; nothing waits here.
 template <int D>
@@ -503,7 +541,7 @@ __device__ __forceinline__ void load_query_pk(int dtype, int nh, bool ok, int la
 // layouts are those of load_query (PK = false) and load_query_pk (PK).
 template <int D, bool PK, int NCW>
 __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw, int lane,
-                                              uint4* __restrict__ qs) {
+                                              uint4* qs, const unsigned char* raw) {
   constexpr int KT = D / 16;
   static_assert(KT % NCW == 0, "k-tiles split evenly over the converting warps");
   constexpr int J = KT / NCW;
@@ -512,7 +550,6 @@ __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw
   const bool low = PK && g8 >= 4;
   const bool valid = ok && hh < nh;
   const float sc = kLog2e * rsqrtf((float)D);
-  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
   float2 x[J][2];
 #pragma unroll
   for (int j = 0; j < J; ++j) {
@@ -549,6 +586,42 @@ __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw
     }
     qs[kt * 32 + lane] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
   }
+}
+
+// Rotating caches: the unit's raw query rows (head hh at hh * D elements of
+// `raw`, dtype) rotated by H / sqrt(d) into fp32 rows `qr`, before the
+// conversion into fragments (the cache holds rotated keys, so q . k is the
+// same in the rotated domain).  Converting warp cw takes heads cw, cw + NCW,
+// ...; a lane holds D / 32 consecutive channels.
+template <int D, int NCW>
+__device__ __forceinline__ void rotate_query_rows(int dtype, int nh, bool ok, int cw, int lane,
+                                                  const unsigned char* raw, float* qr) {
+  constexpr int V = D / 32;
+  for (int hh = cw; hh < nh; hh += NCW) {
+    float y[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int idx = hh * D + V * lane + j;
+      y[j] = !ok ? 0.f
+             : dtype == KVQ_FP16 ? __half2float(reinterpret_cast<const __half*>(raw)[idx])
+             : dtype == KVQ_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw)[idx])
+                                 : reinterpret_cast<const float*>(raw)[idx];
+    }
+    fwht_lanes<D, V>(y, lane);
+#pragma unroll
+    for (int j = 0; j < V; ++j) qr[hh * D + V * lane + j] = y[j] * rot_scale<D>();
+  }
+}
+
+// A warp's four channels (4l .. 4l + 3) of a head's output row, rotated
+// back by H / sqrt(d) when `rot` (D / 4 lanes per row, aligned groups).
+template <int D>
+__device__ __forceinline__ float4 rotate_out4(float4 o, int l, bool rot) {
+  if (!rot) return o;
+  float y[4] = {o.x, o.y, o.z, o.w};
+  fwht_lanes<D, 4>(y, l);
+  const float sc = rot_scale<D>();
+  return make_float4(y[0] * sc, y[1] * sc, y[2] * sc, y[3] * sc);
 }
 
 // Per-head weights of the NW warps' pieces, (h, warp) per thread: the
@@ -613,6 +686,22 @@ __device__ __forceinline__ void softmax_pk(WarpState<D, KB, VB, G, true>& st, fl
       st.z[1] *= a1;
       st.z[2] *= a0;
       st.z[3] *= a1;
+      // the value-offset sums are indexed by head g mod 4 (their row), whose
+      // factor sits in lane h/2 as a0 (h even) or a1 (h odd)
+      const int h = (threadIdx.x >> 2) & 3;
+      const float x0 = __shfl_sync(0xffffffffu, a0, h >> 1);
+      const float x1 = __shfl_sync(0xffffffffu, a1, h >> 1);
+      const float av = (h & 1) ? x1 : x0;
+      st.vb[0] *= av;
+      st.vb[1] *= av;
+      st.vb[2] *= av;
+      st.vb[3] *= av;
+#ifdef KVQ_VB_TWO
+      st.vb2[0] *= av;
+      st.vb2[1] *= av;
+      st.vb2[2] *= av;
+      st.vb2[3] *= av;
+#endif
     }
     st.m[0] = n0;
     st.m[1] = n1;
@@ -626,10 +715,12 @@ __device__ __forceinline__ void softmax_pk(WarpState<D, KB, VB, G, true>& st, fl
   }
 }
 
+// Logits of one group in the S^T layout (first packed form): s[mt] =
+// {(token g, head 2i'), (g, 2i'+1), (g+8, 2i'), (g+8, 2i'+1)}, i' = i & 1.
 template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& st,
-                                                 const unsigned char* __restrict__ sp,
-                                                 const uint4* __restrict__ qsm, int lane) {
+__device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
+                                         const uint4* __restrict__ qsm, int lane,
+                                         float (&s)[G / 16][4]) {
   using C = DecCfg<D, KB, VB, G>;
   constexpr int NM = G / 16;
   constexpr int NT = G / 8;
@@ -681,7 +772,6 @@ __device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& 
       });
     });
   });
-  float s[NM][4];
 #pragma unroll
   for (int mt = 0; mt < NM; ++mt) {
 #pragma unroll
@@ -690,6 +780,15 @@ __device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& 
       s[mt][r] = x + __shfl_xor_sync(0xffffffffu, x, 2);   // high + low columns
     }
   }
+}
+
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& st,
+                                                 const unsigned char* __restrict__ sp,
+                                                 const uint4* __restrict__ qsm, int lane) {
+  constexpr int NM = G / 16;
+  float s[NM][4];
+  kside_pk<D, KB, VB, G>(sp, qsm, lane, s);
   uint32_t pt[NM][2];
   softmax_pk<D, NM, KB, VB, G>(st, s, pt);
   value_side<D, KB, VB, G, true>(st, sp, pt, lane);
@@ -742,14 +841,363 @@ __device__ __forceinline__ void tail_chunk_pk(WarpState<D, KB, VB, G, true>& st,
   }
 }
 
-// Largest b in [0, n) with prefix[b] <= pos (prefix[0] = 0, increasing).
-__device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int pos) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid + 1] <= pos) lo = mid + 1; else hi = mid;
+// ---------------------------------------------------------------------------
+// Packed group loop, second form (GQA group of at most 4 heads).
+//
+// Query fragments: for each pair of k-steps (kt0, kt1) = (2kp, 2kp + 1) a
+// block of QP_STRIDE bytes with four 256-byte areas indexed by (head hh,
+// i): Y = q_hi, X = q_lo, NY = -q_hi, Z = zeros, each a quad of fp16 pairs
+// {(kt0, v0), (kt0, v1), (kt1, v0), (kt1, v1)} at channels 16kt + 8v + 2i,
+// +1.  A lane (g, i) of the S^T tiles owns column g: head g mod 4, its high
+// part (g < 4) or its residual (g >= 4); it reads
+//   y = Y, x = (low ? X : Z), yn = (low ? NY : Z), qb = (low ? X : Y),
+// and builds the B operand of the code tiles as
+//   b = x s' + (y s' - fp16(yn... )) = fma(x, s', fma(y, s', fp16(yn s')))
+// with s' = s_k / m (m the code field's factor): fp16(y s') on high lanes
+// and, on low lanes, the exact residual of that product plus x s'.  Lanes
+// g and g ^ 4 read the same Y bytes, and all high lanes the same zero quad,
+// so every quad load touches half the bytes of a plain per-lane layout.
+//
+// Per pair of k-steps the corrections are two tiles instead of four:
+//  * the code offset (1024 per code) against A = the four b registers of the
+//    pair (rows g: low channel halves, rows g + 8: high halves) and a
+//    constant B of -1024: row g of the result is -1024 times the sum of
+//    column g's operands;
+//  * the key-min bias sum_c q_c z_c against A = the qb quad and a B whose
+//    columns n < 4 carry the low channel halves' mins and n >= 4 the high
+//    halves' (rows g pair with columns n < 4, rows g + 8 with n >= 4).
+// Value codes enter their tiles in the same 1024-offset form as the keys
+// (one LOP3 per pair, no fp16 arithmetic): the factor m of a code field is
+// constant along a row (channel) of V^T, and the offset mass 1024 sum_t B_t
+// is accumulated by two more tiles per 16 tokens (vb); both are removed once
+// per piece (o = (O' - 1024 vb) / m).
+constexpr int QP_STRIDE = 1024;   // bytes per pair of k-steps (Y | X | NY | Z)
+// The packed group loop's form: 1 = process_group_pk (fp16 value unpack,
+// per-k-step bias and offset tiles), 2 = process_group_pk2 (this form).
+#ifndef KVQ_PK_FORM
+#define KVQ_PK_FORM 1
+#endif
+#ifndef KVQ_KSIDE_ACC
+#define KVQ_KSIDE_ACC 1
+#endif
+
+// A lane's four query quads: byte offsets from the fragment area `base`.
+template <int D>
+struct QPtrs {
+  const unsigned char* base;
+  uint32_t y, x, yn, qb;
+};
+
+template <int D>
+__device__ __forceinline__ QPtrs<D> qptrs_pk2(const unsigned char* qbase, int lane) {
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const uint32_t idx = (uint32_t)(((g8 & 3) * 4 + i4) * 16);
+  const bool low = g8 >= 4;
+  QPtrs<D> p;
+  p.base = qbase;
+  p.y = idx;
+  p.x = low ? 256 + idx : 768u;
+  p.yn = low ? 512 + idx : 768u;
+  p.qb = low ? 256 + idx : idx;
+  return p;
+}
+
+template <int D>
+__device__ __forceinline__ uint4 ldq(const QPtrs<D>& qp, uint32_t off, int kp) {
+  return *reinterpret_cast<const uint4*>(qp.base + off + kp * QP_STRIDE);
+}
+
+// 16-byte shared-memory load at a 32-bit shared address.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// The query conversion of the second packed form: NCW warps (64 threads per
+// 32 channels of d ... one (kp, head, i) item per thread) read the unit's
+// raw rows (head hh at hh * D elements, up to 4 heads) from the same bytes,
+// meet at a named barrier, then write the Y / X / NY quads and the zero
+// quads.  Heads at or past nh (and everything when !ok) are zeros.
+template <int D, int NCW>
+__device__ __forceinline__ void convert_query_pk2(int dtype, int nh, bool ok, int ctid,
+                                                  unsigned char* qbase, const unsigned char* raw) {
+  constexpr int KP = D / 32;
+  static_assert(KP * 16 <= NCW * 32, "one item per converting thread");
+  const float sc = kLog2e * rsqrtf((float)D);
+  const int kp = ctid >> 4, hh = (ctid >> 2) & 3, i4 = ctid & 3;
+  const bool item = ctid < KP * 16;
+  const bool valid = ok && item && hh < nh;
+  float2 x[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {   // u = 2 (kt - kt0) + v
+    const int c = 16 * (2 * kp + (u >> 1)) + 8 * (u & 1) + 2 * i4;
+    const int idx = hh * D + c;
+    float2 f = make_float2(0.f, 0.f);
+    if (valid) {
+      if (dtype == KVQ_FP16) {
+        f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
+      } else if (dtype == KVQ_BF16) {
+        f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
+      } else {
+        f = *reinterpret_cast<const float2*>(raw + 4 * idx);
+      }
+    }
+    x[u] = f;
   }
-  return lo;
+  asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+  if (item) {
+    uint32_t yw[4], xw[4], nw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float x0 = x[u].x * sc, x1 = x[u].y * sc;
+      const __half2 h = __floats2half2_rn(x0, x1);
+      const float2 hf = __half22float2(h);
+      yw[u] = h2_as_u32(h);
+      nw[u] = yw[u] ^ 0x80008000u;   // -q_hi, exact
+      xw[u] = pack_h2(x0 - hf.x, x1 - hf.y);
+    }
+    unsigned char* blk = qbase + kp * QP_STRIDE + ((hh * 4 + i4) * 16);
+    *reinterpret_cast<uint4*>(blk) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+    *reinterpret_cast<uint4*>(blk + 256) = make_uint4(xw[0], xw[1], xw[2], xw[3]);
+    *reinterpret_cast<uint4*>(blk + 512) = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+    *reinterpret_cast<uint4*>(blk + 768) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <int D, int KB, int VB, int G, int NACC = KVQ_KSIDE_ACC>
+__device__ __forceinline__ void kside_pk2(const unsigned char* __restrict__ sp,
+                                          const QPtrs<D>& qp, int lane, float (&s)[G / 16][4]) {
+  using C = DecCfg<D, KB, VB, G>;
+  constexpr int NM = G / 16;
+  constexpr int NT = G / 8;
+  constexpr int KP = C::KT / 2;
+  static_assert(C::J <= 4, "at most four value channel groups");
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const bool low = g8 >= 4;
+  const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
+  const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
+  const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
+  constexpr uint32_t kH2Neg1024 = 0xE400E400u;
+
+  float acc[NACC][NM][4];   // NACC independent accumulator sets (k-step pairs kp mod NACC)
+#pragma unroll
+  for (int a = 0; a < NACC; ++a)
+#pragma unroll
+    for (int mt = 0; mt < NM; ++mt) acc[a][mt][0] = acc[a][mt][1] = acc[a][mt][2] = acc[a][mt][3] = 0.f;
+  float bacc[4] = {0.f, 0.f, 0.f, 0.f};   // key-min bias (rows: column g, see above)
+  float cacc[4] = {0.f, 0.f, 0.f, 0.f};   // minus the code offset (rows: column g)
+  // key-code words of the lane's 8-token tiles, all at once when that is at
+  // most 8 registers, else per chunk of k-step pairs
+  constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
+  constexpr int KP_PER_CH = WCH * C::FK / 4;   // k-step pairs covered by a chunk
+  static_assert(KP % KP_PER_CH == 0, "k-step pairs split evenly into code chunks");
+  static_for<KP / KP_PER_CH>([&](auto ch_) {
+    constexpr int ch = decltype(ch_)::value;
+    uint32_t kw[NT][WCH];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      lds_words<WCH>(kcw + (nt * 32 + lane) * C::LWK + ch * WCH, kw[nt]);
+    static_for<KP_PER_CH>([&](auto kk_) {
+      constexpr int kp = ch * KP_PER_CH + decltype(kk_)::value;
+      const uint4 s4 = *reinterpret_cast<const uint4*>(ksw + 4 * kp);
+      const uint4 z4 = *reinterpret_cast<const uint4*>(kzw + 4 * kp);
+      const uint4 qy = ldq(qp, qp.y, kp);
+      const uint4 qx = ldq(qp, qp.x, kp);
+      const uint4 qn = ldq(qp, qp.yn, kp);
+      const uint4 qb = ldq(qp, qp.qb, kp);
+      const uint32_t sv[4] = {s4.x, s4.y, s4.z, s4.w};
+      const uint32_t yv[4] = {qy.x, qy.y, qy.z, qy.w};
+      const uint32_t xv[4] = {qx.x, qx.y, qx.z, qx.w};
+      const uint32_t nv[4] = {qn.x, qn.y, qn.z, qn.w};
+      uint32_t b[4];   // B operands: (kt0, v0), (kt0, v1), (kt1, v0), (kt1, v1)
+      static_for<4>([&](auto u_) {
+        constexpr int u = decltype(u_)::value;
+        constexpr int p = 2 * (2 * kp + (u >> 1)) + (u & 1);   // code pair of the operand
+        constexpr int e = code_log2_mul<KB, p % C::FK>();
+        const uint32_t sm = e ? hmul2_b(sv[u], h2_pow2_neg(e)) : sv[u];
+        b[u] = hfma2_b(xv[u], sm, hfma2_b(yv[u], sm, hmul2_b(nv[u], sm)));
+      });
+      static_for<2>([&](auto t_) {
+        constexpr int t = decltype(t_)::value;
+        constexpr int kt = 2 * kp + t;
+        constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
+        static_for<NM>([&](auto mt_) {
+          constexpr int mt = decltype(mt_)::value;
+          constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
+          mma16816(acc[kp % NACC][mt], code_offset<KB, p0 % C::FK>(kw[2 * mt][w0]),
+                   code_offset<KB, p0 % C::FK>(kw[2 * mt + 1][w0]),
+                   code_offset<KB, p1 % C::FK>(kw[2 * mt][w1]),
+                   code_offset<KB, p1 % C::FK>(kw[2 * mt + 1][w1]), b[2 * t], b[2 * t + 1]);
+        });
+      });
+      mma16816(cacc, b[0], b[1], b[2], b[3], kH2Neg1024, kH2Neg1024);
+      mma16816(bacc, qb.x, qb.y, qb.z, qb.w, low ? z4.y : z4.x, low ? z4.w : z4.z);
+    });
+  });
+  // per-column corrections: column g's bias is bacc[0] on lanes i < 2 plus
+  // bacc[2] on lanes i >= 2; its offset is cacc[0] + cacc[2] on any lane
+  float cor = (i4 < 2) ? bacc[0] + (cacc[0] + cacc[2]) : bacc[2];
+  cor += __shfl_xor_sync(0xffffffffu, cor, 2);    // column g
+  cor += __shfl_xor_sync(0xffffffffu, cor, 16);   // + column g ^ 4: head g mod 4
+  const int h0 = 2 * (i4 & 1);
+  const float cor0 = __shfl_sync(0xffffffffu, cor, 4 * h0);
+  const float cor1 = __shfl_sync(0xffffffffu, cor, 4 * h0 + 4);
+#pragma unroll
+  for (int mt = 0; mt < NM; ++mt) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float y = acc[0][mt][r];
+#pragma unroll
+      for (int a = 1; a < NACC; ++a) y += acc[a][mt][r];
+      const float x = y + __shfl_xor_sync(0xffffffffu, y, 2);   // hi + lo
+      s[mt][r] = x + ((r & 1) ? cor1 : cor0);
+    }
+  }
+}
+
+// The value side of a group in the offset form (second packed form).
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void vside_pk2(WarpState<D, KB, VB, G, true>& st,
+                                          const unsigned char* __restrict__ sp,
+                                          const uint32_t (&pt)[G / 16][2], int lane) {
+  using C = DecCfg<D, KB, VB, G>;
+  const int g8 = lane >> 2, i4 = lane & 3;
+  const bool low = g8 >= 4;
+  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
+  const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
+  const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
+  const int zrow = g8 < C::J ? g8 : 0;
+  const uint32_t zsel = g8 < C::J ? 0xFFFFFFFFu : 0u;
+  const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
+  const uint32_t one_lo = low ? 0u : 0x3C003C00u, one_hi = low ? 0x3C003C00u : 0u;
+  static_for<C::KV>([&](auto kv_) {
+    constexpr int kv = decltype(kv_)::value;
+    const uint32_t bp0 = pt[kv][0], bp1 = pt[kv][1];
+    const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
+    mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
+    uint32_t sw[2 * C::J];
+    lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
+    uint32_t bs[C::J][2];
+#pragma unroll
+    for (int j = 0; j < C::J; ++j) {
+      bs[j][0] = hmul2_b(bp0, sw[2 * j]);
+      bs[j][1] = hmul2_b(bp1, sw[2 * j + 1]);
+    }
+    // offset sums: rows g < 4 take groups (0, 1), rows g >= 4 (columns that
+    // repeat heads 0-3) groups (2, 3)
+    if constexpr (C::J == 4) {
+#ifdef KVQ_VB_TWO
+      mma16816(st.vb, bs[0][0], bs[0][1], bs[1][0], bs[1][1], one_lo, one_hi);
+      mma16816(st.vb2, bs[2][0], bs[2][1], bs[3][0], bs[3][1], one_lo, one_hi);
+#else
+      mma16816(st.vb, low ? bs[2][0] : bs[0][0], low ? bs[2][1] : bs[0][1],
+               low ? bs[3][0] : bs[1][0], low ? bs[3][1] : bs[1][1], one_lo, one_hi);
+#endif
+    } else if constexpr (C::J == 2) {
+      mma16816(st.vb, bs[0][0], bs[0][1], bs[1][0], bs[1][1], one_lo, one_hi);
+    } else {
+      mma16816(st.vb, bs[0][0], bs[0][1], bs[0][0], bs[0][1], one_lo, one_hi);
+    }
+    uint32_t vw[C::LWV];
+    lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
+    static_for<C::MT>([&](auto mt_) {
+      constexpr int mt = decltype(mt_)::value;
+      constexpr int TPW = C::FV / 4;
+      constexpr int wd = mt / TPW, u = mt % TPW;
+      constexpr int j = (16 * mt) / G;
+      mma16816(st.o[mt], code_offset<VB, 2 * u>(vw[wd]), code_offset<VB, 2 * u + 1>(vw[wd]),
+               code_offset<VB, 2 * u + C::FV / 2>(vw[wd]),
+               code_offset<VB, 2 * u + 1 + C::FV / 2>(vw[wd]), bs[j][0], bs[j][1]);
+    });
+  });
+}
+
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void process_group_pk2(WarpState<D, KB, VB, G, true>& st,
+                                                  const unsigned char* __restrict__ sp,
+                                                  const QPtrs<D>& qp, int lane) {
+  constexpr int NM = G / 16;
+  float s[NM][4];
+  kside_pk2<D, KB, VB, G>(sp, qp, lane, s);
+  uint32_t pt[NM][2];
+  softmax_pk<D, NM, KB, VB, G>(st, s, pt);
+  vside_pk2<D, KB, VB, G>(st, sp, pt, lane);
+}
+
+// The field factors of the value-code rows of m-tile mt: rows g (channel
+// 16 mt + g) and rows g + 8 (see process_group_pk2).
+template <int VB>
+__host__ __device__ constexpr int vrow_log2_mul(int mt, int hi) {
+  return VB * ((2 * (mt % (16 / VB / 4)) + hi) % (8 / VB));
+}
+
+// fp16 tail chunk for the second packed form: the B operand of the key tile
+// is the lane's qb (q_hi on high lanes, q_lo on low lanes).
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void tail_chunk_pk2(WarpState<D, KB, VB, G, true>& st,
+                                               const unsigned char* __restrict__ buf, int T,
+                                               int kv, const QPtrs<D>& qp, int lane) {
+  using C = DecCfg<D, KB, VB, G>;
+  using TS = TailStage<D>;
+  const int g8 = lane >> 2, i4 = lane & 3;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
+  const unsigned char* k1 = k0 + 8 * TS::KROW;
+#pragma unroll
+  for (int kp = 0; kp < C::KT / 2; ++kp) {
+    const uint4 qb = ldq(qp, qp.qb, kp);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int kt = 2 * kp + t;
+      mma16816(acc, *reinterpret_cast<const uint32_t*>(k0 + 32 * kt),
+               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt),
+               *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16),
+               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16), t ? qb.z : qb.x,
+               t ? qb.w : qb.y);
+    }
+  }
+  const int t0 = 16 * kv + g8, t1 = t0 + 8;
+  float s[1][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float x = acc[r] + __shfl_xor_sync(0xffffffffu, acc[r], 2);
+    s[0][r] = ((r < 2 ? t0 : t1) < T) ? x : -INFINITY;
+  }
+  uint32_t pt[1][2];
+  softmax_pk<D, 1, KB, VB, G>(st, s, pt);
+  const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
+  mma16816(st.z, ones, 0u, ones, 0u, pt[0][0], pt[0][1]);
+  const int ta = 16 * kv + 2 * i4, tb = ta + 8;
+  const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+  const uint32_t mb = (tb + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
+  const unsigned char* va = buf + TS::VOFF + i4 * TS::VROW + 4 * g8;
+  const unsigned char* vb = va + 4 * TS::VROW;
+#pragma unroll
+  for (int mt = 0; mt < C::MT; ++mt) {
+    const uint32_t a0 = *reinterpret_cast<const uint32_t*>(va + 64 * mt) & ma;
+    const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
+    const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
+    const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
+    mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
+  }
+}
+
+// After a warp's fp16 chunks and before its first group: bring O to the
+// scale of the offset-form rows (row factor m, exact in fp32).
+template <int D, int KB, int VB, int G>
+__device__ __forceinline__ void scale_rows_pk2(WarpState<D, KB, VB, G, true>& st) {
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    const float f0 = (float)(1 << vrow_log2_mul<VB>(mt, 0));
+    const float f1 = (float)(1 << vrow_log2_mul<VB>(mt, 1));
+    st.o[mt][0] *= f0;
+    st.o[mt][1] *= f0;
+    st.o[mt][2] *= f1;
+    st.o[mt][3] *= f1;
+  }
 }
 
 // The last CTA to finish a split unit merges the unit's pieces.  Every
@@ -766,26 +1214,47 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
                                                const DecodeArgs& a, int unit, int64_t p0,
                                                int wb, int T, int grid, int b, int hbase, int nh,
                                                float* __restrict__ scratch, int max_pieces,
-                                               int* __restrict__ flag, int tid) {
+                                               int* __restrict__ flag, int tid, bool rot,
+                                               float* __restrict__ oscr) {
   int32_t* tickets = reinterpret_cast<int32_t*>(a.ws + w.tickets_off);
   const float* partials = reinterpret_cast<const float*>(a.ws + w.partials_off);
+  int32_t* err = reinterpret_cast<int32_t*>(a.ws + w.err_off);
   __syncthreads();
   if (tid == 0) {
-    const int kf = (int)(((p0 + 1) * grid - 1) / T);
-    const int kl = (int)(((p0 + wb) * grid - 1) / T);
-    const int npc = kl - kf + 1;
-    const int old = atomic_add_acq_rel_gpu(tickets + unit, 1);
-    const bool last = old == npc - 1;
-    if (last) tickets[unit] = 0;   // every piece has counted: ready for the next call
-    flag[0] = last ? npc : 0;
-    flag[1] = kf;
-    flag[2] = ((int64_t)kf * T / grid == p0) ? 2 * kf : 2 * kf + 1;
+    const MergePlan mp = merge_plan(p0, wb, T, grid);
+    // debug builds: the ticket, every piece's partial slot, the output rows
+    // and the shared scratch must fit their buffers (checks 10, 9, 8, 11);
+    // a failed check skips the merge
+    const bool fits =
+        debug_ok(unit >= 0 && unit < w.units, err, 10) &&
+        debug_ok(mp.kf >= 0 && merge_piece_slot(mp.kf, mp.s0, mp.npc - 1) < 2 * grid &&
+                     w.partials_off + (int64_t)2 * grid * w.slot_floats * 4 <= w.total,
+                 err, 9) &&
+        debug_ok(b < a.n_seq && hbase + nh <= g.hq, err, 8) &&
+        debug_ok(mp.npc <= 32 || mp.npc <= max_pieces, err, 11);
+    int npc = 0;
+    if (fits) {
+      const int old = atomic_add_acq_rel_gpu(tickets + unit, 1);
+      const bool last = old == mp.npc - 1;
+      if (last) tickets[unit] = 0;   // every piece has counted: ready for the next call
+      npc = last ? mp.npc : 0;
+    }
+    flag[0] = npc;
+    flag[1] = mp.kf;
+    flag[2] = mp.s0;
   }
   __syncthreads();
   const int npc = flag[0], kf = flag[1], s0 = flag[2];
   if (npc == 0) return;
   auto piece = [&](int pc, int h) {
-    return partials + (int64_t)(pc == 0 ? s0 : 2 * (kf + pc)) * w.slot_floats + h * (D + 4);
+    return partials + (int64_t)merge_piece_slot(kf, s0, pc) * w.slot_floats + h * (D + 4);
+  };
+  // the unit's output: fp16 rows of out, or (rotating caches) fp32 rows of
+  // oscr, rotated back and written by the epilogue below
+  __half* orow = reinterpret_cast<__half*>(a.out) + ((int64_t)b * g.hq + hbase) * D;
+  auto put = [&](int h, int c, float v) {
+    if (rot) oscr[h * D + c] = v;
+    else orow[h * D + c] = __float2half_rn(v);
   };
   if (npc > 4 && npc <= 32) {
     // up to 32 pieces: an item is (head, 4 channels); 4 threads share an
@@ -835,14 +1304,15 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
       }
       if (sub == 0) {
         const float inv = 1.0f / L;
-        const uint2 hv = make_uint2(pack_h2(O.x * inv, O.y * inv), pack_h2(O.z * inv, O.w * inv));
-        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.out) +
-                                  ((int64_t)b * g.hq + hbase + h) * D + c) = hv;
+        const float4 on = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+        if (rot)
+          *reinterpret_cast<float4*>(oscr + h * D + c) = on;
+        else
+          *reinterpret_cast<uint2*>(orow + h * D + c) =
+              make_uint2(pack_h2(on.x, on.y), pack_h2(on.z, on.w));
       }
     }
-    return;
-  }
-  if (npc <= 4) {
+  } else if (npc <= 4) {
     // few pieces: every thread loads its element's values and the pieces'
     // (m, l) in one round of L2 loads and forms the weights itself
     for (int idx = tid; idx < nh * D; idx += THREADS) {
@@ -867,12 +1337,9 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
         L += f * ml[pc].y;
         O += f * o[pc];
       }
-      reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-          __float2half_rn(O / L);
+      put(h, c, O / L);
     }
-    return;
-  }
-  if (npc <= max_pieces) {
+  } else if (npc <= max_pieces) {
     // (m, l) of every (piece, head) in one round of loads, then the per-head
     // weights, then every element's pieces with all loads in flight
     float* mlw = scratch;                              // [pc][h]: m, l
@@ -918,11 +1385,9 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
         const float f = wt[pc * kHeadsPerSlice + h];
         if (f != 0.f) O += f * __ldcg(piece(pc, h) + c);
       }
-      reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-          __float2half_rn(O);
+      put(h, c, O);
     }
-    return;
-  }
+  } else {
   // more pieces than the scratch holds: an online merge per element
   for (int idx = tid; idx < nh * D; idx += THREADS) {
     const int h = idx / D, c = idx % D;
@@ -938,52 +1403,23 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
       O = O * sa + o * sb;
       M = Mn;
     }
-    reinterpret_cast<__half*>(a.out)[((int64_t)b * g.hq + hbase + h) * D + c] =
-        __float2half_rn(O / L);
+    put(h, c, O / L);
   }
-}
-
-// The part of unit `unit` (sequence b, kv head kvh, head slice `slice`)
-// that a CTA processes: slots [slot0, slot1) of the unit's wb slots.
-struct Piece {
-  int b, L, ng, Tb, wb, slot0, slot1, kvh, slice, unit, hbase, nh;
-};
-
-// Built from the slot position alone, so that it can be rebuilt after the
-// group loop instead of holding registers through it.
-// (G: the group size when the caller knows it at compile time - a shift
-// instead of a division on the path to the piece's first copies - else 0;
-// WIN: the cache has a recent window, g.window > 0)
-template <int G = 0, bool WIN = false>
-__device__ __forceinline__ Piece make_piece(const Geom& g, const int32_t* prefix,
-                                            const int32_t* slen, int n_seq, int pos, int end) {
-  Piece p;
-  p.b = find_seq(prefix, n_seq, pos);
-  p.L = slen[p.b];
-  if constexpr (WIN) {
-    // the first min(L, sink) tokens stay in fp16; groups after them leave
-    // the newest `window` tokens in fp16; the sink and the tail share the
-    // unit's last (fp16) slot, Tb counts the tail alone
-    const int Sb = min(p.L, g.sink);
-    const int Lq = p.L - Sb - g.window;
-    p.ng = Lq <= 0 ? 0 : G ? Lq / G : Lq / g.G;
-    p.Tb = p.L - Sb - p.ng * (G ? G : g.G);
-    p.wb = p.ng + (p.L > p.ng * (G ? G : g.G) ? 1 : 0);
-  } else {
-    p.ng = G ? p.L / G : p.L / g.G;
-    p.Tb = p.L - p.ng * (G ? G : g.G);
-    p.wb = p.ng + (p.Tb ? 1 : 0);
   }
-  const int local = pos - prefix[p.b];
-  const int uis = local / p.wb;
-  p.slot0 = local - uis * p.wb;
-  p.slot1 = min(p.wb, p.slot0 + (end - pos));
-  p.kvh = g.slices == 1 ? uis : uis / g.slices;
-  p.slice = uis - p.kvh * g.slices;
-  p.unit = p.b * (g.hkv * g.slices) + uis;
-  p.hbase = p.kvh * g.gqa + p.slice * kHeadsPerSlice;
-  p.nh = min(kHeadsPerSlice, g.gqa - p.slice * kHeadsPerSlice);
-  return p;
+  if (rot) {
+    // rotating caches: each head's fp32 row rotated back by H / sqrt(d),
+    // four channels per lane (whole warps, D / 4 lanes per row)
+    __syncthreads();
+    for (int i0 = tid - tid % 32; i0 < nh * (D / 4); i0 += THREADS) {
+      const int idx = i0 + tid % 32;
+      const bool act = idx < nh * (D / 4);
+      const int h = act ? idx / (D / 4) : 0, l = idx % (D / 4);
+      const float4 O = rotate_out4<D>(*reinterpret_cast<const float4*>(oscr + h * D + 4 * l), l, true);
+      if (act)
+        *reinterpret_cast<uint2*>(orow + h * D + 4 * l) =
+            make_uint2(pack_h2(O.x, O.y), pack_h2(O.z, O.w));
+    }
+  }
 }
 
 // WIN: compiled for caches with a recent window (tails of up to R + G - 1
@@ -996,6 +1432,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
   using C = DecCfg<D, KB, VB, G, WIDE>;
   constexpr int NW = C::NW;
+  constexpr bool PK2 = PK && KVQ_PK_FORM == 2;   // the second packed form
   static_assert(C::NST == 2, "the ring rotation below holds two stages");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int32_t wsum[NW];
@@ -1083,14 +1520,30 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
   const int T = prefix[n_seq];
   const int grid = gridDim.x;
   const int k = blockIdx.x;
-  const int start = (int)((int64_t)k * T / grid), end = (int)((int64_t)(k + 1) * T / grid);
-  if (start == end && tid < kHeadsPerSlice) {
-    // an empty range (more CTAs than slots): the split record of a unit
-    // counts every CTA between its first and its last slot, so publish an
-    // empty piece (m = -inf, l = 0) that the combine skips
-    float* ps = partials + (int64_t)(2 * k) * w.slot_floats + tid * (D + 4);
-    ps[D] = -INFINITY;
-    ps[D + 1] = 0.f;
+  int start, end;
+  cta_range(k, T, grid, &start, &end);
+  if (start == end) {
+    // an empty range (more CTAs than slots; the host never plans one, but a
+    // captured decode replayed over shorter lengths can meet it): the split
+    // record of a unit counts every CTA between its first and its last
+    // slot, so publish an empty piece (m = -inf, l = 0) that the merge
+    // skips, and, when split units are merged in the kernel, count it on
+    // the ticket of the unit whose span it lies in (the unit holding slot
+    // `start`, unless that slot is the unit's first)
+    if (tid < kHeadsPerSlice &&
+        debug_ok(w.partials_off + (int64_t)(2 * k + 1) * w.slot_floats * 4 <= w.total, err, 13)) {
+      float* ps = partials + (int64_t)(2 * k) * w.slot_floats + tid * (D + 4);
+      ps[D] = -INFINITY;
+      ps[D + 1] = 0.f;
+    }
+    if (a.inline_merge && start < T) {
+      const Piece p = make_piece<0, WIN>(g, prefix, slen, n_seq, start, start + 1);
+      if (p.slot0 > 0)
+        finish_split_unit<D, C::THREADS>(g, w, a, p.unit, (int64_t)start - p.slot0, p.wb, T,
+                                         grid, p.b, p.hbase, p.nh, merge, C::MAX_MERGE_PIECES,
+                                         ticket_flag, tid, g.rotate != 0,
+                                         merge + C::RING / 4 - C::OSCR_FLOATS);
+    }
   }
 
   // The warp's 2-stage ring: `head` is the stage consumed next, bit s of
@@ -1111,6 +1564,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
 #pragma unroll
     for (int r = 0; r < (PK ? 2 : 1); ++r) st.m[r] = -INFINITY;
+    st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;
+#ifdef KVQ_VB_TWO
+    st.vb2[0] = st.vb2[1] = st.vb2[2] = st.vb2[3] = 0.f;
+#endif
 
     int ngr, nh;         // groups in this piece, heads of the unit
     int64_t gb;          // global block index of the piece's first group
@@ -1131,12 +1588,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       if (tid == 0) {
         const int esz = a.q_dtype == KVQ_FP32 ? 4 : 2;
         const uint32_t qbytes = (uint32_t)(p.nh * D * esz);
+        const unsigned char* q0 = static_cast<const unsigned char*>(a.q);
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(qbar, qbytes);
-        bulk_copy_g2s(qsm,
-                      static_cast<const unsigned char*>(a.q) +
-                          ((int64_t)p.b * g.hq + p.hbase) * D * esz,
-                      qbytes, qbar);
+        checked_bulk_copy(qsm, q0 + ((int64_t)p.b * g.hq + p.hbase) * D * esz, qbytes, qbar, q0,
+                          q0 + (int64_t)a.n_seq * g.hq * D * esz, err, 1);
       }
       if (my_tail) {
         const __half* tk = reinterpret_cast<const __half*>(
@@ -1146,9 +1601,11 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
           const __half *ck, *cv;
           const int Tc = fp16_chunk_src<D, G>(g, a.cache, (int64_t)(a.seq0 + p.b) * g.hkv + p.kvh,
                                               p.L, p.ng, p.Tb, warp, ck, cv);
-          stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
+          if (debug_fp16_rows<D>(g, a.cache, ck, cv, Tc, 0, err))
+            stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
         } else {
-          stage_tail_chunk<D>(tb, tk, tk + G * D, p.Tb, warp, lane);
+          if (debug_fp16_rows<D>(g, a.cache, tk, tk + G * D, p.Tb, warp, err))
+            stage_tail_chunk<D>(tb, tk, tk + G * D, p.Tb, warp, lane);
         }
       }
     }
@@ -1160,8 +1617,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         const int c = atomicAdd(&claim, 1);
         if (c < ngr) {
           gi = c;
-          mbar_arrive_expect_tx(&wbars[stg], C::BLK);
-          bulk_copy_g2s(wring + stg * C::BLK, blocks + (gb + c) * C::BLK, C::BLK, &wbars[stg]);
+          checked_bulk_copy(wring + stg * C::BLK, blocks + (gb + c) * C::BLK, C::BLK, &wbars[stg],
+                            blocks, a.cache + g.tails_off, err, 2);
         }
       }
       return __shfl_sync(0xffffffffu, gi, 0);
@@ -1174,14 +1631,29 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     }
     // while the blocks fly, the first warps turn the query rows into fragments
     {
-      constexpr int NCW = (NW < D / 16) ? NW : D / 16;   // converting warps
+      // converting warps: one per k-step of d/16 (second packed form: one
+      // item per thread)
+      constexpr int NCW = PK2 ? (D / 32 * 16 + 31) / 32 : ((NW < D / 16) ? NW : D / 16);
       if (warp < NCW) {
         bool got = mbar_wait_bounded(qbar, qphase & 1);
         got = __all_sync(0xffffffffu, got);
         if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-        convert_query<D, PK, NCW>(a.q_dtype, nh, got, warp, lane, qsm);
+        const unsigned char* src = smem + C::QA_OFF;
+        int sdt = a.q_dtype;
+        if (g.rotate) {   // rotate the raw rows first (fp32), then convert those
+          float* qr = reinterpret_cast<float*>(smem + C::QR_OFF);
+          rotate_query_rows<D, NCW>(a.q_dtype, nh, got, warp, lane, src, qr);
+          asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+          src = reinterpret_cast<const unsigned char*>(qr);
+          sdt = KVQ_FP32;
+        }
+        if constexpr (PK2)
+          convert_query_pk2<D, NCW>(sdt, nh, got, tid, smem + C::QA_OFF, src);
+        else
+          convert_query<D, PK, NCW>(sdt, nh, got, warp, lane, qsm, src);
       }
     }
+    const QPtrs<D> qp = qptrs_pk2<D>(smem + C::QA_OFF, lane);
     ++qphase;
     __syncthreads();
     if (my_tail) {
@@ -1190,7 +1662,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       unsigned char* tb = C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
       if constexpr (!WIN) {
         const Piece p = piece_s;
-        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+        if constexpr (PK2) tail_chunk_pk2<D, KB, VB, G>(st, tb, p.Tb, warp, qp, lane);
+        else if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
         else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
       } else {
         // fp16 chunks warp, warp + TAIL_CHUNKS, ... (sink chunks first, then
@@ -1203,16 +1676,19 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
           const int Tc = fp16_chunk_src<D, G>(g, a.cache, ui, p.L, p.ng, p.Tb, c, ck, cv);
           if (c != warp) {
             __syncwarp();   // every lane's reads of the stage are done
-            stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
+            if (debug_fp16_rows<D>(g, a.cache, ck, cv, Tc, 0, err))
+              stage_tail_chunk<D>(tb, ck, cv, Tc, 0, lane);
             cp_async_wait_all();
             __syncwarp();
           }
-          if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+          if constexpr (PK2) tail_chunk_pk2<D, KB, VB, G>(st, tb, Tc, 0, qp, lane);
+          else if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
           else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
           c += C::TAIL_CHUNKS;
           if (c >= nck) break;
         }
       }
+      if constexpr (PK2) scale_rows_pk2<D, KB, VB, G>(st);   // before any group
       if (!C::TAIL_EARLY) {   // the ring is free again: start its copies
         __syncwarp();
         cur = claim_into(head);
@@ -1232,7 +1708,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         break;
       }
       phase ^= 1u << head;
-      if constexpr (PK) process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+      if constexpr (PK2) process_group_pk2<D, KB, VB, G>(st, wring + head * C::BLK, qp, lane);
+      else if constexpr (PK) process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
       else process_group<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
       __syncwarp();
       // refill the stage: the warp's reads of it are complete (their values
@@ -1242,8 +1719,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       int nn = -1;
       if (lane == 0 && nc >= 0 && nc < ngr) {
         nn = nc;
-        mbar_arrive_expect_tx(&wbars[head], C::BLK);
-        bulk_copy_g2s(wring + head * C::BLK, blocks + (gb + nc) * C::BLK, C::BLK, &wbars[head]);
+        checked_bulk_copy(wring + head * C::BLK, blocks + (gb + nc) * C::BLK, C::BLK, &wbars[head],
+                          blocks, a.cache + g.tails_off, err, 3);
       }
       nn = __shfl_sync(0xffffffffu, nn, 0);
       cur = nxt;
@@ -1276,15 +1753,48 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       if constexpr (PK) {
         // columns 4-7 repeat heads 0-3 bit for bit (the same B columns and
         // rescale factors), so lanes i4 >= 2 store the channel + 8 half of
-        // lane i4 - 2's heads: every lane stores two values per m-tile
+        // lane i4 - 2's heads: every lane stores two values per m-tile.
+        // Value rows carry the code offset and the field factor m:
+        // o = (O' - 1024 sum_t B_t) / m, the sums of head h and channel
+        // group j held by lane 4h + 2(j & 1) (process_group_pk2).
         const int hh = 2 * (i4 & 1);
         const int co = (i4 >= 2) ? 8 : 0;
+        float sb0[C::J], sb1[C::J];   // second form: 1024 sum_t B_t per (group j, head)
+        if constexpr (PK2) {
+        const float vs = st.vb[0] + st.vb[2];
+#ifdef KVQ_VB_TWO
+        const float vs2 = st.vb2[0] + st.vb2[2];
+#pragma unroll
+        for (int j = 0; j < C::J; ++j) {
+          const float x = (j >= 2 && C::J == 4) ? vs2 : vs;
+          const int src = 4 * hh + 2 * (j & 1);
+          sb0[j] = 1024.f * __shfl_sync(0xffffffffu, x, src);
+          sb1[j] = 1024.f * __shfl_sync(0xffffffffu, x, src + 4);
+        }
+#else
+#pragma unroll
+        for (int j = 0; j < C::J; ++j) {
+          const int src = 4 * hh + 16 * (j >> 1) + 2 * (j & 1);   // lane (h + 4 (j >= 2), j odd)
+          sb0[j] = 1024.f * __shfl_sync(0xffffffffu, vs, src);
+          sb1[j] = 1024.f * __shfl_sync(0xffffffffu, vs, src + 4);
+        }
+#endif
+        }
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
           const int c = 16 * mt + g8 + co;
           const int j = (16 * mt) / G;
-          mo[hh * RS + c] = ((i4 >= 2) ? st.o[mt][2] : st.o[mt][0]) + zl0[j];
-          mo[(hh + 1) * RS + c] = ((i4 >= 2) ? st.o[mt][3] : st.o[mt][1]) + zl1[j];
+          const float o0 = (i4 >= 2) ? st.o[mt][2] : st.o[mt][0];
+          const float o1 = (i4 >= 2) ? st.o[mt][3] : st.o[mt][1];
+          if constexpr (PK2) {
+            const float inv = (i4 >= 2) ? 1.f / (float)(1 << vrow_log2_mul<VB>(mt, 1))
+                                        : 1.f / (float)(1 << vrow_log2_mul<VB>(mt, 0));
+            mo[hh * RS + c] = (o0 - sb0[j]) * inv + zl0[j];
+            mo[(hh + 1) * RS + c] = (o1 - sb1[j]) * inv + zl1[j];
+          } else {
+            mo[hh * RS + c] = o0 + zl0[j];
+            mo[(hh + 1) * RS + c] = o1 + zl1[j];
+          }
         }
         if (g8 == 0 && i4 < 2) {
           mo[(2 * i4) * RS + D] = st.m[0];
@@ -1315,21 +1825,29 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     merge_weights<D, NW, C::MRS>(merge, wts, whole, tid);
     // Partial slots: a CTA holds at most two split pieces, its first (slot
     // 2k) and its last (2k + 1); pieces in between are whole units.
-    const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
+    const int myslot = piece_partial_slot(k, pos, start);
     if (slot0 == 0 && tid == 0) {
       // split record of the unit for the combine kernel: its first partial
       // slot and the number of CTAs holding a piece of it
-      const int64_t last = (int64_t)pos + wb - 1;   // the unit's last slot
-      const int kl = (int)(((last + 1) * grid - 1) / T);
-      *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
+      const int kl = cta_of_slot((int64_t)pos + wb - 1, T, grid);   // the unit's last slot
+      if (debug_ok(unit >= 0 && unit < w.units, err, 7))
+        *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
+    const bool slot_ok =
+        whole || debug_ok(myslot < 2 * grid &&
+                              w.partials_off + (int64_t)(myslot + 1) * w.slot_floats * 4 <= w.total,
+                          err, 6);
+    const bool out_ok = debug_ok(b < a.n_seq && hbase + nh <= g.hq, err, 8);
     __syncthreads();
     // four channels per thread: 128-bit loads of the warps' rows, 128-bit
     // partial stores (rows of D + 8 floats and partial rows of D + 4 keep
     // every such address 16-byte aligned)
     static_assert(C::MRS % 4 == 0 && (D + 4) % 4 == 0, "16-byte aligned merge rows");
-    for (int idx = tid; idx < nh * (D / 4); idx += C::THREADS) {
-      const int h = idx / (D / 4), c = 4 * (idx % (D / 4));
+    const bool rot_out = whole && g.rotate != 0;   // final rows of a rotating cache
+    for (int i0 = tid - lane; i0 < nh * (D / 4); i0 += C::THREADS) {
+      const int idx = i0 + lane;
+      const bool act = idx < nh * (D / 4);
+      const int h = act ? idx / (D / 4) : 0, c = 4 * (idx % (D / 4));
       const float* f = wts + h * NW;
       const float* mo = merge + h * C::MRS + c;
       constexpr int WS = kHeadsPerSlice * C::MRS;   // stride between the warps' areas
@@ -1343,11 +1861,14 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         O.z = fmaf(fw, x.z, O.z);
         O.w = fmaf(fw, x.w, O.w);
       }
+      O = rotate_out4<D>(O, idx % (D / 4), rot_out);
+      if (!act) continue;
       if (whole) {
         const uint2 hv = make_uint2(pack_h2(O.x, O.y), pack_h2(O.z, O.w));
-        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.out) +
-                                  ((int64_t)b * g.hq + hbase + h) * D + c) = hv;
-      } else {
+        if (out_ok)
+          *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.out) +
+                                    ((int64_t)b * g.hq + hbase + h) * D + c) = hv;
+      } else if (slot_ok) {
         float* ps = partials + myslot * w.slot_floats + h * (D + 4);
         *reinterpret_cast<float4*>(ps + c) = O;
         if (c == 0) {
@@ -1358,8 +1879,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     }
     if (!whole && a.inline_merge)
       finish_split_unit<D, C::THREADS>(g, w, a, unit, (int64_t)pos - slot0, wb, T, grid, b, hbase,
-                                       nh, merge, C::RING / (4 * 3 * kHeadsPerSlice), ticket_flag,
-                                       tid);
+                                       nh, merge, C::MAX_MERGE_PIECES, ticket_flag, tid,
+                                       g.rotate != 0, merge + C::RING / 4 - C::OSCR_FLOATS);
     fence_proxy_async_smem();   // generic accesses before the next bulk copies
     __syncthreads();            // merge area and ctl are reused by the next piece
     pos += slot1 - slot0;
@@ -1399,9 +1920,17 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Geom g, 
   const int kvh = uis / g.slices, slice = uis % g.slices;
   const int nh = min(kHeadsPerSlice, g.gqa - slice * kHeadsPerSlice);
   active = active && npc > 1 && h < nh;
-  const float* part = reinterpret_cast<const float*>(a.ws + w.partials_off) + h * (D + 4);
   const int kf = sl0 / 2;
-  auto piece = [&](int pc) { return part + (int64_t)(pc == 0 ? sl0 : 2 * (kf + pc)) * w.slot_floats; };
+  // debug builds: the record's pieces and the output row must fit (checks 12, 8)
+  if (active && kDebug) {
+    int32_t* err = reinterpret_cast<int32_t*>(a.ws + w.err_off);
+    active = debug_ok(sl0 >= 0 && w.partials_off + (int64_t)(merge_piece_slot(kf, sl0, npc - 1) + 1) *
+                                                        w.slot_floats * 4 <= w.total,
+                      err, 12) &&
+             debug_ok(b < a.n_seq, err, 8);
+  }
+  const float* part = reinterpret_cast<const float*>(a.ws + w.partials_off) + h * (D + 4);
+  auto piece = [&](int pc) { return part + (int64_t)merge_piece_slot(kf, sl0, pc) * w.slot_floats; };
 
   float acc[CPL];
 #pragma unroll
@@ -1459,13 +1988,19 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const Geom g, 
   }
   if (wi == 0 && active) {
     const float inv = 1.0f / lsum;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[c] *= inv;
+    if (g.rotate) {   // rotating cache: the head's row rotated back (one warp)
+      fwht_lanes<D, CPL>(acc, lane);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[c] *= rot_scale<D>();
+    }
     const int hbase = kvh * g.gqa + slice * kHeadsPerSlice;
     __half* o = reinterpret_cast<__half*>(a.out) + ((int64_t)b * g.hq + hbase + h) * D + lane * CPL;
     if constexpr (CPL == 4) {
-      *reinterpret_cast<uint2*>(o) =
-          make_uint2(pack_h2(acc[0] * inv, acc[1] * inv), pack_h2(acc[2] * inv, acc[3] * inv));
+      *reinterpret_cast<uint2*>(o) = make_uint2(pack_h2(acc[0], acc[1]), pack_h2(acc[2], acc[3]));
     } else {
-      *reinterpret_cast<uint32_t*>(o) = pack_h2(acc[0] * inv, acc[1] * inv);
+      *reinterpret_cast<uint32_t*>(o) = pack_h2(acc[0], acc[1]);
     }
   }
 }

@@ -308,11 +308,22 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
   const int Tsl = prefix[n_seq];
   const int grid = gridDim.x;
   const int k = blockIdx.x;
-  const int start = (int)((int64_t)k * Tsl / grid), end = (int)((int64_t)(k + 1) * Tsl / grid);
-  if (start == end && tid < kHeadsPerSlice) {
-    float* ps = partials + (int64_t)(2 * k) * w.slot_floats + tid * (D + 4);
-    ps[D] = -INFINITY;
-    ps[D + 1] = 0.f;
+  int start, end;
+  cta_range(k, Tsl, grid, &start, &end);
+  if (start == end) {   // as in decode_kernel: an empty piece, counted on its unit's ticket
+    if (tid < kHeadsPerSlice) {
+      float* ps = partials + (int64_t)(2 * k) * w.slot_floats + tid * (D + 4);
+      ps[D] = -INFINITY;
+      ps[D + 1] = 0.f;
+    }
+    if (a.inline_merge && start < Tsl) {
+      const Piece p = make_piece(g, prefix, slen, n_seq, start, start + 1);
+      if (p.slot0 > 0)
+        finish_split_unit<D, T::THREADS>(g, w, a, p.unit, (int64_t)start - p.slot0, p.wb, Tsl,
+                                         grid, p.b, p.hbase, p.nh, reinterpret_cast<float*>(smem),
+                                         T::NS * T::BLK / (4 * 3 * kHeadsPerSlice), ticket_flag,
+                                         tid, false, nullptr);
+    }
   }
 
   bool ok = true;
@@ -375,7 +386,8 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
       bool got = mbar_wait_bounded(&bars[T::B_Q], qphase & 1);
       got = __all_sync(0xffffffffu, got);
       if (!got && lane == 0) atomicExch(err, KVQ_ERR_DEVICE);
-      convert_query<D, true, 4>(a.q_dtype, nh, got, warp, lane, qsm);
+      convert_query<D, true, 4>(a.q_dtype, nh, got, warp, lane, qsm,
+                                reinterpret_cast<const unsigned char*>(qsm));
     }
     ++qphase;
     __syncthreads();
@@ -806,6 +818,7 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
       for (int m2 = 0; m2 < C::MT; ++m2) st.o[m2][0] = st.o[m2][1] = st.o[m2][2] = st.o[m2][3] = 0.f;
       st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
       st.m[0] = st.m[1] = -INFINITY;
+      st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;   // unused here
       if (has_tail) {
         cp_async_wait_all();
         __syncwarp();
@@ -857,10 +870,9 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
     const bool whole = (slot0 == 0 && slot1 == wb);
     float* wts = merge + T::WTS_OFF;
     merge_weights<D, 2>(merge, wts, whole, tid);
-    const int myslot = (pos == start) ? 2 * k : 2 * k + 1;
+    const int myslot = piece_partial_slot(k, pos, start);
     if (slot0 == 0 && tid == 0) {
-      const int64_t last = (int64_t)pos + wb - 1;
-      const int kl = (int)(((last + 1) * grid - 1) / Tsl);
+      const int kl = cta_of_slot((int64_t)pos + wb - 1, Tsl, grid);
       *reinterpret_cast<int2*>(a.ws + w.units_off + 8LL * unit) = make_int2(myslot, kl - k + 1);
     }
     __syncthreads();
@@ -886,7 +898,7 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
       finish_split_unit<D, T::THREADS>(g, w, a, unit, (int64_t)pos - slot0, wb, Tsl, grid, b,
                                        hbase, nh, reinterpret_cast<float*>(smem),
                                        T::NS * T::BLK / (4 * 3 * kHeadsPerSlice), ticket_flag,
-                                       tid);
+                                       tid, false, nullptr);
     fence_proxy_async_smem();
     __syncthreads();
     tile_base += ntiles;

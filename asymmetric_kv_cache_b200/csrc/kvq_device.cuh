@@ -17,6 +17,25 @@ namespace kvq {
 // hanging; no correct launch ever gets near the cap.
 constexpr uint32_t kWaitSpinLimit = 1u << 24;
 
+// Debug builds (-DKVQ_DEBUG, libkvq_debug.so) check the index of every
+// cache, workspace, query and output access of the decode kernels against
+// its buffer before making it; a check that fails records KVQ_ERR_DEVICE
+// with the check's number (bits 8 and up) in the workspace error word and
+// the access is skipped.  Release builds compile the checks away.
+#ifdef KVQ_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+
+__device__ __forceinline__ bool debug_ok(bool cond, int32_t* err, int code) {
+  if (kDebug && !cond) {
+    atomicCAS(err, 0, 10 | (code << 8));   // 10 = KVQ_ERR_DEVICE; the first failure wins
+    return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -60,6 +79,21 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// A bulk copy of `bytes` from src, which must lie in [lo, hi): debug builds
+// skip a copy that would leave the range (the barrier phase still completes,
+// with no data) and record the failed check.
+__device__ __forceinline__ void checked_bulk_copy(void* dst, const unsigned char* src,
+                                                  uint32_t bytes, uint64_t* bar,
+                                                  const unsigned char* lo, const unsigned char* hi,
+                                                  int32_t* err, int code) {
+  if (!debug_ok(src >= lo && src + bytes <= hi, err, code)) {
+    mbar_arrive(bar);
+    return;
+  }
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_copy_g2s(dst, src, bytes, bar);
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
@@ -187,6 +221,43 @@ __device__ __forceinline__ uint32_t unpack_pair(uint32_t w) {
   constexpr int e = code_log2_mul<BITS, F_IDX>();
   constexpr uint32_t kOff = 0x8000u | ((uint32_t)(25 - e) << 10);   // -2^(10-e)
   return hfma2_b(code_offset<BITS, F_IDX>(w), h2_pow2_neg(e), kOff | (kOff << 16));
+}
+
+// Walsh-Hadamard rotation ("[Framework] The Asymmetric Key-Value Cache
+// Compression", §IV stage 1: Y = X H, H an orthogonal +-1 matrix applied by
+// the fast Walsh-Hadamard transform).  A row of D values is spread over D / V
+// consecutive lanes, V consecutive values per lane (lane index l within the
+// row).  Unnormalized transform in IEEE fp32: stages h = 1, 2, ..., D / 2 in
+// that order, each pair (j, j + h) of a block of 2h values becoming (a + b,
+// a - b); stages h < V inside a lane, the others with lane l ^ (h / V).
+// Every lane of the warp must call it together.
+template <int D, int V>
+__device__ __forceinline__ void fwht_lanes(float (&y)[V], int l) {
+#pragma unroll
+  for (int h = 1; h < V; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (j & h) continue;
+      const float a = y[j], b = y[j + h];
+      y[j] = __fadd_rn(a, b);
+      y[j + h] = __fsub_rn(a, b);
+    }
+  }
+#pragma unroll
+  for (int hl = 1; hl < D / V; hl <<= 1) {
+    const bool upper = (l & hl) != 0;   // this lane holds the b of each pair
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const float p = __shfl_xor_sync(0xffffffffu, y[j], hl);
+      y[j] = upper ? __fsub_rn(p, y[j]) : __fadd_rn(y[j], p);
+    }
+  }
+}
+// fp32(1 / sqrt(D)), the normalization of the rotation (rounded once).
+template <int D>
+__host__ __device__ constexpr float rot_scale() {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  return D == 64 ? 0.125f : 0.0883883461356163f;   // 2^-3.5 = 0.08838834764.. -> fp32
 }
 
 // Compile-time loop: f(std::integral_constant<int, i>) for i = 0 .. N-1.

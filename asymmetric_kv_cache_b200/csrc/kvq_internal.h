@@ -36,6 +36,7 @@ struct Geom {
   int32_t window, tail_slots;   // R, and W = R + G slots of the fp16 tail ring
   int32_t sink, sink_slots;     // S, and SW = S rounded up to 16 sink slots
   int64_t sinks_off, sink_bytes;
+  int32_t rotate;               // tokens, q and the output rotated by H / sqrt(d)
 };
 
 // Workspace of kvq_decode: [error word | per-unit split records | per-unit
@@ -91,6 +92,7 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->tail_slots = c.window + c.group;
   g->sink = c.sink;
   g->sink_slots = (c.sink + 15) / 16 * 16;
+  g->rotate = c.rotate;
   const int G = g->G, d = g->d, J = g->J;
   int off = 0;
   g->sec_kcodes = off; off += G * d * g->kb / 8;

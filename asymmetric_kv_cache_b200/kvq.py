@@ -14,10 +14,14 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvq.so")
+# KVQ_LIBRARY=debug selects libkvq_debug.so, the same library with the
+# decode kernels' range checks compiled in (a failed check is reported by
+# kvq_workspace_status instead of faulting)
+_NAME = "libkvq_debug.so" if os.environ.get("KVQ_LIBRARY") == "debug" else "libkvq.so"
+LIB_PATH = os.path.join(_HERE, _NAME)
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libkvq.so not found at {LIB_PATH}; build it with "
+    raise ImportError(f"{_NAME} not found at {LIB_PATH}; build it with "
                       "`python -m asymmetric_kv_cache_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -34,7 +38,7 @@ LAYOUT_VERSION = 2
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "k_bits", "v_bits", "group", "head_dim", "n_q_heads", "n_kv_heads",
-        "max_seqs", "max_tokens", "layout_version", "window", "sink")]
+        "max_seqs", "max_tokens", "layout_version", "window", "sink", "rotate")]
 
 
 class KvqLayout(ctypes.Structure):
@@ -104,9 +108,9 @@ def check(status: int, where: str) -> None:
 
 
 def make_config(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                max_tokens, window=0, sink=0) -> KvqConfig:
+                max_tokens, window=0, sink=0, rotate=0) -> KvqConfig:
     return KvqConfig(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                     max_tokens, LAYOUT_VERSION, window, sink)
+                     max_tokens, LAYOUT_VERSION, window, sink, int(rotate))
 
 
 def required_bytes(cfg: KvqConfig) -> tuple[int, int]:
@@ -148,6 +152,7 @@ class CacheSpec:
     max_tokens: int
     window: int = 0     # R: recent tokens kept in fp16 beyond the partial group
     sink: int = 0       # S: first tokens of each sequence kept in fp16
+    rotate: int = 0     # 1: tokens, q and the output rotated by H / sqrt(d)
 
 
 class KVQCache:
@@ -161,7 +166,7 @@ class KVQCache:
         self.spec = spec
         self.cfg = make_config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim,
                                spec.n_q_heads, spec.n_kv_heads, spec.max_seqs, spec.max_tokens,
-                               spec.window, spec.sink)
+                               spec.window, spec.sink, spec.rotate)
         cache_bytes, ws_bytes = required_bytes(self.cfg)
         self.buffer = torch.empty(cache_bytes, dtype=torch.uint8, device=device)
         self.workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)

@@ -36,7 +36,14 @@
  * attention-sink tokens) the first S tokens of a sequence stay in fp16 as
  * well; groups are cut from position S on and the rule above applies to the
  * tokens after the sink.  Query head h reads kv head h / (n_q_heads /
- * n_kv_heads).
+ * n_kv_heads).  With kvq_config.rotate ("[Framework] The Asymmetric Key-Value
+ * Cache Compression", §IV stage 1: Y = X H with an orthogonal +-1 matrix,
+ * fast Walsh-Hadamard transform; "Asymmetric Key-Value Quantization: 2-Bit
+ * Values and 4-Bit Keys under Long-Context Drift", §3.1: keys and values
+ * rotated before quantization) every K/V token is rotated before all of the
+ * above, so the whole cache (groups, tail, sink) holds rotated tokens; q .
+ * k is unchanged when q is rotated the same way, and the output is rotated
+ * back (H / sqrt(d) is symmetric and its own inverse).
  *
  * Conventions
  * -----------
@@ -144,6 +151,13 @@ typedef struct {
                               n mod G tail */
   int32_t sink;            /* S: first tokens of each sequence kept in fp16,
                               in [0, 1024]; 0 = none */
+  int32_t rotate;          /* 1: every K/V token is rotated by the normalized
+                              Walsh-Hadamard matrix H / sqrt(d) before it
+                              enters the cache (fp32 butterfly, stages h = 1,
+                              2, .., d/2 with (a, b) -> (a + b, a - b), times
+                              fp32(1 / sqrt(d)), then fp16); the decode
+                              rotates q the same way and rotates its output
+                              back.  0: no rotation */
 } kvq_config;
 
 typedef struct {

@@ -98,8 +98,9 @@ def test_identical_keys_give_mean_of_values():
 
 @pytest.mark.parametrize("name", ["tiny", "llama3_8b", "long_ctx", "llama70b_conc"])
 def test_decode_workloads_full_size(name):
-    """The benchmark workloads at their full sizes, compared element by element
-    with the oracle (every output)."""
+    """The benchmark workloads at their full sizes: every byte of every group
+    block and tail of the cache compared with the oracle's (bit-exact), then
+    the decode compared element by element with the oracle (every output)."""
     K = tl.kvq()
     w = inputs.WORKLOADS[name]()
     spec = K.CacheSpec(w.k_bits, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
@@ -117,6 +118,7 @@ def test_decode_workloads_full_size(name):
     assert cache.workspace_status() == 0
     hk = [x.astype(np.float16) for x in w.keys]
     hv = [x.astype(np.float16) for x in w.values]
+    tl.check_cache_against_oracle(cache, hk, hv)
     want = tl.oracle_decode(spec, hk, hv, w.q)
     err = tl.decode_error(out, want)
     assert err <= tl.DECODE_TOL, (name, err)
@@ -139,9 +141,19 @@ def test_split_count_does_not_change_results(monkeypatch):
             monkeypatch.setenv("KVQ_DECODE_MAX_CTAS", cap)
         outs.append(cache.decode(qd).float().cpu().numpy())
     want = tl.oracle_decode(spec, ks, vs, q)
+    # Split counts only reorder the work: every attention weight p is still
+    # rounded to fp16 once (relative error <= 2^-11), but relative to a
+    # running max that depends on the order, so two orders can round each
+    # p differently by up to 2^-10 relative; through o = sum p v / sum p
+    # that moves each output by at most about 2^-9 * max_t |v_t| of its
+    # sequence (the fp32 accumulation order adds far less).
+    from oracle import kvq_oracle as o
+    cfg = tl.oracle_cfg(spec)
+    vmax = np.array([np.abs(o.dequantized_cache(cfg, k, v)[1]).max() for k, v in zip(ks, vs)])
+    bound = 2.0 ** -9 * vmax[:, None, None]
     for o_ in outs:
         assert np.abs(o_ - want).max() <= tl.DECODE_TOL
-        assert np.abs(o_ - outs[-1]).max() <= 1e-3
+        assert (np.abs(o_ - outs[-1]) <= bound).all(), np.abs(o_ - outs[-1]).max()
     assert cache.workspace_status() == 0
 
 

@@ -145,16 +145,41 @@ def test_append_stream_workload_full_size():
     tl.check_cache_against_oracle(cache, hk, hv)
 
 
-def test_prefill_workload_full_size_sampled():
+def test_prefill_workload_full_size():
     """Prefill of 4 sequences x 32768 tokens x 8 kv heads x d=128 (fp16,
-    K4/V2, G=32) in one call; every 61st group and the lengths checked."""
+    K4/V2, G=32) in one call: every group of the first sequence (all 8 kv
+    heads, 8192 blocks), every 7th group of the others, and the lengths."""
     K = tl.kvq()
     w = inputs.quant_append()
     spec = K.CacheSpec(4, 2, 32, 128, 8, 8, 4, 32768)
     cache = K.KVQCache(spec)
     tl.append_chunks(cache, w.keys, w.values, "fp16")
-    tl.check_cache_against_oracle(cache, w.keys, w.values,
-                                  group_sample=lambda ng: np.arange(0, ng, 61))
+    tl.check_cache_against_oracle(cache, w.keys, w.values, seqs=[0])
+    tl.check_cache_against_oracle(cache, w.keys, w.values, seqs=[1, 2, 3],
+                                  group_sample=lambda ng: np.arange(0, ng, 7))
+
+
+def test_division_rule_case():
+    """The hand-worked golden case that pins IEEE division (quantizer
+    examples, '2-bit, IEEE division not reciprocal multiply'): a key channel
+    and a value group holding 0, 37.5 and 45 must get code 2 for 37.5 (the
+    quotient 37.5 / 15 = 2.5 ties to even); multiplying by fp32(1/15) would
+    give 3."""
+    K = tl.kvq()
+    G, d = 32, 64
+    spec = K.CacheSpec(2, 2, G, d, 1, 1, 1, 64)
+    k = np.zeros((G, 1, d), np.float16)
+    v = np.zeros((G, 1, d), np.float16)
+    k[3, 0, 5] = 37.5
+    k[7, 0, 5] = 45.0
+    v[4, 0, 1] = 37.5
+    v[4, 0, 2] = 45.0
+    cache = K.KVQCache(spec)
+    tl.append_chunks(cache, [k], [v], "fp16")
+    tl.check_cache_against_oracle(cache, [k], [v])
+    from oracle import kvq_oracle as o
+    kc, ks, _ = o.quantize_keys(k[:, 0, :], 2)
+    assert float(ks[5]) == 15.0 and int(kc[3, 5]) == 2 and int(kc[7, 5]) == 3
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
