@@ -64,6 +64,7 @@ function is "parity unpinned".
 """
 from __future__ import annotations
 
+import dataclasses
 import math
 from dataclasses import dataclass
 
@@ -88,6 +89,7 @@ class Config:
     window: int = 0      # R: recent tokens kept in fp16 beyond the partial group
     sink: int = 0        # S: first tokens of a sequence kept in fp16
     rotate: bool = False # cache holds Hadamard-rotated tokens
+    akvq_delta: int = 0  # position-adaptive key bits: region size Delta (0 = off)
 
     @property
     def tail_slots(self) -> int:   # W = R + G slots of the fp16 tail ring
@@ -629,6 +631,110 @@ def dequantized_cache(cfg: Config, k16: np.ndarray, v16: np.ndarray):
     kh[Sb:N] = dequantize_keys(kc, ks, kz).transpose(1, 2, 0, 3).reshape(Nq, hkv, d)
     vh[Sb:N] = dequantize_values(vc, vs, vz, cfg.group).transpose(1, 2, 0, 3).reshape(Nq, hkv, d)
     return kh, vh
+
+
+# ---------------------------------------------------------------------------
+# Position-adaptive key bits ("Asymmetric Key-Value Quantization: 2-Bit
+# Values and 4-Bit Keys under Long-Context Drift", §3.2)
+# ---------------------------------------------------------------------------
+# The page gives b(p) = b_high for the recent tokens (p > n - Delta), b_mid in
+# the middle and b_low for the early tokens (p <= Delta), default Delta =
+# 1024, but its rationale gives the middle tokens the lowest precision and
+# the early ones (attention sinks) a moderate one.  Reading taken, with the
+# two key widths of this cache: the high width cfg.k_bits (4) for the early
+# and the recent key groups, 2 bits in the middle; values keep cfg.v_bits.
+# A group's region follows from its position and the current length n, so
+# a group quantized while recent ages into the middle as the sequence grows;
+# it is then requantized to 2 bits from its dequantized keys (the fp16 keys
+# are gone by then).  Groups that are already in the middle when they are
+# quantized (a long prefill) go to 2 bits from their fp16 keys directly, so
+# the bytes depend on the append history, the widths do not.
+AKVQ_LOW_BITS = 2
+
+
+def akvq_key_bits(cfg: Config, g: int, n: int) -> int:
+    """Key bits of quantized group g (positions gG .. gG + G - 1, counted
+    from 0) in a sequence of n tokens: cfg.k_bits when all its positions
+    are early (< Delta) or its last position is recent (>= n - Delta), else
+    2."""
+    G, D = cfg.group, cfg.akvq_delta
+    if (g + 1) * G <= D or (g + 1) * G > n - D:
+        return cfg.k_bits
+    return AKVQ_LOW_BITS
+
+
+def akvq_requantize_keys(ks: np.ndarray, kz: np.ndarray, kc: np.ndarray):
+    """A high-width key group requantized to 2 bits from its dequantized keys:
+    x = fp16( fp32(s) * code + fp32(z) ) (the product is exact in fp32, the
+    sum rounded to nearest even, then rounded to fp16), then the quantizer
+    of ``quantize_keys``.  kc [..., G, d], ks/kz [..., d] fp16."""
+    s32 = np.asarray(ks, np.float16).astype(np.float32)[..., None, :]
+    z32 = np.asarray(kz, np.float16).astype(np.float32)[..., None, :]
+    x = (s32 * np.asarray(kc).astype(np.float32) + z32).astype(np.float16)
+    return quantize_keys(x, AKVQ_LOW_BITS)
+
+
+def akvq_cache_image(cfg: Config, k16: np.ndarray, v16: np.ndarray, chunks):
+    """Cache contents of a position-adaptive cache after appending the token
+    history [n, Hkv, d] (fp16, as stored) in chunks of the given sizes, one
+    append per chunk.  At each append from n0 to n1 tokens: the groups that
+    complete are quantized at their width for length n1 (keys from their
+    fp16 tokens), then every group quantized earlier whose width for n1 is
+    2 while it holds high-width codes is requantized (akvq_requantize_keys).
+    Returns ``bits`` [ng], ``groups`` (one (kc, ks, kz, vc, vs, vz) tuple per
+    group, leading [Hkv]), ``blocks`` [Hkv, ng, slot] uint8 with slot = the
+    high-width block size and a 2-bit group's block packed from the start of
+    its slot (the rest zero here, unspecified in the cache), and the tail as
+    ``cache_image`` gives it."""
+    G = cfg.group
+    n_all = k16.shape[0]
+    if sum(chunks) != n_all:
+        raise ValueError("chunks must add up to the history length")
+    if cfg.window or cfg.sink:
+        raise ValueError("position-adaptive bits are defined without window and sink")
+    groups, bits = [], []
+    n = 0
+    for nn in chunks:
+        n0, n1 = n, n + nn
+        for g in range(n0 // G, n1 // G):
+            kk = np.asarray(k16[g * G:(g + 1) * G], np.float16).transpose(1, 0, 2)
+            vv = np.asarray(v16[g * G:(g + 1) * G], np.float16).transpose(1, 0, 2)
+            b = akvq_key_bits(cfg, g, n1)
+            kc, ks, kz = quantize_keys(kk, b)
+            vc, vs, vz = quantize_values(vv, cfg.v_bits, G)
+            groups.append((kc, ks, kz, vc, vs, vz))
+            bits.append(b)
+        for g in range(n0 // G):
+            if bits[g] == cfg.k_bits and akvq_key_bits(cfg, g, n1) == AKVQ_LOW_BITS:
+                kc, ks, kz, vc, vs, vz = groups[g]
+                kc2, ks2, kz2 = akvq_requantize_keys(ks, kz, kc)
+                groups[g] = (kc2, ks2, kz2, vc, vs, vz)
+                bits[g] = AKVQ_LOW_BITS
+        n = n1
+    hkv = k16.shape[1]
+    slot = block_bytes(cfg)
+    blocks = np.zeros((hkv, len(groups), slot), np.uint8)
+    for g, (q, b) in enumerate(zip(groups, bits)):
+        cb = dataclasses.replace(cfg, k_bits=b)
+        blocks[:, g, :block_bytes(cb)] = pack_blocks(cb, *q)
+    N = G * (n_all // G)
+    return {"bits": bits, "groups": groups, "blocks": blocks, "N": N, "T": n_all - N,
+            "tail_k": np.ascontiguousarray(np.asarray(k16[N:], np.float16).transpose(1, 0, 2)),
+            "tail_v": np.ascontiguousarray(np.asarray(v16[N:], np.float16).transpose(1, 0, 2))}
+
+
+def akvq_decode(cfg: Config, k16: np.ndarray, v16: np.ndarray, q: np.ndarray, chunks) -> np.ndarray:
+    """Decode output [Hq, d] (float64) on the position-adaptive cache built by
+    appending k16, v16 (fp16) in the given chunks: every group dequantized at
+    its own key width, the tail as stored."""
+    img = akvq_cache_image(cfg, k16, v16, chunks)
+    kh = np.asarray(k16, np.float64).copy()
+    vh = np.asarray(v16, np.float64).copy()
+    G = cfg.group
+    for g, (kc, ks, kz, vc, vs, vz) in enumerate(img["groups"]):
+        kh[g * G:(g + 1) * G] = dequantize_keys(kc, ks, kz).transpose(1, 0, 2)
+        vh[g * G:(g + 1) * G] = dequantize_values(vc, vs, vz, G).transpose(1, 0, 2)
+    return attention(q, kh, vh, cfg.gqa)
 
 
 # ---------------------------------------------------------------------------
