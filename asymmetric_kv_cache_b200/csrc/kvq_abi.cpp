@@ -82,6 +82,13 @@ kvq_status validate_config(const kvq_config* c) {
     return fail(KVQ_ERR_CONFIG, "sink must be in [0, 1024] (got %d)", c->sink);
   if (c->rotate != 0 && c->rotate != 1)
     return fail(KVQ_ERR_CONFIG, "rotate must be 0 or 1 (got %d)", c->rotate);
+  if (c->akvq_delta != 0) {
+    if (c->akvq_delta < 0 || c->akvq_delta > (1 << 20) || c->akvq_delta % c->group != 0)
+      return fail(KVQ_ERR_CONFIG, "akvq_delta must be a multiple of group in [0, 2^20] (got %d)",
+                  c->akvq_delta);
+    if (c->k_bits != 4 || c->window != 0 || c->sink != 0)
+      return fail(KVQ_ERR_CONFIG, "akvq_delta needs k_bits = 4 and window = sink = 0");
+  }
   // decode addresses slots (groups + tail) of all units with 32-bit prefixes
   const int64_t slices = (c->n_q_heads / c->n_kv_heads + kvq::kHeadsPerSlice - 1) / kvq::kHeadsPerSlice;
   const int64_t slots = (int64_t)c->max_seqs * c->n_kv_heads * slices * (c->max_tokens / c->group + 1);
@@ -115,6 +122,12 @@ void fill_layout(const kvq::Geom& g, kvq_layout* o) {
   o->vcodes_offset = g.sec_vcodes;
   o->vscale_offset = g.sec_vscale;
   o->vmin_offset = g.sec_vmin;
+  o->akvq_block_bytes = g.a2_bytes;
+  o->akvq_kscale_offset = g.a2_kscale;
+  o->akvq_kmin_offset = g.a2_kmin;
+  o->akvq_vcodes_offset = g.a2_vcodes;
+  o->akvq_vscale_offset = g.a2_vscale;
+  o->akvq_vmin_offset = g.a2_vmin;
 }
 
 }  // namespace
@@ -251,6 +264,14 @@ kvq_status kvq_append(kvq_cache* cache, const void* k, const void* v, kvq_dtype 
       seqs.row_off[i] = (int32_t)row;
       seqs.n_new[i] = nn;
       tasks += nn > 0 ? std::max(F, 1) : 0;
+      if (g.akvq_delta && nn > 0) {
+        // requantization tasks of the groups that age into the middle: one
+        // reserved below G new tokens (the launch shape then does not depend
+        // on the lengths), else the exact count
+        int first;
+        tasks += nn < g.G ? 1
+                          : kvq::akvq_aging(len0, len0 + nn, len0 / g.G, g.G, g.akvq_delta, &first);
+      }
       row += nn;
     }
     seqs.task_prefix[n] = tasks;

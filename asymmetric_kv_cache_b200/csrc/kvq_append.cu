@@ -207,6 +207,111 @@ __device__ __forceinline__ void codes2(float x0, float x1, float z0, float z1, f
   near_tie |= (a0 >= 0x3EFFF800u) | (a1 >= 0x3EFFF800u);   // 0.5 - 2048 ulp
 }
 
+// Key statistics of a staged group (fp16 rows of DP halves, G tokens):
+// per channel min and max over the tokens (fp16x2, exact), the stored fp16
+// scale fp16((max - min) / QK) and min, their fp32 {z, 1/s, s} for the
+// codes, and the metadata in slot order i*(D/4) + 4kt + 2v + e.  Threads
+// 0..63.
+template <int D, int G, int QK>
+__device__ __forceinline__ void key_stats(const __half* __restrict__ sk, float4* __restrict__ kp,
+                                          __half* __restrict__ ks, __half* __restrict__ kz,
+                                          int tid) {
+  constexpr int DP = D + 8;
+  const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
+  for (int cp = tid; cp < D / 2; cp += 64) {
+    __half2 mn = sk2[cp], mx = mn;
+    for (int r = 1; r < G; ++r) {
+      const __half2 x = sk2[r * (DP / 2) + cp];
+      mn = __hmin2(mn, x);
+      mx = __hmax2(mx, x);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = 2 * cp + e;
+      const float mnf = e ? __high2float(mn) : __low2float(mn);
+      const float mxf = e ? __high2float(mx) : __low2float(mx);
+      const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)QK));
+      const __half z16 = __float2half_rn(mnf);
+      const float sf = __half2float(s16);
+      kp[c] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
+      // metadata slot i*(D/4) + 4kt + 2v + e
+      const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3, ee = c & 1;
+      const int slot = i * (D / 4) + 4 * kt + 2 * v + ee;
+      ks[slot] = s16;
+      kz[slot] = z16;
+    }
+  }
+}
+
+// Key codes of a staged group at KBq bits, packed word by word into the
+// fragment order of the key-code section kw (see kvq.h).  128 threads.
+template <int D, int G, int KBq>
+__device__ __forceinline__ void key_codes(const __half* __restrict__ sk, const float4* __restrict__ kp,
+                                          uint32_t* __restrict__ kw, int tid) {
+  constexpr int DP = D + 8;
+  constexpr int QK = (1 << KBq) - 1;
+  constexpr int FK = 16 / KBq;               // code pairs per 32-bit word
+  constexpr int KWPL = D * KBq / 128;        // key words per lane per 8-token tile
+  constexpr int KWORDS = G * D * KBq / 32;
+  const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
+  {
+    // Thread items wi = tid + 128k: lane = wi % 32 varies fastest (a warp
+    // reads 8 tokens x 4 channel pairs: 32 distinct banks of the padded
+    // rows), then the word w of the lane, then the token tile.  A thread's
+    // items share w and the lane, hence one set of channels: their (z, 1/s)
+    // are loaded once.
+    static_assert(4 % KWPL == 0, "key words of a thread share their channels");
+    const int lane = tid % 32;
+    const int w = (tid / 32) % KWPL;
+    const int i = lane & 3;
+    float zk[FK][2], rk[FK][2];
+#pragma unroll
+    for (int f = 0; f < FK; ++f) {
+      const int p = w * FK + f;
+      const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4 pc = kp[c + e];
+        zk[f][e] = pc.x;
+        rk[f][e] = pc.y;
+      }
+    }
+    for (int wi = tid; wi < KWORDS; wi += 128) {
+      const int nt = wi / (KWPL * 32);
+      const int t = 8 * nt + (lane >> 2);
+      const int widx = (nt * 32 + lane) * KWPL + w;   // layout word
+      uint32_t word = 0;
+      bool tie = false;
+#pragma unroll
+      for (int f = 0; f < FK; ++f) {
+        // field f of the low half and of the high half: channels c, c + 1
+        const int p = w * FK + f;
+        const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+        const float2 x = __half22float2(sk2[(t * DP + c) >> 1]);
+        uint32_t c0, c1;
+        codes2(x.x, x.y, zk[f][0], zk[f][1], rk[f][0], rk[f][1], QK, c0, c1, tie);
+        word |= ((c0 & QK) << (KBq * f)) | ((c1 & QK) << (KBq * (FK + f)));
+      }
+      if (tie) {   // rare: IEEE division for the whole word
+        word = 0;
+#pragma unroll
+        for (int f = 0; f < FK; ++f) {
+          const int p = w * FK + f;
+          const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 pc = kp[c + e];
+            const uint32_t code =
+                (uint32_t)quant_code(__half2float(sk[t * DP + c + e]), pc.x, pc.z, QK);
+            word |= code << (KBq * (e * FK + f));
+          }
+        }
+      }
+      kw[widx] = word;
+    }
+  }
+}
+
 template <int D, int G, int KB, int VB>
 __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char* __restrict__ cache,
                                                      const void* __restrict__ kin,
@@ -291,6 +396,63 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
       if (act) store_tail8(sinkk, sinkv, len0 + j, cc, D, k8, v8);
     }
   };
+  // Position-adaptive key bits: the tasks after the append's own (max(F, 1))
+  // requantize the 4-bit key groups that this append moves from the recent
+  // region into the middle ("Asymmetric Key-Value Quantization: 2-Bit
+  // Values and 4-Bit Keys under Long-Context Drift", §3.2, with the aging
+  // rule of this library): keys dequantized to fp16(fp32(s) * code +
+  // fp32(z)), quantized again at 2 bits; the value sections move unchanged
+  // to their places in the 2-bit block.  The host reserves one such task
+  // per sequence for appends of fewer than G tokens (at most one group ages
+  // then); a task with no group to age does nothing.
+  if constexpr (KB == 4) {
+    if (g.akvq_delta && tau >= (F > 0 ? F : 1)) {
+      int first;
+      const int A = akvq_aging(len0, n1, N0 / G, G, g.akvq_delta, &first);
+      const int r = tau - (F > 0 ? F : 1);
+      if (r < A) {
+        unsigned char* blk = cache + g.blocks_off +
+                             (unit * g.max_groups + first + r) * (int64_t)g.block_bytes;
+        const unsigned char* kc4 = blk + g.sec_kcodes;
+        const __half* ks4 = reinterpret_cast<const __half*>(blk + g.sec_kscale);
+        const __half* kz4 = reinterpret_cast<const __half*>(blk + g.sec_kmin);
+        constexpr int LB = D * 4 / 32;   // key-code bytes per lane per 8-token tile
+        for (int idx = tid; idx < G * D; idx += 128) {
+          // code (t, c) of the 4-bit key section (layout in kvq.h)
+          const int t = idx / D, c = idx % D;
+          const int nt = t >> 3, rr = t & 7, kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3,
+                    e = c & 1;
+          const int p = 2 * kt + v;
+          const uint32_t word = *reinterpret_cast<const uint32_t*>(
+              kc4 + nt * 32 * LB + (4 * rr + i) * LB + 4 * (p / 4));
+          const uint32_t code = (word >> (4 * (p % 4 + 4 * e))) & 15u;
+          const int slot = i * (D / 4) + 4 * kt + 2 * v + e;
+          const float x = __fadd_rn(__fmul_rn(__half2float(ks4[slot]), (float)code),
+                                    __half2float(kz4[slot]));
+          sk[t * C::DP + c] = __float2half_rn(x);
+        }
+        // the value sections, kept in the (unused) value staging area
+        unsigned char* vkeep = reinterpret_cast<unsigned char*>(sv);
+        constexpr int VBYTES = G * D * VB / 8 + 4 * G * C::J;   // codes, scales, mins
+        static_assert(VBYTES % 16 == 0 && VBYTES <= 2 * G * (D + 8), "value sections fit the area");
+        for (int i = tid * 16; i < VBYTES; i += 128 * 16)
+          *reinterpret_cast<uint4*>(vkeep + i) = *reinterpret_cast<const uint4*>(blk + g.sec_vcodes + i);
+        __syncthreads();   // every read of the old block is done
+        float4* kp = reinterpret_cast<float4*>(sm + C::SM_KP);
+        if (tid < 64) key_stats<D, G, 3>(sk, kp, ks, kz, tid);
+        __syncthreads();
+        key_codes<D, G, 2>(sk, kp, reinterpret_cast<uint32_t*>(blk), tid);
+        for (int i = tid; i < D / 2; i += 128) {
+          reinterpret_cast<uint32_t*>(blk + g.a2_kscale)[i] = reinterpret_cast<const uint32_t*>(ks)[i];
+          reinterpret_cast<uint32_t*>(blk + g.a2_kmin)[i] = reinterpret_cast<const uint32_t*>(kz)[i];
+        }
+        for (int i = tid * 16; i < VBYTES; i += 128 * 16)
+          *reinterpret_cast<uint4*>(blk + g.a2_vcodes + i) = *reinterpret_cast<const uint4*>(vkeep + i);
+      }
+      finish();
+      return;
+    }
+  }
   if (F == 0) {
     // no group completes: post-sink position a0 + j (input row nsink + j) goes
     // to ring slot (a0 + j) mod W, which holds no tail token (the tail
@@ -347,36 +509,18 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   }
   __syncthreads();
 
+  // key width of this group: the cache's, or with position-adaptive bits
+  // the width of its region once this append is done
+  const int kbits = (KB == 4 && g.akvq_delta) ? akvq_key_bits(N0 / G + tau, n1, G, g.akvq_delta) : KB;
+
   // ---- statistics.  Warps 0-1: keys, two channels per thread (fp16x2
   // min/max over the G tokens).  Warps 2-3: values, (token, group of G
   // channels) items, 16-byte loads.  fp16 min/max of fp16 values is exact.
   float4* kp = reinterpret_cast<float4*>(sm + C::SM_KP);   // [c]: {z, 1/s, s, -}
   float4* vp = reinterpret_cast<float4*>(sm + C::SM_VP);   // [r * J + j]
   if (tid < 64) {
-    const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
-    for (int cp = tid; cp < D / 2; cp += 64) {
-      __half2 mn = sk2[cp], mx = mn;
-      for (int r = 1; r < G; ++r) {
-        const __half2 x = sk2[r * (C::DP / 2) + cp];
-        mn = __hmin2(mn, x);
-        mx = __hmax2(mx, x);
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int c = 2 * cp + e;
-        const float mnf = e ? __high2float(mn) : __low2float(mn);
-        const float mxf = e ? __high2float(mx) : __low2float(mx);
-        const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)C::QK));
-        const __half z16 = __float2half_rn(mnf);
-        const float sf = __half2float(s16);
-        kp[c] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
-        // metadata slot i*(D/4) + 4kt + 2v + e
-        const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3, ee = c & 1;
-        const int slot = i * (D / 4) + 4 * kt + 2 * v + ee;
-        ks[slot] = s16;
-        kz[slot] = z16;
-      }
-    }
+    if (kbits == KB) key_stats<D, G, (1 << KB) - 1>(sk, kp, ks, kz, tid);
+    else key_stats<D, G, 3>(sk, kp, ks, kz, tid);
   } else {
     for (int q = tid - 64; q < G * C::J; q += 64) {
       const int r = q / C::J, j = q % C::J;
@@ -413,65 +557,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   // ---- codes, quantized and packed word by word into the group block
   unsigned char* blk = cache + g.blocks_off +
                        (unit * g.max_groups + (N0 / G + tau)) * (int64_t)g.block_bytes;
-  uint32_t* kw = reinterpret_cast<uint32_t*>(blk + g.sec_kcodes);
-  const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
-  {
-    // Thread items wi = tid + 128k: lane = wi % 32 varies fastest (a warp
-    // reads 8 tokens x 4 channel pairs: 32 distinct banks of the padded
-    // rows), then the word w of the lane, then the token tile.  A thread's
-    // items share w and the lane, hence one set of channels: their (z, 1/s)
-    // are loaded once.
-    static_assert(4 % C::KWORDS_PER_LANE == 0, "key words of a thread share their channels");
-    const int lane = tid % 32;
-    const int w = (tid / 32) % C::KWORDS_PER_LANE;
-    const int i = lane & 3;
-    float zk[C::FK][2], rk[C::FK][2];
-#pragma unroll
-    for (int f = 0; f < C::FK; ++f) {
-      const int p = w * C::FK + f;
-      const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float4 pc = kp[c + e];
-        zk[f][e] = pc.x;
-        rk[f][e] = pc.y;
-      }
-    }
-    for (int wi = tid; wi < C::KWORDS; wi += blockDim.x) {
-      const int nt = wi / (C::KWORDS_PER_LANE * 32);
-      const int t = 8 * nt + (lane >> 2);
-      const int widx = (nt * 32 + lane) * C::KWORDS_PER_LANE + w;   // layout word
-      uint32_t word = 0;
-      bool tie = false;
-#pragma unroll
-      for (int f = 0; f < C::FK; ++f) {
-        // field f of the low half and of the high half: channels c, c + 1
-        const int p = w * C::FK + f;
-        const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
-        const float2 x = __half22float2(sk2[(t * C::DP + c) >> 1]);
-        uint32_t c0, c1;
-        codes2(x.x, x.y, zk[f][0], zk[f][1], rk[f][0], rk[f][1], C::QK, c0, c1, tie);
-        word |= ((c0 & C::QK) << (KB * f)) | ((c1 & C::QK) << (KB * (C::FK + f)));
-      }
-      if (tie) {   // rare: IEEE division for the whole word
-        word = 0;
-#pragma unroll
-        for (int f = 0; f < C::FK; ++f) {
-          const int p = w * C::FK + f;
-          const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float4 pc = kp[c + e];
-            const uint32_t code =
-                (uint32_t)quant_code(__half2float(sk[t * C::DP + c + e]), pc.x, pc.z, C::QK);
-            word |= code << (KB * (e * C::FK + f));
-          }
-        }
-      }
-      kw[widx] = word;
-    }
-  }
-  uint32_t* vw = reinterpret_cast<uint32_t*>(blk + g.sec_vcodes);
+  if (kbits == KB) key_codes<D, G, KB>(sk, kp, reinterpret_cast<uint32_t*>(blk + g.sec_kcodes), tid);
+  else key_codes<D, G, 2>(sk, kp, reinterpret_cast<uint32_t*>(blk), tid);
+  uint32_t* vw = reinterpret_cast<uint32_t*>(blk + (kbits == KB ? g.sec_vcodes : g.a2_vcodes));
   for (int wi = tid; wi < C::VWORDS; wi += blockDim.x) {
     // lane fastest (a warp reads 4 token pairs x 8 channels: distinct banks
     // of the padded rows), then the lane's word w, then the token tile
@@ -528,17 +616,18 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   {
     const uint32_t* src;
     uint32_t* dst;
+    const bool full = kbits == KB;   // else a 2-bit key group (position-adaptive bits)
     src = reinterpret_cast<const uint32_t*>(ks);
-    dst = reinterpret_cast<uint32_t*>(blk + g.sec_kscale);
+    dst = reinterpret_cast<uint32_t*>(blk + (full ? g.sec_kscale : g.a2_kscale));
     for (int i = tid; i < D / 2; i += blockDim.x) dst[i] = src[i];
     src = reinterpret_cast<const uint32_t*>(kz);
-    dst = reinterpret_cast<uint32_t*>(blk + g.sec_kmin);
+    dst = reinterpret_cast<uint32_t*>(blk + (full ? g.sec_kmin : g.a2_kmin));
     for (int i = tid; i < D / 2; i += blockDim.x) dst[i] = src[i];
     src = reinterpret_cast<const uint32_t*>(vs);
-    dst = reinterpret_cast<uint32_t*>(blk + g.sec_vscale);
+    dst = reinterpret_cast<uint32_t*>(blk + (full ? g.sec_vscale : g.a2_vscale));
     for (int i = tid; i < G * C::J / 2; i += blockDim.x) dst[i] = src[i];
     src = reinterpret_cast<const uint32_t*>(vz);
-    dst = reinterpret_cast<uint32_t*>(blk + g.sec_vmin);
+    dst = reinterpret_cast<uint32_t*>(blk + (full ? g.sec_vmin : g.a2_vmin));
     for (int i = tid; i < G * C::J / 2; i += blockDim.x) dst[i] = src[i];
   }
 

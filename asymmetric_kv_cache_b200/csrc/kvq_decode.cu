@@ -460,7 +460,7 @@ cudaError_t decode_max_ctas(const Geom& g, bool wide, int* max_ctas) {
 // dominate), so the mma.sync kernel is the default.
 bool decode_tc_eligible(const Geom& g) {
   if (!(g.d == 128 && g.G == 32 && g.vb == 2 && (g.kb == 2 || g.kb == 4) && g.gqa <= 4 &&
-        g.slices == 1 && g.window == 0 && g.sink == 0 && g.rotate == 0))
+        g.slices == 1 && g.window == 0 && g.sink == 0 && g.rotate == 0 && g.akvq_delta == 0))
     return false;
   const char* env = std::getenv("KVQ_DECODE_TC");
   return env && env[0] == '1';

@@ -217,11 +217,12 @@ __device__ __forceinline__ void softmax_update(WarpState<D, KB, VB, G>& st, floa
 
 // The value side of a group (O^T += V^T (p s_v), Z += [z_v; 1]^T p), shared
 // by both layouts: pt[kv] = B fragments of 16 tokens.
-template <int D, int KB, int VB, int G, bool PK>
+// KBL: key width of the block's layout (the value sections follow its keys).
+template <int D, int KB, int VB, int G, bool PK, int KBL = KB>
 __device__ __forceinline__ void value_side(WarpState<D, KB, VB, G, PK>& st,
                                            const unsigned char* __restrict__ sp,
                                            const uint32_t (&pt)[G / 16][2], int lane) {
-  using C = DecCfg<D, KB, VB, G>;
+  using C = DecCfg<D, KBL, VB, G>;
   const int g8 = lane >> 2, i4 = lane & 3;
   const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
   const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
@@ -269,11 +270,12 @@ __device__ __forceinline__ void value_side(WarpState<D, KB, VB, G, PK>& st,
 // one tile per k-step against a constant -1024 operand, which sums exactly
 // the fp16 A values the tensor core saw, and accumulates with the key-min
 // bias.  Value codes are unpacked to exact fp16 integers (unpack_pair).
-template <int D, int KB, int VB, int G>
+// KBL: key width of the block (the state's KB unless the cache mixes widths).
+template <int D, int KB, int VB, int G, int KBL = KB>
 __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
                                               const unsigned char* __restrict__ sp,
                                               const uint4* __restrict__ qsm, int lane) {
-  using C = DecCfg<D, KB, VB, G>;
+  using C = DecCfg<D, KBL, VB, G>;
   constexpr int NT = G / 8;
   // key-code words held at once per token tile: all of them when that is at
   // most 8 registers, two at a time otherwise
@@ -306,7 +308,7 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
       const uint4 q4 = qsm[kt * 32 + lane];
       // s_k / m of the code pair's field (a power-of-two scaling: exact
       // while s_k / m stays a normal fp16 number)
-      constexpr int e0 = code_log2_mul<KB, p0 % C::FK>(), e1 = code_log2_mul<KB, p1 % C::FK>();
+      constexpr int e0 = code_log2_mul<KBL, p0 % C::FK>(), e1 = code_log2_mul<KBL, p1 % C::FK>();
       const uint32_t sm0 = e0 ? hmul2_b(s2.x, h2_pow2_neg(e0)) : s2.x;
       const uint32_t sm1 = e1 ? hmul2_b(s2.y, h2_pow2_neg(e1)) : s2.y;
       // high part: one rounding of hi*s + lo*s; residual: (hi*s - high) in
@@ -320,8 +322,8 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
       static_for<NT>([&](auto nt_) {
         constexpr int nt = decltype(nt_)::value;
         constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
-        mma16816(acc[nt], a0, a1, a2, a3, code_offset<KB, p0 % C::FK>(kw[nt][w0]),
-                 code_offset<KB, p1 % C::FK>(kw[nt][w1]));
+        mma16816(acc[nt], a0, a1, a2, a3, code_offset<KBL, p0 % C::FK>(kw[nt][w0]),
+                 code_offset<KBL, p1 % C::FK>(kw[nt][w1]));
       });
     });
   });
@@ -337,7 +339,7 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   uint32_t pt[G / 16][2];   // B fragments of the value product, 16 tokens each
   softmax_update<D, NT, KB, VB, G>(st, s, *reinterpret_cast<uint32_t(*)[NT]>(&pt[0][0]),
                                    lane & 3);
-  value_side<D, KB, VB, G, false>(st, sp, pt, lane);
+  value_side<D, KB, VB, G, false, KBL>(st, sp, pt, lane);
 }
 
 // Decode slots of a unit with L tokens: its quantized groups plus one for a
@@ -782,16 +784,16 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
   }
 }
 
-template <int D, int KB, int VB, int G>
+template <int D, int KB, int VB, int G, int KBL = KB>
 __device__ __forceinline__ void process_group_pk(WarpState<D, KB, VB, G, true>& st,
                                                  const unsigned char* __restrict__ sp,
                                                  const uint4* __restrict__ qsm, int lane) {
   constexpr int NM = G / 16;
   float s[NM][4];
-  kside_pk<D, KB, VB, G>(sp, qsm, lane, s);
+  kside_pk<D, KBL, VB, G>(sp, qsm, lane, s);
   uint32_t pt[NM][2];
   softmax_pk<D, NM, KB, VB, G>(st, s, pt);
-  value_side<D, KB, VB, G, true>(st, sp, pt, lane);
+  value_side<D, KB, VB, G, true, KBL>(st, sp, pt, lane);
 }
 
 template <int D, int KB, int VB, int G>
@@ -1426,7 +1428,9 @@ __device__ __noinline__ void finish_split_unit(const Geom& g, const WsLayout& w,
 // tokens in a ring of R + G slots) and/or a sink window (the first S tokens
 // in an fp16 area, folded in with the tail); the kernels without it keep
 // the single-chunk-per-warp tail and its register budget.
-template <int D, int KB, int VB, int G, bool PK, bool WIDE, bool WIN>
+// AK: position-adaptive key widths (KB = 4): a group whose width is 2 holds
+// the 2-bit block at the start of its slot; only those bytes are copied.
+template <int D, int KB, int VB, int G, bool PK, bool WIDE, bool WIN, bool AK = false>
 __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
                                   DecCfg<D, KB, VB, G, WIDE>::MIN_BLOCKS)
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
@@ -1570,6 +1574,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
 #endif
 
     int ngr, nh;         // groups in this piece, heads of the unit
+    int gs0, glen;       // the piece's first group in its sequence, the length
     int64_t gb;          // global block index of the piece's first group
     bool my_tail;        // this warp owns tail chunks warp, warp + TAIL_CHUNKS, ...
     {
@@ -1578,6 +1583,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       gb = ((int64_t)(a.seq0 + p.b) * g.hkv + p.kvh) * g.max_groups + p.slot0;
       ngr = max(0, min(p.slot1, p.ng) - p.slot0);
       nh = p.nh;
+      gs0 = p.slot0;
+      glen = p.L;
       if constexpr (WIN)
         my_tail = ok && p.slot1 == p.wb && p.slot0 <= p.ng && warp < C::TAIL_CHUNKS &&
                   warp < fp16_chunks(g, p.L, p.Tb);
@@ -1609,6 +1616,10 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         }
       }
     }
+    // group c of the piece holds 2-bit keys (position-adaptive widths)
+    auto narrow = [&](int c) -> bool {
+      return AK && akvq_key_bits(gs0 + c, glen, G, g.akvq_delta) != KB;
+    };
     // Claim a group (lane 0) and start its copy into stage `stg`; -1 once
     // the piece has none left.
     auto claim_into = [&](int stg) -> int {
@@ -1617,7 +1628,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         const int c = atomicAdd(&claim, 1);
         if (c < ngr) {
           gi = c;
-          checked_bulk_copy(wring + stg * C::BLK, blocks + (gb + c) * C::BLK, C::BLK, &wbars[stg],
+          checked_bulk_copy(wring + stg * C::BLK, blocks + (gb + c) * C::BLK,
+                            narrow(c) ? (uint32_t)g.a2_bytes : (uint32_t)C::BLK, &wbars[stg],
                             blocks, a.cache + g.tails_off, err, 2);
         }
       }
@@ -1708,9 +1720,21 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         break;
       }
       phase ^= 1u << head;
-      if constexpr (PK2) process_group_pk2<D, KB, VB, G>(st, wring + head * C::BLK, qp, lane);
-      else if constexpr (PK) process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
-      else process_group<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+      if constexpr (PK2) {
+        process_group_pk2<D, KB, VB, G>(st, wring + head * C::BLK, qp, lane);
+      } else if constexpr (AK) {
+        if (narrow(cur)) {
+          if constexpr (PK) process_group_pk<D, KB, VB, G, 2>(st, wring + head * C::BLK, qsm, lane);
+          else process_group<D, KB, VB, G, 2>(st, wring + head * C::BLK, qsm, lane);
+        } else {
+          if constexpr (PK) process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+          else process_group<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+        }
+      } else if constexpr (PK) {
+        process_group_pk<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+      } else {
+        process_group<D, KB, VB, G>(st, wring + head * C::BLK, qsm, lane);
+      }
       __syncwarp();
       // refill the stage: the warp's reads of it are complete (their values
       // were consumed before __syncwarp), and a bulk copy that overwrites
@@ -1719,7 +1743,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       int nn = -1;
       if (lane == 0 && nc >= 0 && nc < ngr) {
         nn = nc;
-        checked_bulk_copy(wring + head * C::BLK, blocks + (gb + nc) * C::BLK, C::BLK, &wbars[head],
+        checked_bulk_copy(wring + head * C::BLK, blocks + (gb + nc) * C::BLK,
+                          narrow(nc) ? (uint32_t)g.a2_bytes : (uint32_t)C::BLK, &wbars[head],
                           blocks, a.cache + g.tails_off, err, 3);
       }
       nn = __shfl_sync(0xffffffffu, nn, 0);
@@ -2010,15 +2035,35 @@ size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
   return DecCfg<D, KB, VB, G, WIDE>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
 }
 
+// The position-adaptive variant exists for 4-bit keys (not in the second
+// packed form).
+template <int KB, bool PK>
+constexpr bool has_ak() {
+  return KB == 4 && !(PK && KVQ_PK_FORM == 2);
+}
+
 template <int D, int KB, int VB, int G, bool PK, bool WIDE>
-cudaError_t max_ctas_t(int* out) {
+cudaError_t max_ctas_t(bool ak, int* out) {
   using C = DecCfg<D, KB, VB, G, WIDE>;
   const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(64);
   // residency of the kernels with and without a recent window (the same
-  // launch bounds and shared memory: normally equal), the smaller one
+  // launch bounds and shared memory: normally equal), the smaller one; of
+  // the position-adaptive one alone when the cache uses it
+  using K = decltype(&decode_kernel<D, KB, VB, G, PK, WIDE, false>);
+  K kerns[2] = {decode_kernel<D, KB, VB, G, PK, WIDE, false>,
+                decode_kernel<D, KB, VB, G, PK, WIDE, true>};
+  int nk = 2;
+  if (ak) {
+    if constexpr (has_ak<KB, PK>()) {
+      kerns[0] = decode_kernel<D, KB, VB, G, PK, WIDE, false, true>;
+      nk = 1;
+    } else {
+      return cudaErrorInvalidValue;
+    }
+  }
   int per_sm = 1 << 30;
-  for (auto kern : {decode_kernel<D, KB, VB, G, PK, WIDE, false>,
-                    decode_kernel<D, KB, VB, G, PK, WIDE, true>}) {
+  for (int ki = 0; ki < nk; ++ki) {
+    const K kern = kerns[ki];
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
     if (e != cudaSuccess) return e;
@@ -2044,15 +2089,25 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
   if (g.block_bytes != C::BLK || g.sec_vmin != C::SEC_VMIN || g.sec_kscale != C::SEC_KSCALE)
     return cudaErrorInvalidValue;
   const bool win = g.window > 0 || g.sink > 0;
+  const bool ak = g.akvq_delta > 0;
   auto kern = win ? decode_kernel<D, KB, VB, G, PK, WIDE, true>
                   : decode_kernel<D, KB, VB, G, PK, WIDE, false>;
+  if (ak) {
+    if constexpr (has_ak<KB, PK>()) {
+      if (win) return cudaErrorInvalidValue;
+      kern = decode_kernel<D, KB, VB, G, PK, WIDE, false, true>;
+    } else {
+      return cudaErrorInvalidValue;
+    }
+  }
+  const int variant = ak ? 2 : (int)win;
   const size_t sm = smem_bytes<D, KB, VB, G, WIDE>(a.n_seq);
-  static bool configured[2] = {false, false};   // attribute set once, before any capture
-  if (!configured[win]) {
+  static bool configured[3] = {false, false, false};   // attribute set once, before any capture
+  if (!configured[variant]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<D, KB, VB, G, WIDE>(kSeqsPerLaunch));
     if (e != cudaSuccess) return e;
-    configured[win] = true;
+    configured[variant] = true;
   }
   {
     // a programmatic dependent of the previous kernel (it waits for it
@@ -2100,10 +2155,11 @@ cudaError_t launch_t(const Geom& g, const WsLayout& w, const DecodeArgs& a, int 
 #define KVQ_DECODE_DEFINE(D_, KB_, VB_, G_)                                               \
   cudaError_t decode_max_ctas_##D_##_##KB_##_##VB_##_##G_(const Geom& g, bool wide,       \
                                                           int* out) {                     \
-    return g.gqa <= 4 ? (wide ? max_ctas_t<D_, KB_, VB_, G_, true, true>(out)             \
-                              : max_ctas_t<D_, KB_, VB_, G_, true, false>(out))           \
-                      : (wide ? max_ctas_t<D_, KB_, VB_, G_, false, true>(out)            \
-                              : max_ctas_t<D_, KB_, VB_, G_, false, false>(out));         \
+    const bool ak = g.akvq_delta > 0;                                                     \
+    return g.gqa <= 4 ? (wide ? max_ctas_t<D_, KB_, VB_, G_, true, true>(ak, out)         \
+                              : max_ctas_t<D_, KB_, VB_, G_, true, false>(ak, out))       \
+                      : (wide ? max_ctas_t<D_, KB_, VB_, G_, false, true>(ak, out)        \
+                              : max_ctas_t<D_, KB_, VB_, G_, false, false>(ak, out));     \
   }                                                                                       \
   cudaError_t launch_decode_##D_##_##KB_##_##VB_##_##G_(                                  \
       const Geom& g, const WsLayout& w, const DecodeArgs& a, int grid, bool wide,         \

@@ -37,6 +37,10 @@ struct Geom {
   int32_t sink, sink_slots;     // S, and SW = S rounded up to 16 sink slots
   int64_t sinks_off, sink_bytes;
   int32_t rotate;               // tokens, q and the output rotated by H / sqrt(d)
+  // position-adaptive key bits: Delta (0 = off) and the 2-bit group block
+  // inside a slot of block_bytes (codes at 0)
+  int32_t akvq_delta;
+  int32_t a2_bytes, a2_kscale, a2_kmin, a2_vcodes, a2_vscale, a2_vmin;
 };
 
 // Workspace of kvq_decode: [error word | per-unit split records | per-unit
@@ -74,6 +78,32 @@ __host__ __device__ inline int unit_slots_s(int L, int G, int window, int sink) 
   return ng + (L > ng * G ? 1 : 0);
 }
 
+// Position-adaptive key bits ("Asymmetric Key-Value Quantization: 2-Bit
+// Values and 4-Bit Keys under Long-Context Drift", §3.2, read as 4-bit keys
+// for the early and the recent key groups and 2-bit keys in between): the
+// key width of quantized group g (positions gG .. gG + G - 1) when the
+// sequence holds n tokens.
+__host__ __device__ inline int akvq_key_bits(int g, int n, int G, int delta) {
+  return ((g + 1) * G <= delta || (g + 1) * G > n - delta) ? 4 : 2;
+}
+// The first group that is recent at length n (every group from it on has
+// its last position >= n - delta).
+__host__ __device__ inline int akvq_recent_start(int n, int G, int delta) {
+  return n >= delta ? (n - delta) / G : 0;
+}
+// Groups that an append from n0 to n1 tokens moves from the recent region
+// into the middle and that were quantized before it (N0 = groups quantized
+// at n0): they are requantized to 2 bits.  [first, first + count).
+__host__ __device__ inline int akvq_aging(int n0, int n1, int N0g, int G, int delta,
+                                          int* first) {
+  const int lo0 = delta / G, lo1 = akvq_recent_start(n0, G, delta);
+  const int lo = lo0 > lo1 ? lo0 : lo1;
+  const int hi1 = akvq_recent_start(n1, G, delta);
+  const int hi = hi1 < N0g ? hi1 : N0g;
+  *first = lo;
+  return hi > lo ? hi - lo : 0;
+}
+
 // Fill g from a validated configuration (no checks here).
 inline void make_geom(const kvq_config& c, Geom* g) {
   g->kb = c.k_bits;
@@ -93,7 +123,17 @@ inline void make_geom(const kvq_config& c, Geom* g) {
   g->sink = c.sink;
   g->sink_slots = (c.sink + 15) / 16 * 16;
   g->rotate = c.rotate;
+  g->akvq_delta = c.akvq_delta;
   const int G = g->G, d = g->d, J = g->J;
+  {
+    int o2 = G * d * 2 / 8;   // 2-bit key codes
+    g->a2_kscale = o2; o2 += 2 * d;
+    g->a2_kmin = o2;   o2 += 2 * d;
+    g->a2_vcodes = o2; o2 += G * d * c.v_bits / 8;
+    g->a2_vscale = o2; o2 += 2 * G * J;
+    g->a2_vmin = o2;   o2 += 2 * G * J;
+    g->a2_bytes = o2;
+  }
   int off = 0;
   g->sec_kcodes = off; off += G * d * g->kb / 8;
   g->sec_kscale = off; off += 2 * d;

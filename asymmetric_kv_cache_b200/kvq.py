@@ -38,7 +38,7 @@ LAYOUT_VERSION = 2
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "k_bits", "v_bits", "group", "head_dim", "n_q_heads", "n_kv_heads",
-        "max_seqs", "max_tokens", "layout_version", "window", "sink", "rotate")]
+        "max_seqs", "max_tokens", "layout_version", "window", "sink", "rotate", "akvq_delta")]
 
 
 class KvqLayout(ctypes.Structure):
@@ -46,7 +46,8 @@ class KvqLayout(ctypes.Structure):
         "total_bytes", "lens_offset", "counters_offset", "blocks_offset", "block_bytes", "max_groups",
         "tails_offset", "tail_bytes", "kcodes_offset", "kscale_offset", "kmin_offset",
         "vcodes_offset", "vscale_offset", "vmin_offset", "tail_slots", "sinks_offset",
-        "sink_bytes", "sink_slots")]
+        "sink_bytes", "sink_slots", "akvq_block_bytes", "akvq_kscale_offset", "akvq_kmin_offset",
+        "akvq_vcodes_offset", "akvq_vscale_offset", "akvq_vmin_offset")]
 
 
 _c_status = ctypes.c_int32
@@ -108,9 +109,9 @@ def check(status: int, where: str) -> None:
 
 
 def make_config(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                max_tokens, window=0, sink=0, rotate=0) -> KvqConfig:
+                max_tokens, window=0, sink=0, rotate=0, akvq_delta=0) -> KvqConfig:
     return KvqConfig(k_bits, v_bits, group, head_dim, n_q_heads, n_kv_heads, max_seqs,
-                     max_tokens, LAYOUT_VERSION, window, sink, int(rotate))
+                     max_tokens, LAYOUT_VERSION, window, sink, int(rotate), int(akvq_delta))
 
 
 def required_bytes(cfg: KvqConfig) -> tuple[int, int]:
@@ -153,6 +154,7 @@ class CacheSpec:
     window: int = 0     # R: recent tokens kept in fp16 beyond the partial group
     sink: int = 0       # S: first tokens of each sequence kept in fp16
     rotate: int = 0     # 1: tokens, q and the output rotated by H / sqrt(d)
+    akvq_delta: int = 0  # Delta > 0: position-adaptive key bits (4 early/recent, 2 middle)
 
 
 class KVQCache:
@@ -166,7 +168,7 @@ class KVQCache:
         self.spec = spec
         self.cfg = make_config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim,
                                spec.n_q_heads, spec.n_kv_heads, spec.max_seqs, spec.max_tokens,
-                               spec.window, spec.sink, spec.rotate)
+                               spec.window, spec.sink, spec.rotate, spec.akvq_delta)
         cache_bytes, ws_bytes = required_bytes(self.cfg)
         self.buffer = torch.empty(cache_bytes, dtype=torch.uint8, device=device)
         self.workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)

@@ -335,6 +335,8 @@ def run_ours(args, rank, world, device):
               if args.long_context and args.window else None)
     sinkw = (run_long_context(stream, device, window=args.window, sink=args.sink, fp16=False)
              if args.long_context and args.sink else None)
+    akvq = (run_long_context(stream, device, akvq_delta=args.akvq_delta, fp16=False)
+            if args.long_context and args.akvq_delta else None)
     qa = run_quant_append(stream, device) if args.other_legs else None
     c70 = run_concurrent_70b(stream, device) if args.other_legs else None
 
@@ -361,7 +363,7 @@ def run_ours(args, rank, world, device):
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
         "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K, "long_ctx": long_ctx,
-        "window": window, "sink": sinkw, "quant_append": qa, "conc70b": c70,
+        "window": window, "sink": sinkw, "akvq": akvq, "quant_append": qa, "conc70b": c70,
     }
 
 
@@ -403,7 +405,7 @@ def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
             "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
 
 
-def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0):
+def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akvq_delta=0):
     """Decode alone on the 128k-token long-context workload (batch 1, 32 q /
     8 kv heads, d 128, K2/V2, G 32): the configuration the HBM-roofline
     target is stated on.  Copies of the cache (> 3x L2 in total) are
@@ -412,18 +414,30 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0):
     the same shape (fp16 K/V, two copies) when `fp16`.  `window` > 0 keeps
     that many recent tokens in fp16 beyond the partial group, `sink` > 0 the
     first tokens of the sequence (their bytes counted at 4d per
-    token-head)."""
+    token-head).  `akvq_delta` > 0: position-adaptive key widths on the same
+    context (4-bit keys for the first and the last Delta tokens' groups,
+    2-bit keys in between, 2-bit values), each group's bytes counted at its
+    own width."""
     import torch
     from asymmetric_kv_cache_b200 import inputs, kvq
     w = inputs.WORKLOADS["long_ctx"]()
     n = w.lens[0]
-    spec = kvq.CacheSpec(w.k_bits, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
-                         w.batch, n, window=window, sink=sink)
+    kb = 4 if akvq_delta else w.k_bits
+    spec = kvq.CacheSpec(kb, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
+                         w.batch, n, window=window, sink=sink, akvq_delta=akvq_delta)
     G, d = w.group, w.head_dim
-    blk = G * d * (w.k_bits + w.v_bits) // 8 + 8 * d
+    blk = G * d * (kb + w.v_bits) // 8 + 8 * d
     after = n - min(n, sink)                                  # tokens after the sink
     nq = G * ((after - window) // G) if after > window else 0   # quantized tokens
-    byts = w.n_kv_heads * ((nq // G) * blk + (n - nq) * 4 * d) + w.n_q_heads * d * 2
+    if akvq_delta:
+        # groups wholly before Delta or ending after n - Delta keep 4-bit keys
+        blk2 = G * d * (2 + w.v_bits) // 8 + 8 * d
+        wide = sum(1 for g in range(nq // G)
+                   if (g + 1) * G <= akvq_delta or (g + 1) * G > n - akvq_delta)
+        qbytes = wide * blk + (nq // G - wide) * blk2
+    else:
+        qbytes = (nq // G) * blk
+    byts = w.n_kv_heads * (qbytes + (n - nq) * 4 * d) + w.n_q_heads * d * 2
     copies = max(2, math.ceil(3 * L2_BYTES / byts))
     k = torch.from_numpy(np.concatenate(w.keys)).to(device)
     v = torch.from_numpy(np.concatenate(w.values)).to(device)
@@ -450,7 +464,9 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0):
             raise RuntimeError("decode kernel reported a failed wait")
     peak, peak_kind = _peaks()
     res = {"workload": "long_ctx", "context": n, "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv",
-           "bits": f"K{w.k_bits}/V{w.v_bits}", "group": G, "window": window, "sink": sink,
+           "bits": (f"K4 (first and last {akvq_delta} tokens) / K2 (middle) / V{w.v_bits}"
+                    if akvq_delta else f"K{w.k_bits}/V{w.v_bits}"),
+           "group": G, "window": window, "sink": sink, "akvq_delta": akvq_delta,
            "fp16_tokens": n - nq, "copies": copies,
            "bytes_per_launch": int(byts), "avg_launch_us": round(us, 3),
            "achieved_gbs": round(byts / us / 1e3, 1), "peak": peak, "peak_kind": peak_kind,
@@ -901,6 +917,9 @@ def main():
                     help="recent fp16 window of the extra 128k-token decode leg (0: skip it)")
     ap.add_argument("--sink", type=int, default=32,
                     help="fp16 sink window of one more 128k-token leg, with --window (0: skip it)")
+    ap.add_argument("--akvq-delta", type=int, default=1024,
+                    help="Delta of one more 128k-token leg with position-adaptive key widths "
+                         "(0: skip it)")
     ap.add_argument("--other-legs", type=int, default=1,
                     help="also time the quantize/append workload and the 70B-shaped batch "
                          "(0: skip)")
@@ -965,6 +984,10 @@ def main():
                 out["sink_window_decode"] = run_long_context(
                     stream, device, iters=max(1, args.steps), window=args.window, fp16=False,
                     sink=args.sink)
+            if args.akvq_delta:
+                out["akvq_decode"] = run_long_context(
+                    stream, device, iters=max(1, args.steps), fp16=False,
+                    akvq_delta=args.akvq_delta)
             print(json.dumps(out))
         if world > 1:
             import torch.distributed as tdist
@@ -994,6 +1017,8 @@ def main():
             line["recent_window_decode"] = res["window"]
         if res["sink"]:
             line["sink_window_decode"] = res["sink"]
+        if res["akvq"]:
+            line["akvq_decode"] = res["akvq"]
         if res.get("quant_append"):
             line["quant_append"] = res["quant_append"]
         if res.get("conc70b"):

@@ -158,6 +158,21 @@ typedef struct {
                               fp32(1 / sqrt(d)), then fp16); the decode
                               rotates q the same way and rotates its output
                               back.  0: no rotation */
+  int32_t akvq_delta;      /* Delta > 0: position-adaptive key bits ("Asymmetric
+                              Key-Value Quantization: 2-Bit Values and 4-Bit
+                              Keys under Long-Context Drift", §3.2): 4-bit keys
+                              (k_bits must be 4) for the early key groups (all
+                              positions < Delta) and the recent ones (last
+                              position >= n - Delta), 2-bit keys in between; a
+                              4-bit group that ages into the middle is
+                              requantized to 2 bits from its dequantized keys,
+                              fp16(fp32(s) * code + fp32(z)), by the append
+                              that moves it there.  A multiple of group, at
+                              most 2^20; needs window = sink = 0.  Every group
+                              keeps a slot of block_bytes (the 4-bit block);
+                              a 2-bit group's block (akvq_block_bytes, the
+                              sections at the akvq_* offsets) starts at its
+                              slot.  0: off */
 } kvq_config;
 
 typedef struct {
@@ -175,6 +190,9 @@ typedef struct {
   uint64_t sinks_offset;   /* first sink area (0 bytes each when sink = 0) */
   uint64_t sink_bytes;     /* K + V sink of one (seq, kv head) = 4*SW*d */
   uint64_t sink_slots;     /* SW: sink rounded up to a multiple of 16 */
+  uint64_t akvq_block_bytes;                          /* a 2-bit key group's block */
+  uint64_t akvq_kscale_offset, akvq_kmin_offset;      /* within that block (codes at 0) */
+  uint64_t akvq_vcodes_offset, akvq_vscale_offset, akvq_vmin_offset;
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache;
@@ -284,9 +302,9 @@ KVQ_API kvq_status kvq_decode(kvq_cache* cache, const void* q, kvq_dtype q_dtype
  * number of CTAs until the partials fit, and launches the same decode
  * kernel.  All calls share the array, which keeps the last call's contents,
  * so calls that overlap on the GPU (other streams, other threads) race:
- * serialize them.  The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress); make that first call before any
- * stream capture.  Arguments and errors as kvq_decode; KVQ_ERR_CAPACITY
+ * serialize them.  The first call on each device also looks up the array's
+ * device address (cudaGetSymbolAddress).  Arguments and errors as
+ * kvq_decode; KVQ_ERR_CAPACITY
  * (nothing launched) when the units of one launch - min(n_seq, 2048)
  * sequences x n_kv_heads x head slices of 8 query heads - need more split
  * records than the array holds (about 690,000 units).  A failed internal

@@ -19,7 +19,8 @@ def kvq():
 def oracle_cfg(spec) -> o.Config:
     return o.Config(spec.k_bits, spec.v_bits, spec.group, spec.head_dim, spec.n_q_heads,
                     spec.n_kv_heads, window=getattr(spec, "window", 0),
-                    sink=getattr(spec, "sink", 0), rotate=bool(getattr(spec, "rotate", 0)))
+                    sink=getattr(spec, "sink", 0), rotate=bool(getattr(spec, "rotate", 0)),
+                    akvq_delta=getattr(spec, "akvq_delta", 0))
 
 
 def to_device(x: np.ndarray, dtype: str) -> torch.Tensor:

@@ -107,6 +107,32 @@ def test_bad_config_rejected(kvq, field, value):
     assert not h.value
 
 
+@pytest.mark.parametrize("kw", [dict(akvq_delta=48), dict(akvq_delta=-32),
+                                dict(akvq_delta=(1 << 20) + 32), dict(akvq_delta=64, k_bits=2),
+                                dict(akvq_delta=64, window=32), dict(akvq_delta=64, sink=4)])
+def test_bad_position_adaptive_config_rejected(kvq, kw):
+    """Delta: a multiple of the group size in [0, 2^20], with 4-bit keys and
+    neither a recent window nor a sink window."""
+    cfg = _cfg(kvq, **kw)
+    assert kvq.kvq_cache_required_bytes(ctypes.byref(cfg), None, None) == 2
+    assert "akvq_delta" in kvq.kvq_last_error().decode()
+
+
+@pytest.mark.parametrize("vb,G,d", [(2, 32, 128), (4, 64, 128), (2, 32, 64), (2, 64, 64)])
+def test_position_adaptive_block_sections(kvq, vb, G, d):
+    """The 2-bit-key block of a position-adaptive cache has the sections of a
+    plain 2-bit-key block and sits at the start of the 4-bit slot."""
+    cfg = _cfg(kvq, v_bits=vb, group=G, head_dim=d, akvq_delta=4 * G)
+    assert kvq.kvq_cache_required_bytes(ctypes.byref(cfg), None, None) == 0
+    lay = kvq.layout_for(cfg)
+    sec2 = o.block_sections(o.Config(2, vb, G, d, 32, 8))
+    assert lay["akvq_block_bytes"] == sec2["total"][1]
+    for name in ("kscale", "kmin", "vcodes", "vscale", "vmin"):
+        assert lay["akvq_" + name + "_offset"] == sec2[name][0]
+    assert lay["block_bytes"] == o.block_sections(o.Config(4, vb, G, d, 32, 8))["total"][1]
+    assert lay["akvq_block_bytes"] < lay["block_bytes"] and lay["akvq_block_bytes"] % 16 == 0
+
+
 def test_head_dim_64_with_group_64_is_valid(kvq):
     cfg = _cfg(kvq, head_dim=64, group=64)
     assert kvq.kvq_cache_required_bytes(ctypes.byref(cfg), None, None) == 0
