@@ -23,9 +23,10 @@
 // it (q = p - S).
 //
 // Every CTA reads the sequence's current length from the device copy when
-// it starts; the last CTA of the sequence to finish (atomic ticket in the
-// cache buffer, no waiting) stores the new length and re-arms the ticket.
-// All reads of the old length therefore precede its update.
+// it starts and counts itself on the sequence's ticket (an atomic in the
+// cache buffer, no waiting); the CTA that counts last stores the new length
+// at its end and re-arms the ticket.  All reads of the old length therefore
+// precede its update.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -59,7 +60,9 @@ struct AppCfg {
   static constexpr int SM_VZ = SM_VS + 2 * G * J;
   static constexpr int SM_KP = (SM_VZ + 2 * G * J + 15) / 16 * 16;
   static constexpr int SM_VP = SM_KP + 16 * D;
-  static constexpr int SM_TOTAL = SM_VP + 16 * G * J;
+  // per row slice and key channel pair: fp16x2 {min, max} (key_stats_part)
+  static constexpr int SM_KR = SM_VP + 16 * G * J;
+  static constexpr int SM_TOTAL = SM_KR + 8 * (128 / (D / 2)) * (D / 2);
 };
 
 // Eight consecutive input elements (16-byte aligned) rounded to fp16
@@ -207,40 +210,106 @@ __device__ __forceinline__ void codes2(float x0, float x1, float z0, float z1, f
   near_tie |= (a0 >= 0x3EFFF800u) | (a1 >= 0x3EFFF800u);   // 0.5 - 2048 ulp
 }
 
-// Key statistics of a staged group (fp16 rows of DP halves, G tokens):
-// per channel min and max over the tokens (fp16x2, exact), the stored fp16
-// scale fp16((max - min) / QK) and min, their fp32 {z, 1/s, s} for the
-// codes, and the metadata in slot order i*(D/4) + 4kt + 2v + e.  Threads
-// 0..63.
-template <int D, int G, int QK>
-__device__ __forceinline__ void key_stats(const __half* __restrict__ sk, float4* __restrict__ kp,
-                                          __half* __restrict__ ks, __half* __restrict__ kz,
-                                          int tid) {
+// Key statistics of a staged group (fp16 rows of DP halves, G tokens), in
+// two phases over the 128 threads.  Part: thread (slice rs, channel pair
+// cp) takes the fp16x2 min and max (exact) over its G / NS rows into
+// part[rs][cp] = {min, max}.  Final (after a barrier; thread c < D): the
+// channel's min and max over the slices, the stored fp16 scale
+// fp16((max - min) / QK) and min, their fp32 {z, 1/s, s} for the codes,
+// and the metadata in slot order i*(D/4) + 4kt + 2v + e.
+template <int D, int G>
+__device__ __forceinline__ void key_stats_part(const __half* __restrict__ sk,
+                                               uint2* __restrict__ part, int tid) {
   constexpr int DP = D + 8;
+  constexpr int NS = 128 / (D / 2);   // row slices
+  constexpr int RS = G / NS;          // rows per slice
   const __half2* sk2 = reinterpret_cast<const __half2*>(sk);
-  for (int cp = tid; cp < D / 2; cp += 64) {
-    __half2 mn = sk2[cp], mx = mn;
-    for (int r = 1; r < G; ++r) {
-      const __half2 x = sk2[r * (DP / 2) + cp];
-      mn = __hmin2(mn, x);
-      mx = __hmax2(mx, x);
-    }
+  const int cp = tid % (D / 2), rs = tid / (D / 2);
+  const __half2* col = sk2 + rs * RS * (DP / 2) + cp;
+  __half2 mn = col[0], mx = mn;
 #pragma unroll
+  for (int r = 1; r < RS; ++r) {
+    const __half2 x = col[r * (DP / 2)];
+    mn = __hmin2(mn, x);
+    mx = __hmax2(mx, x);
+  }
+  part[rs * (D / 2) + cp] = make_uint2(h2_as_u32(mn), h2_as_u32(mx));
+}
+template <int D, int G, int QK>
+__device__ __forceinline__ void key_stats_final(const uint2* __restrict__ part,
+                                                float4* __restrict__ kp, __half* __restrict__ ks,
+                                                __half* __restrict__ kz, int c) {
+  constexpr int NS = 128 / (D / 2);
+  const int cp = c >> 1, e = c & 1;
+  float mnf = INFINITY, mxf = -INFINITY;
+#pragma unroll
+  for (int rs = 0; rs < NS; ++rs) {
+    const uint2 pm = part[rs * (D / 2) + cp];
+    const __half2 mn = *reinterpret_cast<const __half2*>(&pm.x);
+    const __half2 mx = *reinterpret_cast<const __half2*>(&pm.y);
+    mnf = fminf(mnf, e ? __high2float(mn) : __low2float(mn));
+    mxf = fmaxf(mxf, e ? __high2float(mx) : __low2float(mx));
+  }
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)QK));
+  const __half z16 = __float2half_rn(mnf);
+  const float sf = __half2float(s16);
+  kp[c] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
+  // metadata slot i*(D/4) + 4kt + 2v + e
+  const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3;
+  const int slot = i * (D / 4) + 4 * kt + 2 * v + e;
+  ks[slot] = s16;
+  kz[slot] = z16;
+}
+
+// A key-code word recomputed with IEEE division (the rare words whose fast
+// quotients lie near a rounding boundary): token t, word w of lane group i.
+// Out of line, so that the hot loops stay small in the instruction cache.
+template <int D, int KBq>
+__device__ __noinline__ uint32_t key_word_exact(const __half* __restrict__ sk,
+                                                const float4* __restrict__ kp, int t, int w, int i) {
+  constexpr int DP = D + 8;
+  constexpr int QK = (1 << KBq) - 1;
+  constexpr int FK = 16 / KBq;
+  uint32_t word = 0;
+#pragma unroll 1
+  for (int f = 0; f < FK; ++f) {
+    const int p = w * FK + f;
+    const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
+#pragma unroll 1
     for (int e = 0; e < 2; ++e) {
-      const int c = 2 * cp + e;
-      const float mnf = e ? __high2float(mn) : __low2float(mn);
-      const float mxf = e ? __high2float(mx) : __low2float(mx);
-      const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mxf, mnf), (float)QK));
-      const __half z16 = __float2half_rn(mnf);
-      const float sf = __half2float(s16);
-      kp[c] = make_float4(__half2float(z16), sf == 0.0f ? 0.0f : __frcp_rn(sf), sf, 0.0f);
-      // metadata slot i*(D/4) + 4kt + 2v + e
-      const int kt = c >> 4, v = (c >> 3) & 1, i = (c >> 1) & 3, ee = c & 1;
-      const int slot = i * (D / 4) + 4 * kt + 2 * v + ee;
-      ks[slot] = s16;
-      kz[slot] = z16;
+      const float4 pc = kp[c + e];
+      const uint32_t code = (uint32_t)quant_code(__half2float(sk[t * DP + c + e]), pc.x, pc.z, QK);
+      word |= code << (KBq * (e * FK + f));
     }
   }
+  return word;
+}
+
+// The same for a value-code word: token tile kv, word w, lane (gg, i).
+template <int D, int G, int VB>
+__device__ __noinline__ uint32_t value_word_exact(const __half* __restrict__ sv,
+                                                  const float4* __restrict__ vp, int kv, int w,
+                                                  int gg, int i) {
+  constexpr int DP = D + 8;
+  constexpr int J = D / G;
+  constexpr int QV = (1 << VB) - 1;
+  constexpr int FV = 16 / VB;
+  uint32_t word = 0;
+#pragma unroll 1
+  for (int fl = 0; fl < FV; ++fl) {
+    const int kh = fl / (FV / 2), rem = fl % (FV / 2);
+    const int u = rem >> 1, hr = rem & 1;
+    const int mt = w * (FV / 4) + u;
+    const int c = 16 * mt + 8 * hr + gg;
+#pragma unroll 1
+    for (int e = 0; e < 2; ++e) {
+      const int t = 16 * kv + 8 * kh + 2 * i + e;
+      const float4 pc = vp[t * J + c / G];
+      const uint32_t code = (uint32_t)quant_code(__half2float(sv[t * DP + c]), pc.x, pc.z, QV);
+      word |= code << (VB * (e * FV + fl));
+    }
+  }
+  return word;
 }
 
 // Key codes of a staged group at KBq bits, packed word by word into the
@@ -276,7 +345,10 @@ __device__ __forceinline__ void key_codes(const __half* __restrict__ sk, const f
         rk[f][e] = pc.y;
       }
     }
-    for (int wi = tid; wi < KWORDS; wi += 128) {
+    static_assert(KWORDS % 128 == 0, "whole passes of the 128 threads");
+#pragma unroll 1
+    for (int pass = 0; pass < KWORDS / 128; ++pass) {
+      const int wi = tid + 128 * pass;
       const int nt = wi / (KWPL * 32);
       const int t = 8 * nt + (lane >> 2);
       const int widx = (nt * 32 + lane) * KWPL + w;   // layout word
@@ -292,33 +364,26 @@ __device__ __forceinline__ void key_codes(const __half* __restrict__ sk, const f
         codes2(x.x, x.y, zk[f][0], zk[f][1], rk[f][0], rk[f][1], QK, c0, c1, tie);
         word |= ((c0 & QK) << (KBq * f)) | ((c1 & QK) << (KBq * (FK + f)));
       }
-      if (tie) {   // rare: IEEE division for the whole word
-        word = 0;
-#pragma unroll
-        for (int f = 0; f < FK; ++f) {
-          const int p = w * FK + f;
-          const int c = 16 * (p >> 1) + 8 * (p & 1) + 2 * i;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float4 pc = kp[c + e];
-            const uint32_t code =
-                (uint32_t)quant_code(__half2float(sk[t * DP + c + e]), pc.x, pc.z, QK);
-            word |= code << (KBq * (e * FK + f));
-          }
-        }
-      }
+      if (tie) word = key_word_exact<D, KBq>(sk, kp, t, w, i);   // rare
       kw[widx] = word;
     }
   }
 }
 
-template <int D, int G, int KB, int VB>
+// PLAIN: fp16 inputs into a cache with no recent window, no sink window, no
+// rotation and one key width (the common case, compiled without the code of
+// the others).
+template <int D, int G, int KB, int VB, bool PLAIN>
 __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char* __restrict__ cache,
                                                      const void* __restrict__ kin,
-                                                     const void* __restrict__ vin, const int dtype,
+                                                     const void* __restrict__ vin, const int dtype_arg,
                                                      const AppendSeqs s) {
   using C = AppCfg<D, G, KB, VB>;
   extern __shared__ __align__(16) unsigned char sm[];
+  const int dtype = PLAIN ? (int)KVQ_FP16 : dtype_arg;
+  const int g_sink = PLAIN ? 0 : g.sink;
+  const int g_window = PLAIN ? 0 : g.window;
+  const int g_akvq = PLAIN ? 0 : g.akvq_delta;
   __half* sk = reinterpret_cast<__half*>(sm + C::SM_K);
   __half* sv = reinterpret_cast<__half*>(sm + C::SM_V);
   __half* ks = reinterpret_cast<__half*>(sm + C::SM_KS);
@@ -343,19 +408,33 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   const int seq = s.seq0 + b;
   int32_t* lens = reinterpret_cast<int32_t*>(cache + g.lens_off);
   int32_t* tickets = reinterpret_cast<int32_t*>(cache + g.counters_off);
-  const int len0 = *reinterpret_cast<volatile int32_t*>(lens + seq);
   const int nn = s.n_new[b];
   const int seq_ctas = (s.task_prefix[b + 1] - s.task_prefix[b]) * gridDim.y;
-  const int W = g.tail_slots;      // ring slots of the tail: R + G
+  // The sequence's current length: read once (thread 0, acquire), then
+  // counted on the sequence's ticket.  The CTA that counts last has seen
+  // every other CTA of the sequence read the length, so it may publish the
+  // new one (below, after its acquire count: no later read of the old value
+  // can see it); nothing else of this launch reads the length.  No fence
+  // orders the cache writes: the next kernel on the stream sees them all.
+  __shared__ int32_t len_s;
+  int ticket_old = -1;
+  if (tid == 0) {
+    const int l0 = ld_acquire_gpu(lens + seq);
+    len_s = l0;
+    ticket_old = atomic_add_acquire_gpu(tickets + seq, 1);
+  }
+  __syncthreads();
+  const int len0 = len_s;
+  const int W = PLAIN ? G : g.tail_slots;   // ring slots of the tail: R + G
   const int n1 = len0 + nn;
   // positions after the sink (q = p - S): a0 before, a1 after this append;
   // the first nsink new tokens (input rows 0 .. nsink-1) go to the sink
-  const int a0 = max(len0 - g.sink, 0);
-  const int a1 = max(n1 - g.sink, 0);
-  const int nsink = max(min(n1, g.sink) - len0, 0);
-  const int N0 = G * quantized_groups(a0, G, g.window);
+  const int a0 = max(len0 - g_sink, 0);
+  const int a1 = max(n1 - g_sink, 0);
+  const int nsink = PLAIN ? 0 : max(min(n1, g_sink) - len0, 0);
+  const int N0 = G * quantized_groups(a0, G, g_window);
   const int T0 = a0 - N0;          // tail length before
-  const int N1 = G * quantized_groups(a1, G, g.window);
+  const int N1 = G * quantized_groups(a1, G, g_window);
   const int F = (N1 - N0) / G;     // groups completed by this append
   const int64_t row0 = s.row_off[b];
   const int64_t unit = (int64_t)seq * g.hkv + kvh;
@@ -366,10 +445,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   // A replayed capture can ask for more than the capacity, which the host
   // could not check: such an append writes nothing and the length stays.
   const bool fits = (int64_t)len0 + nn <= g.max_tokens;
-  // the last CTA of this sequence to finish publishes the new length
+  // the CTA that counted last publishes the new length and re-arms the ticket
   auto finish = [&]() {
-    __syncthreads();
-    if (tid == 0 && atomic_add_acq_rel_gpu(tickets + seq, 1) == seq_ctas - 1) {
+    if (tid == 0 && ticket_old == seq_ctas - 1) {
       if (fits) lens[seq] = len0 + nn;
       tickets[seq] = 0;
     }
@@ -381,7 +459,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
 
   constexpr int CPR = D / 8;   // 16-byte fp16 chunks per token row
   // new sink tokens: input row j -> sink slot len0 + j (nobody reads them here)
-  const bool rot = g.rotate != 0;
+  const bool rot = PLAIN ? false : g.rotate != 0;
   // The loops over input rows below run whole warps (row_chunk16 exchanges
   // across a warp when the cache rotates); a lane past the end loads nothing.
   auto write_sink = [&]() {
@@ -406,9 +484,9 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   // per sequence for appends of fewer than G tokens (at most one group ages
   // then); a task with no group to age does nothing.
   if constexpr (KB == 4) {
-    if (g.akvq_delta && tau >= (F > 0 ? F : 1)) {
+    if (g_akvq && tau >= (F > 0 ? F : 1)) {
       int first;
-      const int A = akvq_aging(len0, n1, N0 / G, G, g.akvq_delta, &first);
+      const int A = akvq_aging(len0, n1, N0 / G, G, g_akvq, &first);
       const int r = tau - (F > 0 ? F : 1);
       if (r < A) {
         unsigned char* blk = cache + g.blocks_off +
@@ -439,7 +517,10 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
           *reinterpret_cast<uint4*>(vkeep + i) = *reinterpret_cast<const uint4*>(blk + g.sec_vcodes + i);
         __syncthreads();   // every read of the old block is done
         float4* kp = reinterpret_cast<float4*>(sm + C::SM_KP);
-        if (tid < 64) key_stats<D, G, 3>(sk, kp, ks, kz, tid);
+        uint2* kr = reinterpret_cast<uint2*>(sm + C::SM_KR);
+        key_stats_part<D, G>(sk, kr, tid);
+        __syncthreads();
+        if (tid < D) key_stats_final<D, G, 3>(kr, kp, ks, kz, tid);
         __syncthreads();
         key_codes<D, G, 2>(sk, kp, reinterpret_cast<uint32_t*>(blk), tid);
         for (int i = tid; i < D / 2; i += 128) {
@@ -511,18 +592,24 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
 
   // key width of this group: the cache's, or with position-adaptive bits
   // the width of its region once this append is done
-  const int kbits = (KB == 4 && g.akvq_delta) ? akvq_key_bits(N0 / G + tau, n1, G, g.akvq_delta) : KB;
+  const int kbits = (KB == 4 && g_akvq) ? akvq_key_bits(N0 / G + tau, n1, G, g_akvq) : KB;
 
-  // ---- statistics.  Warps 0-1: keys, two channels per thread (fp16x2
-  // min/max over the G tokens).  Warps 2-3: values, (token, group of G
-  // channels) items, 16-byte loads.  fp16 min/max of fp16 values is exact.
+  // ---- statistics.  Keys: partial fp16x2 min/max per (row slice, channel
+  // pair) by every thread, then one channel per thread after a barrier.
+  // Values: one (token, group of G channels) item per thread, 16-byte
+  // loads.  fp16 min/max of fp16 values is exact.
   float4* kp = reinterpret_cast<float4*>(sm + C::SM_KP);   // [c]: {z, 1/s, s, -}
   float4* vp = reinterpret_cast<float4*>(sm + C::SM_VP);   // [r * J + j]
-  if (tid < 64) {
-    if (kbits == KB) key_stats<D, G, (1 << KB) - 1>(sk, kp, ks, kz, tid);
-    else key_stats<D, G, 3>(sk, kp, ks, kz, tid);
-  } else {
-    for (int q = tid - 64; q < G * C::J; q += 64) {
+  uint2* kr = reinterpret_cast<uint2*>(sm + C::SM_KR);
+  key_stats_part<D, G>(sk, kr, tid);
+  __syncthreads();
+  if (tid < D) {
+    if (kbits == KB) key_stats_final<D, G, (1 << KB) - 1>(kr, kp, ks, kz, tid);
+    else key_stats_final<D, G, 3>(kr, kp, ks, kz, tid);
+  }
+  {
+    static_assert(G * C::J <= 128, "one value item per thread");
+    for (int q = tid; q < G * C::J; q += 128) {
       const int r = q / C::J, j = q % C::J;
       const uint4* row = reinterpret_cast<const uint4*>(sv + r * C::DP + j * G);
       constexpr int NV = G / 8;
@@ -560,7 +647,10 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   if (kbits == KB) key_codes<D, G, KB>(sk, kp, reinterpret_cast<uint32_t*>(blk + g.sec_kcodes), tid);
   else key_codes<D, G, 2>(sk, kp, reinterpret_cast<uint32_t*>(blk), tid);
   uint32_t* vw = reinterpret_cast<uint32_t*>(blk + (kbits == KB ? g.sec_vcodes : g.a2_vcodes));
-  for (int wi = tid; wi < C::VWORDS; wi += blockDim.x) {
+  static_assert(C::VWORDS % 128 == 0, "whole passes of the 128 threads");
+#pragma unroll 1
+  for (int pass = 0; pass < C::VWORDS / 128; ++pass) {
+    const int wi = tid + 128 * pass;
     // lane fastest (a warp reads 4 token pairs x 8 channels: distinct banks
     // of the padded rows), then the lane's word w, then the token tile
     const int lane = wi % 32;
@@ -592,24 +682,7 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
              p0.y, p1.y, C::QV, c0, c1, tie);
       word |= ((c0 & C::QV) << (VB * fl)) | ((c1 & C::QV) << (VB * (C::FV + fl)));
     }
-    if (tie) {
-      word = 0;
-#pragma unroll
-      for (int fl = 0; fl < C::FV; ++fl) {
-        const int kh = fl / (C::FV / 2), rem = fl % (C::FV / 2);
-        const int u = rem >> 1, hr = rem & 1;
-        const int mt = w * (C::FV / 4) + u;
-        const int c = 16 * mt + 8 * hr + gg;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 16 * kv + 8 * kh + 2 * i + e;
-          const float4 pc = vp[t * C::J + c / G];
-          const uint32_t code =
-              (uint32_t)quant_code(__half2float(sv[t * C::DP + c]), pc.x, pc.z, C::QV);
-          word |= code << (VB * (e * C::FV + fl));
-        }
-      }
-    }
+    if (tie) word = value_word_exact<D, G, VB>(sv, vp, kv, w, gg, i);   // rare
     vw[widx] = word;
   }
   // metadata sections are copied verbatim (already in slot order)
@@ -672,12 +745,14 @@ template <int D, int G, int KB, int VB>
 cudaError_t launch_append_t(const Geom& g, unsigned char* cache, const void* k, const void* v,
                             int dtype, const AppendSeqs& seqs, int n_tasks, cudaStream_t stream) {
   using C = AppCfg<D, G, KB, VB>;
-  auto kern = append_kernel<D, G, KB, VB>;
-  static bool configured = false;   // attribute set once, before any capture
-  if (!configured) {
+  const bool plain = dtype == KVQ_FP16 && g.window == 0 && g.sink == 0 && g.rotate == 0 &&
+                     g.akvq_delta == 0;
+  auto kern = plain ? append_kernel<D, G, KB, VB, true> : append_kernel<D, G, KB, VB, false>;
+  static bool configured[2] = {false, false};   // attribute set once, before any capture
+  if (!configured[plain]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SM_TOTAL);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[plain] = true;
   }
   dim3 grid(n_tasks, g.hkv);
   kern<<<grid, 128, C::SM_TOTAL, stream>>>(g, cache, k, v, dtype, seqs);

@@ -160,6 +160,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // that precede it (the CTA's, when a CTA barrier comes first) are visible to
 // whoever reads the incremented value, and it is ordered before the caller's
 // later accesses.
+__device__ __forceinline__ int atomic_add_acquire_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acquire.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
   int old;
   asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
