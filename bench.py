@@ -753,12 +753,24 @@ def _traffic():
             rec = json.load(f)
     except Exception:
         return None
-    import hashlib
-    src = os.path.join(ROOT, "asymmetric_kv_cache_b200", "csrc", "kvq_decode.cu")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if rec.get("kernel_sha256_16") != h:
+    if rec.get("kernel_sha256_16") != decode_source_hash():
         return None
     return rec.get("dram_bytes_per_launch_full_workload")
+
+
+# the sources of the timed decode kernel (the record of its DRAM traffic is
+# valid only for these bytes)
+DECODE_SOURCES = ("kvq_decode.cu", "kvq_decode_kernels.cuh", "kvq_decode_d128_g32_v2.cu",
+                  "kvq_split.h", "kvq_device.cuh", "kvq_internal.h")
+
+
+def decode_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "asymmetric_kv_cache_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------

@@ -99,6 +99,11 @@
  * (These are the tensor-core fragment orders the decode kernel reads with
  * 128-bit loads; the packing is a fixed permutation, so every token still
  * costs a fixed number of bits.)
+ * Position-adaptive key bits (kvq_config.akvq_delta > 0, k_bits = 4): slots
+ * stay block_bytes apart (the 4-bit block); a group whose keys are at 2 bits
+ * holds, from the start of its slot, the block of a 2-bit-key cache (the
+ * same sections and packing with kbits = 2: offsets akvq_* in kvq_layout,
+ * akvq_block_bytes long); the rest of that slot is unspecified.
  */
 #ifndef KVQ_H_
 #define KVQ_H_
