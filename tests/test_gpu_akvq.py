@@ -182,3 +182,35 @@ def test_long_context_full_size():
     want = o.akvq_decode(cfg, w.keys[0], w.values[0], w.q[0], sched)[None]
     assert tl.decode_error(out, want) <= tl.DECODE_TOL
     assert cache.workspace_status() == 0
+
+
+@pytest.mark.parametrize("gqa", [4, 8])
+def test_rotated_adaptive_cache(gqa):
+    """Rotation and position-adaptive widths together: the cache holds the
+    rotated tokens (fp32 butterfly, fp16), the widths and requantizations
+    act on them, the decode rotates q and its output back.  Expected values:
+    the oracle's adaptive image and decode of the rotated tokens, with the
+    query rotated in and the output rotated back (the steps of its rotated
+    decode)."""
+    K = tl.kvq()
+    G, d, hkv = 32, 128, 2
+    spec = K.CacheSpec(4, 2, G, d, hkv * gqa, hkv, 3, 1024, rotate=1, akvq_delta=2 * G)
+    schedules = [[5 * G + 3] + [1] * 40, [1] * 70 + [3 * G], [9 * G + 1, G, 7]]
+    lens = [sum(s) for s in schedules]
+    rng = np.random.default_rng(990 + gqa)
+    ks, vs = _hist(rng, lens, hkv, d)
+    cache = K.KVQCache(spec)
+    _append_schedule(cache, ks, vs, schedules)
+    cfg = tl.oracle_cfg(spec)
+    plain = o.Config(cfg.k_bits, cfg.v_bits, cfg.group, cfg.head_dim, cfg.n_q_heads,
+                     cfg.n_kv_heads, akvq_delta=cfg.akvq_delta)
+    kr = [o.cache_tokens(cfg, x) for x in ks]
+    vr = [o.cache_tokens(cfg, x) for x in vs]
+    for b in range(len(lens)):
+        _check_bytes(cache, plain, kr[b], vr[b], schedules[b], b)
+    q = rng.standard_normal((len(lens), hkv * gqa, d)).astype(np.float16).astype(np.float32)
+    out = cache.decode(tl.to_device(q, "fp16"))
+    want = np.stack([o.rotate_fp64(o.akvq_decode(plain, kr[b], vr[b], o.rotate_fp64(q[b]),
+                                                 schedules[b])) for b in range(len(lens))])
+    assert tl.decode_error(out, want) <= tl.DECODE_TOL
+    assert cache.workspace_status() == 0
