@@ -337,6 +337,8 @@ def run_ours(args, rank, world, device):
              if args.long_context and args.sink else None)
     akvq = (run_long_context(stream, device, akvq_delta=args.akvq_delta, fp16=False)
             if args.long_context and args.akvq_delta else None)
+    rot = (run_long_context(stream, device, rotate=1, fp16=False)
+           if args.long_context and args.rotate else None)
     qa = run_quant_append(stream, device) if args.other_legs else None
     c70 = run_concurrent_70b(stream, device) if args.other_legs else None
 
@@ -363,7 +365,8 @@ def run_ours(args, rank, world, device):
         "value": value, "ms_per_step": total_ms / wl.K, "e2e": e2e, "roofline": roof,
         "clocks": clocks, "gpu_launches": 3 * wl.K, "wl": wl, "fp16": fp16,
         "decode_ms": dec_avg_ms, "kv_tokens_per_step": kv_tokens / wl.K, "long_ctx": long_ctx,
-        "window": window, "sink": sinkw, "akvq": akvq, "quant_append": qa, "conc70b": c70,
+        "window": window, "sink": sinkw, "akvq": akvq, "rot": rot, "quant_append": qa,
+        "conc70b": c70,
     }
 
 
@@ -405,7 +408,8 @@ def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
             "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
 
 
-def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akvq_delta=0):
+def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akvq_delta=0,
+                     rotate=0):
     """Decode alone on the 128k-token long-context workload (batch 1, 32 q /
     8 kv heads, d 128, K2/V2, G 32): the configuration the HBM-roofline
     target is stated on.  Copies of the cache (> 3x L2 in total) are
@@ -417,14 +421,16 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akv
     token-head).  `akvq_delta` > 0: position-adaptive key widths on the same
     context (4-bit keys for the first and the last Delta tokens' groups,
     2-bit keys in between, 2-bit values), each group's bytes counted at its
-    own width."""
+    own width.  `rotate` = 1: the rotating cache (q rotated in, the output
+    rotated back)."""
     import torch
     from asymmetric_kv_cache_b200 import inputs, kvq
     w = inputs.WORKLOADS["long_ctx"]()
     n = w.lens[0]
     kb = 4 if akvq_delta else w.k_bits
     spec = kvq.CacheSpec(kb, w.v_bits, w.group, w.head_dim, w.n_q_heads, w.n_kv_heads,
-                         w.batch, n, window=window, sink=sink, akvq_delta=akvq_delta)
+                         w.batch, n, window=window, sink=sink, akvq_delta=akvq_delta,
+                         rotate=rotate)
     G, d = w.group, w.head_dim
     blk = G * d * (kb + w.v_bits) // 8 + 8 * d
     after = n - min(n, sink)                                  # tokens after the sink
@@ -467,12 +473,15 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akv
            "bits": (f"K4 (first and last {akvq_delta} tokens) / K2 (middle) / V{w.v_bits}"
                     if akvq_delta else f"K{w.k_bits}/V{w.v_bits}"),
            "group": G, "window": window, "sink": sink, "akvq_delta": akvq_delta,
+           "rotate": rotate,
            "fp16_tokens": n - nq, "copies": copies,
            "bytes_per_launch": int(byts), "avg_launch_us": round(us, 3),
            "achieved_gbs": round(byts / us / 1e3, 1), "peak": peak, "peak_kind": peak_kind,
            "frac": round(byts / us / 1e3 / peak, 4), "launches": iters,
            "kv_tokens_per_s": round(n * iters / (e0.elapsed_time(e1) / 1e3), 1),
            "note": "decode + combine per launch, CUDA events around the launches"}
+    if not (window or sink or akvq_delta or rotate):
+        res["traffic"] = _traffic("decode_long_ctx_traffic.json")
     del caches
     if not fp16:
         del k, v
@@ -744,10 +753,10 @@ def run_e2e(args, wl, caches, nk, nv, q, stream, device):
             "mode": "CUDA graph; host<->device copies double-buffered on copy streams"}
 
 
-def _traffic():
+def _traffic(record="decode_traffic.json"):
     """DRAM bytes per decode launch from the committed ncu summary, if it was
     taken on the current decode kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    path = os.path.join(ROOT, "profiles", record)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -932,6 +941,8 @@ def main():
     ap.add_argument("--akvq-delta", type=int, default=1024,
                     help="Delta of one more 128k-token leg with position-adaptive key widths "
                          "(0: skip it)")
+    ap.add_argument("--rotate", type=int, default=1,
+                    help="one more 128k-token leg on the rotating cache (0: skip it)")
     ap.add_argument("--other-legs", type=int, default=1,
                     help="also time the quantize/append workload and the 70B-shaped batch "
                          "(0: skip)")
@@ -1000,6 +1011,9 @@ def main():
                 out["akvq_decode"] = run_long_context(
                     stream, device, iters=max(1, args.steps), fp16=False,
                     akvq_delta=args.akvq_delta)
+            if args.rotate:
+                out["rotated_decode"] = run_long_context(
+                    stream, device, iters=max(1, args.steps), fp16=False, rotate=1)
             print(json.dumps(out))
         if world > 1:
             import torch.distributed as tdist
@@ -1031,6 +1045,8 @@ def main():
             line["sink_window_decode"] = res["sink"]
         if res["akvq"]:
             line["akvq_decode"] = res["akvq"]
+        if res["rot"]:
+            line["rotated_decode"] = res["rot"]
         if res.get("quant_append"):
             line["quant_append"] = res["quant_append"]
         if res.get("conc70b"):
