@@ -418,6 +418,11 @@ __global__ void __launch_bounds__(128) append_kernel(const Geom g, unsigned char
   // orders the cache writes: the next kernel on the stream sees them all.
   __shared__ int32_t len_s;
   int ticket_old = -1;
+  // launched as a programmatic dependent of the previous kernel on the
+  // stream (the decode of the previous step, typically): the planning above
+  // reads only kernel parameters; nothing in memory is read or written
+  // before the previous grid has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) {
     const int l0 = ld_acquire_gpu(lens + seq);
     len_s = l0;
@@ -754,9 +759,20 @@ cudaError_t launch_append_t(const Geom& g, unsigned char* cache, const void* k, 
     if (e != cudaSuccess) return e;
     configured[plain] = true;
   }
-  dim3 grid(n_tasks, g.hkv);
-  kern<<<grid, 128, C::SM_TOTAL, stream>>>(g, cache, k, v, dtype, seqs);
-  return cudaGetLastError();
+  // a programmatic dependent of the previous kernel: its CTAs may be
+  // resident while that kernel runs, and wait for it (griddepcontrol.wait)
+  // before touching memory
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)n_tasks, (unsigned)g.hkv);
+  lc.blockDim = dim3(128);
+  lc.dynamicSmemBytes = C::SM_TOTAL;
+  lc.stream = stream;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = la;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, g, cache, k, v, dtype, seqs);
 }
 
 }  // namespace
