@@ -229,20 +229,23 @@ def run_ours(args, rank, world, device):
     # steps run as a user's loop would
     EV = 8
 
+    def evented(i, n):   # the 8th, 16th, ... step of a graph (its last if it has fewer)
+        return i % EV == EV - 1 or (n < EV and i == n - 1)
+
     def capture(n_steps, first_step):
         evs = [(torch.cuda.Event(enable_timing=True, external=True),
                 torch.cuda.Event(enable_timing=True, external=True))
-               for i in range(n_steps) if i % EV == 0]
+               for i in range(n_steps) if evented(i, n_steps)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n_steps):
                 s = first_step + i
                 c = s % C
                 caches[c].append(nk_dev[s % pool], nv_dev[s % pool], [1] * wl.batch, stream=stream)
-                if i % EV == 0:
+                if evented(i, n_steps):
                     evs[i // EV][0].record(stream)
                 caches[c].decode(q_dev[s % pool], out=out, stream=stream)
-                if i % EV == 0:
+                if evented(i, n_steps):
                     evs[i // EV][1].record(stream)
         return g, evs
 
@@ -315,10 +318,10 @@ def run_ours(args, rank, world, device):
         if last is None:
             continue
         collect(evs)
-        ev_idx += [last * C + i for i in range(steps_in_round) if i % EV == 0]
+        ev_idx += [last * C + i for i in range(steps_in_round) if evented(i, steps_in_round)]
     if gR is not None:
         collect(gR[1])
-        ev_idx += [rounds * C + i for i in range(rem) if i % EV == 0]
+        ev_idx += [rounds * C + i for i in range(rem) if evented(i, rem)]
     if ev_idx:
         ev_bytes = statistics.fmean(wl.algorithmic_bytes([lens_at[j]] * wl.batch)
                                     for j in ev_idx)
