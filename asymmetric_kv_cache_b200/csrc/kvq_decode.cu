@@ -17,8 +17,12 @@
 // one at a time from a shared counter (so warps that the schedulers favour
 // simply take more groups and all finish together), each with its own
 // online softmax, and merge through shared memory at the end of the piece.
-// A unit cut by CTA boundaries writes per-piece partials (m, l, o) that the
-// combine kernel merges.
+// A unit cut by CTA boundaries writes per-piece partials (m, l, o): the
+// last of its CTAs merges them (acquire-release ticket; wide CTAs with at
+// most 32 pieces per unit), else the combine kernel does.  With a rotating
+// cache the query rows are rotated before the fp16 split and every final
+// output row is rotated back; with position-adaptive key widths each group
+// is copied and read at its own width.
 //
 // Per group (one 32/64-token slot) a warp:
 //   * waits for the group block, brought into its own shared-memory ring by

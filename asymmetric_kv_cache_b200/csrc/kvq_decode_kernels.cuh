@@ -1,8 +1,9 @@
 // Kernel templates of the split-K decode over the quantized cache (libkvq,
 // sm_100a), shared by the translation units that instantiate them: one per
 // (head dim, group, value bits) family, so that the library builds in
-// parallel.  See kvq_decode.cu for the design; every definition here lives
-// in an unnamed namespace, so each translation unit keeps its own copies.
+// parallel.  The design is described at the top of kvq_decode.cu (dispatch,
+// fp16 baseline, no-alloc scratch); every definition here lives in an
+// unnamed namespace, so each translation unit keeps its own copies.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -1,11 +1,12 @@
 // Decode on the 5th-generation tensor cores (tcgen05) for d = 128, 32-token
 // groups, 2-bit values and GQA groups of at most 4 heads (the Llama-3-8B
 // shaped layer and the 128k-token long context).  Included by
-// kvq_decode.cu inside its anonymous namespace (it uses that file's Geom,
+// kvq_decode.cu after kvq_decode_kernels.cuh (it uses that header's Geom,
 // DecCfg, Piece, query conversion, fp16-tail code, merge helpers and split
 // records).  Same attention as decode_kernel (per-channel key and per-token
-// value dequantization, KIVI "Method" section; online softmax and the split
-// merge of the first page's flash-decoding baseline, Section IV), same
+// value dequantization, "[Framework] The Asymmetric Key-Value Cache
+// Compression", §III; online softmax and the split merge of that page's
+// flash-decoding baseline, §IV), same
 // stream-K split and partial format, so combine_kernel and
 // finish_split_unit serve both.
 //
