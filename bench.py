@@ -776,12 +776,19 @@ DECODE_SOURCES = ("kvq_decode.cu", "kvq_decode_kernels.cuh", "kvq_decode_d128_g3
                   "kvq_split.h", "kvq_device.cuh", "kvq_internal.h")
 
 
-def decode_source_hash() -> str:
+def decode_source_hash(root=None) -> str:
+    """Hash of the decode sources with their comments and blank lines taken
+    out (a comment edit does not change the kernel the record was taken on)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in DECODE_SOURCES:
-        with open(os.path.join(ROOT, "asymmetric_kv_cache_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(root or ROOT, "asymmetric_kv_cache_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        text = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 
