@@ -272,7 +272,6 @@ __global__ void __launch_bounds__(F16Cfg<D>::THREADS, 1)
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
 #pragma unroll
     for (int r = 0; r < (PK ? 2 : 1); ++r) st.m[r] = -INFINITY;
-    st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;   // unused here
     // the piece: slots [s0, s1) of unit (b, kvh, slice), slot = 16 tokens
     const int b = find_seq(prefix, n_seq, pos);
     const int L = slen[b];

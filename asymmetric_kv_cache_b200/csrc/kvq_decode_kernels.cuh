@@ -118,14 +118,6 @@ struct WarpState {
   float z[4];           // rows: value-min terms (j < J) and sum p (row J); cols heads
   float m[PK ? 2 : 1];  // running max, log2 domain: head lane/4, or (PK) heads
                         // 2(i&1), 2(i&1)+1
-  // (PK) sums of the value product's B operands, sum_t fp16(p_t s_tj): lane
-  // (g, i) holds, in vb[0] + vb[2], the sum for head g mod 4 and channel
-  // group j = 2 (g >= 4) + (i >= 2)  (groups 2 and 3 only when d / G = 4;
-  // with d / G = 1 group 0 twice)
-  float vb[4];
-#ifdef KVQ_VB_TWO
-  float vb2[4];
-#endif
 };
 
 // Query fragments of head g = lane/4 (zeros for a padding head), channels
@@ -689,22 +681,6 @@ __device__ __forceinline__ void softmax_pk(WarpState<D, KB, VB, G, true>& st, fl
       st.z[1] *= a1;
       st.z[2] *= a0;
       st.z[3] *= a1;
-      // the value-offset sums are indexed by head g mod 4 (their row), whose
-      // factor sits in lane h/2 as a0 (h even) or a1 (h odd)
-      const int h = (threadIdx.x >> 2) & 3;
-      const float x0 = __shfl_sync(0xffffffffu, a0, h >> 1);
-      const float x1 = __shfl_sync(0xffffffffu, a1, h >> 1);
-      const float av = (h & 1) ? x1 : x0;
-      st.vb[0] *= av;
-      st.vb[1] *= av;
-      st.vb[2] *= av;
-      st.vb[3] *= av;
-#ifdef KVQ_VB_TWO
-      st.vb2[0] *= av;
-      st.vb2[1] *= av;
-      st.vb2[2] *= av;
-      st.vb2[3] *= av;
-#endif
     }
     st.m[0] = n0;
     st.m[1] = n1;
@@ -841,365 +817,6 @@ __device__ __forceinline__ void tail_chunk_pk(WarpState<D, KB, VB, G, true>& st,
     const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
     const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
     mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Packed group loop, second form (GQA group of at most 4 heads).
-//
-// Query fragments: for each pair of k-steps (kt0, kt1) = (2kp, 2kp + 1) a
-// block of QP_STRIDE bytes with four 256-byte areas indexed by (head hh,
-// i): Y = q_hi, X = q_lo, NY = -q_hi, Z = zeros, each a quad of fp16 pairs
-// {(kt0, v0), (kt0, v1), (kt1, v0), (kt1, v1)} at channels 16kt + 8v + 2i,
-// +1.  A lane (g, i) of the S^T tiles owns column g: head g mod 4, its high
-// part (g < 4) or its residual (g >= 4); it reads
-//   y = Y, x = (low ? X : Z), yn = (low ? NY : Z), qb = (low ? X : Y),
-// and builds the B operand of the code tiles as
-//   b = x s' + (y s' - fp16(yn... )) = fma(x, s', fma(y, s', fp16(yn s')))
-// with s' = s_k / m (m the code field's factor): fp16(y s') on high lanes
-// and, on low lanes, the exact residual of that product plus x s'.  Lanes
-// g and g ^ 4 read the same Y bytes, and all high lanes the same zero quad,
-// so every quad load touches half the bytes of a plain per-lane layout.
-//
-// Per pair of k-steps the corrections are two tiles instead of four:
-//  * the code offset (1024 per code) against A = the four b registers of the
-//    pair (rows g: low channel halves, rows g + 8: high halves) and a
-//    constant B of -1024: row g of the result is -1024 times the sum of
-//    column g's operands;
-//  * the key-min bias sum_c q_c z_c against A = the qb quad and a B whose
-//    columns n < 4 carry the low channel halves' mins and n >= 4 the high
-//    halves' (rows g pair with columns n < 4, rows g + 8 with n >= 4).
-// Value codes enter their tiles in the same 1024-offset form as the keys
-// (one LOP3 per pair, no fp16 arithmetic): the factor m of a code field is
-// constant along a row (channel) of V^T, and the offset mass 1024 sum_t B_t
-// is accumulated by two more tiles per 16 tokens (vb); both are removed once
-// per piece (o = (O' - 1024 vb) / m).
-constexpr int QP_STRIDE = 1024;   // bytes per pair of k-steps (Y | X | NY | Z)
-// The packed group loop's form: 1 = process_group_pk (fp16 value unpack,
-// per-k-step bias and offset tiles), 2 = process_group_pk2 (this form).
-#ifndef KVQ_PK_FORM
-#define KVQ_PK_FORM 1
-#endif
-#ifndef KVQ_KSIDE_ACC
-#define KVQ_KSIDE_ACC 1
-#endif
-
-// A lane's four query quads: byte offsets from the fragment area `base`.
-template <int D>
-struct QPtrs {
-  const unsigned char* base;
-  uint32_t y, x, yn, qb;
-};
-
-template <int D>
-__device__ __forceinline__ QPtrs<D> qptrs_pk2(const unsigned char* qbase, int lane) {
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const uint32_t idx = (uint32_t)(((g8 & 3) * 4 + i4) * 16);
-  const bool low = g8 >= 4;
-  QPtrs<D> p;
-  p.base = qbase;
-  p.y = idx;
-  p.x = low ? 256 + idx : 768u;
-  p.yn = low ? 512 + idx : 768u;
-  p.qb = low ? 256 + idx : idx;
-  return p;
-}
-
-template <int D>
-__device__ __forceinline__ uint4 ldq(const QPtrs<D>& qp, uint32_t off, int kp) {
-  return *reinterpret_cast<const uint4*>(qp.base + off + kp * QP_STRIDE);
-}
-
-// 16-byte shared-memory load at a 32-bit shared address.
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-
-// The query conversion of the second packed form: NCW warps (64 threads per
-// 32 channels of d ... one (kp, head, i) item per thread) read the unit's
-// raw rows (head hh at hh * D elements, up to 4 heads) from the same bytes,
-// meet at a named barrier, then write the Y / X / NY quads and the zero
-// quads.  Heads at or past nh (and everything when !ok) are zeros.
-template <int D, int NCW>
-__device__ __forceinline__ void convert_query_pk2(int dtype, int nh, bool ok, int ctid,
-                                                  unsigned char* qbase, const unsigned char* raw) {
-  constexpr int KP = D / 32;
-  static_assert(KP * 16 <= NCW * 32, "one item per converting thread");
-  const float sc = kLog2e * rsqrtf((float)D);
-  const int kp = ctid >> 4, hh = (ctid >> 2) & 3, i4 = ctid & 3;
-  const bool item = ctid < KP * 16;
-  const bool valid = ok && item && hh < nh;
-  float2 x[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {   // u = 2 (kt - kt0) + v
-    const int c = 16 * (2 * kp + (u >> 1)) + 8 * (u & 1) + 2 * i4;
-    const int idx = hh * D + c;
-    float2 f = make_float2(0.f, 0.f);
-    if (valid) {
-      if (dtype == KVQ_FP16) {
-        f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
-      } else if (dtype == KVQ_BF16) {
-        f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
-      } else {
-        f = *reinterpret_cast<const float2*>(raw + 4 * idx);
-      }
-    }
-    x[u] = f;
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
-  if (item) {
-    uint32_t yw[4], xw[4], nw[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float x0 = x[u].x * sc, x1 = x[u].y * sc;
-      const __half2 h = __floats2half2_rn(x0, x1);
-      const float2 hf = __half22float2(h);
-      yw[u] = h2_as_u32(h);
-      nw[u] = yw[u] ^ 0x80008000u;   // -q_hi, exact
-      xw[u] = pack_h2(x0 - hf.x, x1 - hf.y);
-    }
-    unsigned char* blk = qbase + kp * QP_STRIDE + ((hh * 4 + i4) * 16);
-    *reinterpret_cast<uint4*>(blk) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
-    *reinterpret_cast<uint4*>(blk + 256) = make_uint4(xw[0], xw[1], xw[2], xw[3]);
-    *reinterpret_cast<uint4*>(blk + 512) = make_uint4(nw[0], nw[1], nw[2], nw[3]);
-    *reinterpret_cast<uint4*>(blk + 768) = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-template <int D, int KB, int VB, int G, int NACC = KVQ_KSIDE_ACC>
-__device__ __forceinline__ void kside_pk2(const unsigned char* __restrict__ sp,
-                                          const QPtrs<D>& qp, int lane, float (&s)[G / 16][4]) {
-  using C = DecCfg<D, KB, VB, G>;
-  constexpr int NM = G / 16;
-  constexpr int NT = G / 8;
-  constexpr int KP = C::KT / 2;
-  static_assert(C::J <= 4, "at most four value channel groups");
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const bool low = g8 >= 4;
-  const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
-  const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
-  const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
-  constexpr uint32_t kH2Neg1024 = 0xE400E400u;
-
-  float acc[NACC][NM][4];   // NACC independent accumulator sets (k-step pairs kp mod NACC)
-#pragma unroll
-  for (int a = 0; a < NACC; ++a)
-#pragma unroll
-    for (int mt = 0; mt < NM; ++mt) acc[a][mt][0] = acc[a][mt][1] = acc[a][mt][2] = acc[a][mt][3] = 0.f;
-  float bacc[4] = {0.f, 0.f, 0.f, 0.f};   // key-min bias (rows: column g, see above)
-  float cacc[4] = {0.f, 0.f, 0.f, 0.f};   // minus the code offset (rows: column g)
-  // key-code words of the lane's 8-token tiles, all at once when that is at
-  // most 8 registers, else per chunk of k-step pairs
-  constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
-  constexpr int KP_PER_CH = WCH * C::FK / 4;   // k-step pairs covered by a chunk
-  static_assert(KP % KP_PER_CH == 0, "k-step pairs split evenly into code chunks");
-  static_for<KP / KP_PER_CH>([&](auto ch_) {
-    constexpr int ch = decltype(ch_)::value;
-    uint32_t kw[NT][WCH];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      lds_words<WCH>(kcw + (nt * 32 + lane) * C::LWK + ch * WCH, kw[nt]);
-    static_for<KP_PER_CH>([&](auto kk_) {
-      constexpr int kp = ch * KP_PER_CH + decltype(kk_)::value;
-      const uint4 s4 = *reinterpret_cast<const uint4*>(ksw + 4 * kp);
-      const uint4 z4 = *reinterpret_cast<const uint4*>(kzw + 4 * kp);
-      const uint4 qy = ldq(qp, qp.y, kp);
-      const uint4 qx = ldq(qp, qp.x, kp);
-      const uint4 qn = ldq(qp, qp.yn, kp);
-      const uint4 qb = ldq(qp, qp.qb, kp);
-      const uint32_t sv[4] = {s4.x, s4.y, s4.z, s4.w};
-      const uint32_t yv[4] = {qy.x, qy.y, qy.z, qy.w};
-      const uint32_t xv[4] = {qx.x, qx.y, qx.z, qx.w};
-      const uint32_t nv[4] = {qn.x, qn.y, qn.z, qn.w};
-      uint32_t b[4];   // B operands: (kt0, v0), (kt0, v1), (kt1, v0), (kt1, v1)
-      static_for<4>([&](auto u_) {
-        constexpr int u = decltype(u_)::value;
-        constexpr int p = 2 * (2 * kp + (u >> 1)) + (u & 1);   // code pair of the operand
-        constexpr int e = code_log2_mul<KB, p % C::FK>();
-        const uint32_t sm = e ? hmul2_b(sv[u], h2_pow2_neg(e)) : sv[u];
-        b[u] = hfma2_b(xv[u], sm, hfma2_b(yv[u], sm, hmul2_b(nv[u], sm)));
-      });
-      static_for<2>([&](auto t_) {
-        constexpr int t = decltype(t_)::value;
-        constexpr int kt = 2 * kp + t;
-        constexpr int p0 = 2 * kt, p1 = 2 * kt + 1;
-        static_for<NM>([&](auto mt_) {
-          constexpr int mt = decltype(mt_)::value;
-          constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
-          mma16816(acc[kp % NACC][mt], code_offset<KB, p0 % C::FK>(kw[2 * mt][w0]),
-                   code_offset<KB, p0 % C::FK>(kw[2 * mt + 1][w0]),
-                   code_offset<KB, p1 % C::FK>(kw[2 * mt][w1]),
-                   code_offset<KB, p1 % C::FK>(kw[2 * mt + 1][w1]), b[2 * t], b[2 * t + 1]);
-        });
-      });
-      mma16816(cacc, b[0], b[1], b[2], b[3], kH2Neg1024, kH2Neg1024);
-      mma16816(bacc, qb.x, qb.y, qb.z, qb.w, low ? z4.y : z4.x, low ? z4.w : z4.z);
-    });
-  });
-  // per-column corrections: column g's bias is bacc[0] on lanes i < 2 plus
-  // bacc[2] on lanes i >= 2; its offset is cacc[0] + cacc[2] on any lane
-  float cor = (i4 < 2) ? bacc[0] + (cacc[0] + cacc[2]) : bacc[2];
-  cor += __shfl_xor_sync(0xffffffffu, cor, 2);    // column g
-  cor += __shfl_xor_sync(0xffffffffu, cor, 16);   // + column g ^ 4: head g mod 4
-  const int h0 = 2 * (i4 & 1);
-  const float cor0 = __shfl_sync(0xffffffffu, cor, 4 * h0);
-  const float cor1 = __shfl_sync(0xffffffffu, cor, 4 * h0 + 4);
-#pragma unroll
-  for (int mt = 0; mt < NM; ++mt) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float y = acc[0][mt][r];
-#pragma unroll
-      for (int a = 1; a < NACC; ++a) y += acc[a][mt][r];
-      const float x = y + __shfl_xor_sync(0xffffffffu, y, 2);   // hi + lo
-      s[mt][r] = x + ((r & 1) ? cor1 : cor0);
-    }
-  }
-}
-
-// The value side of a group in the offset form (second packed form).
-template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void vside_pk2(WarpState<D, KB, VB, G, true>& st,
-                                          const unsigned char* __restrict__ sp,
-                                          const uint32_t (&pt)[G / 16][2], int lane) {
-  using C = DecCfg<D, KB, VB, G>;
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const bool low = g8 >= 4;
-  const uint32_t* vcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VCODES);
-  const uint32_t* vsw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VSCALE);
-  const uint32_t* vzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_VMIN);
-  const int zrow = g8 < C::J ? g8 : 0;
-  const uint32_t zsel = g8 < C::J ? 0xFFFFFFFFu : 0u;
-  const uint32_t zone = g8 == C::J ? 0x3C003C00u : 0u;
-  const uint32_t one_lo = low ? 0u : 0x3C003C00u, one_hi = low ? 0x3C003C00u : 0u;
-  static_for<C::KV>([&](auto kv_) {
-    constexpr int kv = decltype(kv_)::value;
-    const uint32_t bp0 = pt[kv][0], bp1 = pt[kv][1];
-    const uint2 zz = *reinterpret_cast<const uint2*>(vzw + ((4 * kv + i4) * C::J + zrow) * 2);
-    mma16816(st.z, (zz.x & zsel) | zone, 0u, (zz.y & zsel) | zone, 0u, bp0, bp1);
-    uint32_t sw[2 * C::J];
-    lds_words<2 * C::J>(vsw + (4 * kv + i4) * C::J * 2, sw);
-    uint32_t bs[C::J][2];
-#pragma unroll
-    for (int j = 0; j < C::J; ++j) {
-      bs[j][0] = hmul2_b(bp0, sw[2 * j]);
-      bs[j][1] = hmul2_b(bp1, sw[2 * j + 1]);
-    }
-    // offset sums: rows g < 4 take groups (0, 1), rows g >= 4 (columns that
-    // repeat heads 0-3) groups (2, 3)
-    if constexpr (C::J == 4) {
-#ifdef KVQ_VB_TWO
-      mma16816(st.vb, bs[0][0], bs[0][1], bs[1][0], bs[1][1], one_lo, one_hi);
-      mma16816(st.vb2, bs[2][0], bs[2][1], bs[3][0], bs[3][1], one_lo, one_hi);
-#else
-      mma16816(st.vb, low ? bs[2][0] : bs[0][0], low ? bs[2][1] : bs[0][1],
-               low ? bs[3][0] : bs[1][0], low ? bs[3][1] : bs[1][1], one_lo, one_hi);
-#endif
-    } else if constexpr (C::J == 2) {
-      mma16816(st.vb, bs[0][0], bs[0][1], bs[1][0], bs[1][1], one_lo, one_hi);
-    } else {
-      mma16816(st.vb, bs[0][0], bs[0][1], bs[0][0], bs[0][1], one_lo, one_hi);
-    }
-    uint32_t vw[C::LWV];
-    lds_words<C::LWV>(vcw + (kv * 32 + lane) * C::LWV, vw);
-    static_for<C::MT>([&](auto mt_) {
-      constexpr int mt = decltype(mt_)::value;
-      constexpr int TPW = C::FV / 4;
-      constexpr int wd = mt / TPW, u = mt % TPW;
-      constexpr int j = (16 * mt) / G;
-      mma16816(st.o[mt], code_offset<VB, 2 * u>(vw[wd]), code_offset<VB, 2 * u + 1>(vw[wd]),
-               code_offset<VB, 2 * u + C::FV / 2>(vw[wd]),
-               code_offset<VB, 2 * u + 1 + C::FV / 2>(vw[wd]), bs[j][0], bs[j][1]);
-    });
-  });
-}
-
-template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void process_group_pk2(WarpState<D, KB, VB, G, true>& st,
-                                                  const unsigned char* __restrict__ sp,
-                                                  const QPtrs<D>& qp, int lane) {
-  constexpr int NM = G / 16;
-  float s[NM][4];
-  kside_pk2<D, KB, VB, G>(sp, qp, lane, s);
-  uint32_t pt[NM][2];
-  softmax_pk<D, NM, KB, VB, G>(st, s, pt);
-  vside_pk2<D, KB, VB, G>(st, sp, pt, lane);
-}
-
-// The field factors of the value-code rows of m-tile mt: rows g (channel
-// 16 mt + g) and rows g + 8 (see process_group_pk2).
-template <int VB>
-__host__ __device__ constexpr int vrow_log2_mul(int mt, int hi) {
-  return VB * ((2 * (mt % (16 / VB / 4)) + hi) % (8 / VB));
-}
-
-// fp16 tail chunk for the second packed form: the B operand of the key tile
-// is the lane's qb (q_hi on high lanes, q_lo on low lanes).
-template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void tail_chunk_pk2(WarpState<D, KB, VB, G, true>& st,
-                                               const unsigned char* __restrict__ buf, int T,
-                                               int kv, const QPtrs<D>& qp, int lane) {
-  using C = DecCfg<D, KB, VB, G>;
-  using TS = TailStage<D>;
-  const int g8 = lane >> 2, i4 = lane & 3;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
-  const unsigned char* k1 = k0 + 8 * TS::KROW;
-#pragma unroll
-  for (int kp = 0; kp < C::KT / 2; ++kp) {
-    const uint4 qb = ldq(qp, qp.qb, kp);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int kt = 2 * kp + t;
-      mma16816(acc, *reinterpret_cast<const uint32_t*>(k0 + 32 * kt),
-               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt),
-               *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16),
-               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16), t ? qb.z : qb.x,
-               t ? qb.w : qb.y);
-    }
-  }
-  const int t0 = 16 * kv + g8, t1 = t0 + 8;
-  float s[1][4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float x = acc[r] + __shfl_xor_sync(0xffffffffu, acc[r], 2);
-    s[0][r] = ((r < 2 ? t0 : t1) < T) ? x : -INFINITY;
-  }
-  uint32_t pt[1][2];
-  softmax_pk<D, 1, KB, VB, G>(st, s, pt);
-  const uint32_t ones = (g8 == C::J) ? 0x3C003C00u : 0u;
-  mma16816(st.z, ones, 0u, ones, 0u, pt[0][0], pt[0][1]);
-  const int ta = 16 * kv + 2 * i4, tb = ta + 8;
-  const uint32_t ma = (ta + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
-  const uint32_t mb = (tb + 1 < T) ? 0xFFFFFFFFu : 0x0000FFFFu;
-  const unsigned char* va = buf + TS::VOFF + i4 * TS::VROW + 4 * g8;
-  const unsigned char* vb = va + 4 * TS::VROW;
-#pragma unroll
-  for (int mt = 0; mt < C::MT; ++mt) {
-    const uint32_t a0 = *reinterpret_cast<const uint32_t*>(va + 64 * mt) & ma;
-    const uint32_t a1 = *reinterpret_cast<const uint32_t*>(va + 64 * mt + 32) & ma;
-    const uint32_t a2 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt) & mb;
-    const uint32_t a3 = *reinterpret_cast<const uint32_t*>(vb + 64 * mt + 32) & mb;
-    mma16816(st.o[mt], a0, a1, a2, a3, pt[0][0], pt[0][1]);
-  }
-}
-
-// After a warp's fp16 chunks and before its first group: bring O to the
-// scale of the offset-form rows (row factor m, exact in fp32).
-template <int D, int KB, int VB, int G>
-__device__ __forceinline__ void scale_rows_pk2(WarpState<D, KB, VB, G, true>& st) {
-#pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) {
-    const float f0 = (float)(1 << vrow_log2_mul<VB>(mt, 0));
-    const float f1 = (float)(1 << vrow_log2_mul<VB>(mt, 1));
-    st.o[mt][0] *= f0;
-    st.o[mt][1] *= f0;
-    st.o[mt][2] *= f1;
-    st.o[mt][3] *= f1;
   }
 }
 
@@ -1437,7 +1054,6 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     decode_kernel(const Geom g, const WsLayout w, const DecodeArgs a) {
   using C = DecCfg<D, KB, VB, G, WIDE>;
   constexpr int NW = C::NW;
-  constexpr bool PK2 = PK && KVQ_PK_FORM == 2;   // the second packed form
   static_assert(C::NST == 2, "the ring rotation below holds two stages");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int32_t wsum[NW];
@@ -1569,10 +1185,6 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
 #pragma unroll
     for (int r = 0; r < (PK ? 2 : 1); ++r) st.m[r] = -INFINITY;
-    st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;
-#ifdef KVQ_VB_TWO
-    st.vb2[0] = st.vb2[1] = st.vb2[2] = st.vb2[3] = 0.f;
-#endif
 
     int ngr, nh;         // groups in this piece, heads of the unit
     int gs0, glen;       // the piece's first group in its sequence, the length
@@ -1644,9 +1256,8 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
     }
     // while the blocks fly, the first warps turn the query rows into fragments
     {
-      // converting warps: one per k-step of d/16 (second packed form: one
-      // item per thread)
-      constexpr int NCW = PK2 ? (D / 32 * 16 + 31) / 32 : ((NW < D / 16) ? NW : D / 16);
+      // converting warps: one per k-step of d/16
+      constexpr int NCW = (NW < D / 16) ? NW : D / 16;
       if (warp < NCW) {
         bool got = mbar_wait_bounded(qbar, qphase & 1);
         got = __all_sync(0xffffffffu, got);
@@ -1660,13 +1271,9 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
           src = reinterpret_cast<const unsigned char*>(qr);
           sdt = KVQ_FP32;
         }
-        if constexpr (PK2)
-          convert_query_pk2<D, NCW>(sdt, nh, got, tid, smem + C::QA_OFF, src);
-        else
-          convert_query<D, PK, NCW>(sdt, nh, got, warp, lane, qsm, src);
+        convert_query<D, PK, NCW>(sdt, nh, got, warp, lane, qsm, src);
       }
     }
-    const QPtrs<D> qp = qptrs_pk2<D>(smem + C::QA_OFF, lane);
     ++qphase;
     __syncthreads();
     if (my_tail) {
@@ -1675,8 +1282,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
       unsigned char* tb = C::TAIL_EARLY ? smem + C::TAIL_OFF + warp * TailStage<D>::BYTES : wring;
       if constexpr (!WIN) {
         const Piece p = piece_s;
-        if constexpr (PK2) tail_chunk_pk2<D, KB, VB, G>(st, tb, p.Tb, warp, qp, lane);
-        else if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
+        if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
         else tail_chunk<D, KB, VB, G>(st, tb, p.Tb, warp, qsm, lane);
       } else {
         // fp16 chunks warp, warp + TAIL_CHUNKS, ... (sink chunks first, then
@@ -1694,14 +1300,12 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
             cp_async_wait_all();
             __syncwarp();
           }
-          if constexpr (PK2) tail_chunk_pk2<D, KB, VB, G>(st, tb, Tc, 0, qp, lane);
-          else if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
+          if constexpr (PK) tail_chunk_pk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
           else tail_chunk<D, KB, VB, G>(st, tb, Tc, 0, qsm, lane);
           c += C::TAIL_CHUNKS;
           if (c >= nck) break;
         }
       }
-      if constexpr (PK2) scale_rows_pk2<D, KB, VB, G>(st);   // before any group
       if (!C::TAIL_EARLY) {   // the ring is free again: start its copies
         __syncwarp();
         cur = claim_into(head);
@@ -1721,9 +1325,7 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         break;
       }
       phase ^= 1u << head;
-      if constexpr (PK2) {
-        process_group_pk2<D, KB, VB, G>(st, wring + head * C::BLK, qp, lane);
-      } else if constexpr (AK) {
+      if constexpr (AK) {
         if (narrow(cur)) {
           if constexpr (PK) process_group_pk<D, KB, VB, G, 2>(st, wring + head * C::BLK, qsm, lane);
           else process_group<D, KB, VB, G, 2>(st, wring + head * C::BLK, qsm, lane);
@@ -1780,47 +1382,16 @@ __global__ void __launch_bounds__(DecCfg<D, KB, VB, G, WIDE>::THREADS,
         // columns 4-7 repeat heads 0-3 bit for bit (the same B columns and
         // rescale factors), so lanes i4 >= 2 store the channel + 8 half of
         // lane i4 - 2's heads: every lane stores two values per m-tile.
-        // Value rows carry the code offset and the field factor m:
-        // o = (O' - 1024 sum_t B_t) / m, the sums of head h and channel
-        // group j held by lane 4h + 2(j & 1) (process_group_pk2).
         const int hh = 2 * (i4 & 1);
         const int co = (i4 >= 2) ? 8 : 0;
-        float sb0[C::J], sb1[C::J];   // second form: 1024 sum_t B_t per (group j, head)
-        if constexpr (PK2) {
-        const float vs = st.vb[0] + st.vb[2];
-#ifdef KVQ_VB_TWO
-        const float vs2 = st.vb2[0] + st.vb2[2];
-#pragma unroll
-        for (int j = 0; j < C::J; ++j) {
-          const float x = (j >= 2 && C::J == 4) ? vs2 : vs;
-          const int src = 4 * hh + 2 * (j & 1);
-          sb0[j] = 1024.f * __shfl_sync(0xffffffffu, x, src);
-          sb1[j] = 1024.f * __shfl_sync(0xffffffffu, x, src + 4);
-        }
-#else
-#pragma unroll
-        for (int j = 0; j < C::J; ++j) {
-          const int src = 4 * hh + 16 * (j >> 1) + 2 * (j & 1);   // lane (h + 4 (j >= 2), j odd)
-          sb0[j] = 1024.f * __shfl_sync(0xffffffffu, vs, src);
-          sb1[j] = 1024.f * __shfl_sync(0xffffffffu, vs, src + 4);
-        }
-#endif
-        }
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
           const int c = 16 * mt + g8 + co;
           const int j = (16 * mt) / G;
           const float o0 = (i4 >= 2) ? st.o[mt][2] : st.o[mt][0];
           const float o1 = (i4 >= 2) ? st.o[mt][3] : st.o[mt][1];
-          if constexpr (PK2) {
-            const float inv = (i4 >= 2) ? 1.f / (float)(1 << vrow_log2_mul<VB>(mt, 1))
-                                        : 1.f / (float)(1 << vrow_log2_mul<VB>(mt, 0));
-            mo[hh * RS + c] = (o0 - sb0[j]) * inv + zl0[j];
-            mo[(hh + 1) * RS + c] = (o1 - sb1[j]) * inv + zl1[j];
-          } else {
-            mo[hh * RS + c] = o0 + zl0[j];
-            mo[(hh + 1) * RS + c] = o1 + zl1[j];
-          }
+          mo[hh * RS + c] = o0 + zl0[j];
+          mo[(hh + 1) * RS + c] = o1 + zl1[j];
         }
         if (g8 == 0 && i4 < 2) {
           mo[(2 * i4) * RS + D] = st.m[0];
@@ -2036,11 +1607,10 @@ size_t smem_bytes(int n_seq) {   // + slot prefix and lengths of the sequences
   return DecCfg<D, KB, VB, G, WIDE>::SMEM_FIXED + 4 * (size_t)(2 * n_seq + 1);
 }
 
-// The position-adaptive variant exists for 4-bit keys (not in the second
-// packed form).
+// The position-adaptive variant exists for 4-bit keys.
 template <int KB, bool PK>
 constexpr bool has_ak() {
-  return KB == 4 && !(PK && KVQ_PK_FORM == 2);
+  return KB == 4;
 }
 
 template <int D, int KB, int VB, int G, bool PK, bool WIDE>

@@ -819,7 +819,6 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
       for (int m2 = 0; m2 < C::MT; ++m2) st.o[m2][0] = st.o[m2][1] = st.o[m2][2] = st.o[m2][3] = 0.f;
       st.z[0] = st.z[1] = st.z[2] = st.z[3] = 0.f;
       st.m[0] = st.m[1] = -INFINITY;
-      st.vb[0] = st.vb[1] = st.vb[2] = st.vb[3] = 0.f;   // unused here
       if (has_tail) {
         cp_async_wait_all();
         __syncwarp();
