@@ -708,7 +708,6 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
   static_assert(C::KT % KT_PER_CH == 0, "k-steps split evenly into code chunks");
   const int g8 = lane >> 2, i4 = lane & 3;
   const uint32_t f1 = g8 >= 4 ? 0x3C003C00u : 0u;    // (1, 1) on low lanes
-  const uint32_t nf1 = g8 >= 4 ? 0u : 0x3C003C00u;   // (1, 1) on high lanes
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
   const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
   const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
@@ -717,7 +716,13 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
   float acc[NM][4];
 #pragma unroll
   for (int mt = 0; mt < NM; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-  float bacc[4] = {0.f, 0.f, 0.f, 0.f};   // key-min bias minus the code offset, per column
+  float oacc[4] = {0.f, 0.f, 0.f, 0.f};   // minus the code offset, per column
+  // the key-min bias sum_c q_c z_c on an untransposed tile: A = the query
+  // quad (rows g: the high parts y of head g mod 4; rows g + 8: the low
+  // parts x, which lanes g < 4 hold as zeros), B = the mins (the same in
+  // every column): rows g + 4 and g + 12 (g < 4) hold the bias of head g -
+  // no operand to build
+  float zacc[4] = {0.f, 0.f, 0.f, 0.f};
   static_for<C::KT / KT_PER_CH>([&](auto ch_) {
     constexpr int ch = decltype(ch_)::value;
     uint32_t kw[NT][WCH];
@@ -736,11 +741,8 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
       const uint32_t h0 = hmul2_b(q4.x, sm0), h1 = hmul2_b(q4.z, sm1);
       const uint32_t b0 = hfma2_b(q4.y, sm0, hfma2_negc_b(q4.x, sm0, hmul2_b(h0, f1)));
       const uint32_t b1 = hfma2_b(q4.w, sm1, hfma2_negc_b(q4.z, sm1, hmul2_b(h1, f1)));
-      // the key-min bias against the raw query part of the column,
-      // y (1 - f) + x: q_hi on high lanes, q_lo on low lanes
-      const uint32_t qb0 = hfma2_b(q4.x, nf1, q4.y), qb1 = hfma2_b(q4.z, nf1, q4.w);
-      mma16816(bacc, z2.x, z2.x, z2.y, z2.y, qb0, qb1);
-      mma16816(bacc, kH2Neg1024, kH2Neg1024, kH2Neg1024, kH2Neg1024, b0, b1);
+      mma16816(zacc, q4.x, q4.y, q4.z, q4.w, z2.x, z2.y);
+      mma16816(oacc, kH2Neg1024, kH2Neg1024, kH2Neg1024, kH2Neg1024, b0, b1);
       static_for<NM>([&](auto mt_) {
         constexpr int mt = decltype(mt_)::value;
         constexpr int w0 = p0 / C::FK - ch * WCH, w1 = p1 / C::FK - ch * WCH;
@@ -751,12 +753,17 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
       });
     });
   });
+  // column 2 i4 + e (after the high + low sum) is head h = (2 i4 + e) mod 4,
+  // whose whole bias (high rows + low rows) sits in lane 4 (h + 4)
+  const float zb = zacc[0] + zacc[2];
+  const float bias0 = __shfl_sync(0xffffffffu, zb, 16 + 4 * ((2 * i4) & 3));
+  const float bias1 = __shfl_sync(0xffffffffu, zb, 16 + 4 * ((2 * i4 + 1) & 3));
 #pragma unroll
   for (int mt = 0; mt < NM; ++mt) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float x = acc[mt][r] + bacc[r & 1];
-      s[mt][r] = x + __shfl_xor_sync(0xffffffffu, x, 2);   // high + low columns
+      const float x = acc[mt][r] + oacc[r & 1];
+      s[mt][r] = (x + __shfl_xor_sync(0xffffffffu, x, 2)) + ((r & 1) ? bias1 : bias0);
     }
   }
 }
