@@ -128,8 +128,8 @@ __device__ __forceinline__ void f16_slot(WarpState<D, 4, 2, 32, PK>& st,
   const unsigned char* vbuf = buf + F::CH * F::ROW;
   uint32_t pt[2];
   if constexpr (PK) {
-    // S^T = K q^T: rows 16 tokens, columns q_hi (n < 4) / q_lo (n >= 4)
-    const uint32_t nf = g8 >= 4 ? 0u : 0x3C003C00u;
+    // S^T = K q^T: rows 16 tokens, columns q_hi (n < 4) / q_lo (n >= 4): the
+    // lanes' x words
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const unsigned char* k0 = kb + g8 * F::ROW + 4 * i4;
     const unsigned char* k1 = k0 + 8 * F::ROW;
@@ -139,8 +139,7 @@ __device__ __forceinline__ void f16_slot(WarpState<D, 4, 2, 32, PK>& st,
       mma16816(acc, *reinterpret_cast<const uint32_t*>(k0 + 32 * kt),
                *reinterpret_cast<const uint32_t*>(k1 + 32 * kt),
                *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16),
-               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16),
-               hfma2_b(q4.x, nf, q4.y), hfma2_b(q4.z, nf, q4.w));
+               *reinterpret_cast<const uint32_t*>(k1 + 32 * kt + 16), q4.y, q4.w);
     }
     float s[1][4];
 #pragma unroll

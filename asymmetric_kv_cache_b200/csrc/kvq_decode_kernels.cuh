@@ -120,54 +120,6 @@ struct WarpState {
                         // 2(i&1), 2(i&1)+1
 };
 
-// Query fragments of head g = lane/4 (zeros for a padding head), channels
-// 16kt + 2i + {0,1} (v = 0) and + 8 (v = 1), i = lane & 3: q is scaled by
-// log2(e)/sqrt(d), split into fp16 high and low parts and stored per lane
-// as qs[kt * 32 + lane] = {hi v0, lo v0, hi v1, lo v1} - the A quad of the
-// q.k tiles (rows g: high part, rows g + 8: low part).  The unit's raw rows
-// (head g at g * D elements) were copied into the same bytes; every lane
-// reads its values before any lane writes.
-template <int D>
-__device__ __forceinline__ void load_query(int dtype, bool valid, int lane,
-                                           uint4* __restrict__ qs) {
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const float sc = kLog2e * rsqrtf((float)D);
-  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
-  float2 x[D / 16][2];
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int idx = g8 * D + 16 * kt + 8 * v + 2 * i4;
-      float2 f = make_float2(0.f, 0.f);
-      if (valid) {
-        if (dtype == KVQ_FP16) {
-          f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
-        } else if (dtype == KVQ_BF16) {
-          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
-        } else {
-          f = *reinterpret_cast<const float2*>(raw + 4 * idx);
-        }
-      }
-      x[kt][v] = f;
-    }
-  }
-  __syncwarp();
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
-    uint32_t w[4];
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const float x0 = x[kt][v].x * sc, x1 = x[kt][v].y * sc;
-      const __half2 h = __floats2half2_rn(x0, x1);
-      const float2 hf = __half22float2(h);
-      w[2 * v] = h2_as_u32(h);
-      w[2 * v + 1] = pack_h2(x0 - hf.x, x1 - hf.y);
-    }
-    qs[kt * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 // Online-softmax update for new logits in the S tile layout: s[nt] =
 // {(head g, token 8nt + 2i), (head g, token 8nt + 2i + 1)} (g = lane/4,
 // i = lane&3).  Produces the fp16 probabilities pt[nt] in the same places,
@@ -479,61 +431,24 @@ __device__ __forceinline__ void tail_chunk(WarpState<D, KB, VB, G>& st,
 // tiles), columns n = heads 0-3 with q' rounded to fp16 (n < 4) and the
 // rounding residual of the same heads (n >= 4).  Lane (g, i) then holds the
 // B operand of column g, so each lane computes either a high or a low part:
-// its query words (load_query_pk) are y = q_hi and x = (low lane ? q_lo : 0),
-// and with f = (low lane ? 1 : 0),
-//   h = y s,  B = x s + (y s - f h)
-// gives h on high lanes and the exact residual of h on low lanes with the
-// same instructions.  The two halves of a logit meet with one shuffle
-// (lane i and i ^ 2 hold columns n and n + 4).
-
-template <int D>
-__device__ __forceinline__ void load_query_pk(int dtype, int nh, bool ok, int lane,
-                                              uint4* __restrict__ qs) {
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const int hh = g8 & 3;
-  const bool low = g8 >= 4;
-  const bool valid = ok && hh < nh;
-  const float sc = kLog2e * rsqrtf((float)D);
-  const unsigned char* raw = reinterpret_cast<const unsigned char*>(qs);
-  float2 x[D / 16][2];
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int idx = hh * D + 16 * kt + 8 * v + 2 * i4;
-      float2 f = make_float2(0.f, 0.f);
-      if (valid) {
-        if (dtype == KVQ_FP16) {
-          f = __half22float2(*reinterpret_cast<const __half2*>(raw + 2 * idx));
-        } else if (dtype == KVQ_BF16) {
-          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(raw + 2 * idx));
-        } else {
-          f = *reinterpret_cast<const float2*>(raw + 4 * idx);
-        }
-      }
-      x[kt][v] = f;
-    }
-  }
-  __syncwarp();
-#pragma unroll
-  for (int kt = 0; kt < D / 16; ++kt) {
-    uint32_t w[4];
-#pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const float x0 = x[kt][v].x * sc, x1 = x[kt][v].y * sc;
-      const __half2 h = __floats2half2_rn(x0, x1);
-      const float2 hf = __half22float2(h);
-      w[2 * v] = h2_as_u32(h);
-      w[2 * v + 1] = low ? pack_h2(x0 - hf.x, x1 - hf.y) : 0u;
-    }
-    qs[kt * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
+// its query words (convert_query) are y = (low lane ? q_hi : 0) and
+// x = (low lane ? q_lo : q_hi), and
+//   h = y s,  B = x s + (y s - h)
+// gives fp16(q_hi s) on high lanes (y = 0) and the exact residual of that
+// product on low lanes with the same instructions.  The two halves of a
+// logit meet with one shuffle (lane i and i ^ 2 hold columns n and n + 4).
+// The fp16 tail's B operand is x itself (q_hi on high lanes, q_lo on low).
 
 // The query conversion split over NCW warps (k-tiles cw, cw + NCW, ...):
 // every converting warp reads its raw values first, the warps meet at a
-// named barrier, then they write their fragments into the same bytes.  The
-// layouts are those of load_query (PK = false) and load_query_pk (PK).
+// named barrier, then they write their fragments into the same bytes.
+// q is scaled by log2(e)/sqrt(d) and split into fp16 high and low parts; the
+// fragments of k-step kt sit at qs[kt * 32 + lane] as a quad over the
+// channels 16kt + 2i + {0,1} (v = 0) and + 8 (v = 1), i = lane & 3:
+//   PK = false: {hi v0, lo v0, hi v1, lo v1} of head lane/4 - the A quad of
+//     the q.k tiles (rows g: high part, rows g + 8: low part);
+//   PK: {y v0, x v0, y v1, x v1} of head (lane/4) mod 4 (see above).
+// A padding head gets zeros.
 template <int D, bool PK, int NCW>
 __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw, int lane,
                                               uint4* qs, const unsigned char* raw) {
@@ -575,9 +490,10 @@ __device__ __forceinline__ void convert_query(int dtype, int nh, bool ok, int cw
       const float x0 = x[j][v].x * sc, x1 = x[j][v].y * sc;
       const __half2 h = __floats2half2_rn(x0, x1);
       const float2 hf = __half22float2(h);
-      wv[2 * v] = h2_as_u32(h);
+      const uint32_t hi = h2_as_u32(h);
       const uint32_t lo = pack_h2(x0 - hf.x, x1 - hf.y);
-      wv[2 * v + 1] = PK ? (low ? lo : 0u) : lo;
+      wv[2 * v] = (PK && !low) ? 0u : hi;
+      wv[2 * v + 1] = (PK && !low) ? hi : lo;
     }
     qs[kt * 32 + lane] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
   }
@@ -706,8 +622,7 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
   constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
   constexpr int KT_PER_CH = WCH * C::FK / 2;
   static_assert(C::KT % KT_PER_CH == 0, "k-steps split evenly into code chunks");
-  const int g8 = lane >> 2, i4 = lane & 3;
-  const uint32_t f1 = g8 >= 4 ? 0x3C003C00u : 0u;    // (1, 1) on low lanes
+  const int i4 = lane & 3;
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
   const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);
   const uint32_t* kzw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KMIN) + i4 * (D / 8);
@@ -718,10 +633,9 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
   for (int mt = 0; mt < NM; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
   float oacc[4] = {0.f, 0.f, 0.f, 0.f};   // minus the code offset, per column
   // the key-min bias sum_c q_c z_c on an untransposed tile: A = the query
-  // quad (rows g: the high parts y of head g mod 4; rows g + 8: the low
-  // parts x, which lanes g < 4 hold as zeros), B = the mins (the same in
-  // every column): rows g + 4 and g + 12 (g < 4) hold the bias of head g -
-  // no operand to build
+  // quad (rows g: y of head g mod 4, rows g + 8: x), B = the mins (the same
+  // in every column): rows g + 4 (q_hi) and g + 12 (q_lo), g < 4, hold the
+  // bias of head g - no operand to build
   float zacc[4] = {0.f, 0.f, 0.f, 0.f};
   static_for<C::KT / KT_PER_CH>([&](auto ch_) {
     constexpr int ch = decltype(ch_)::value;
@@ -739,8 +653,8 @@ __device__ __forceinline__ void kside_pk(const unsigned char* __restrict__ sp,
       const uint32_t sm0 = e0 ? hmul2_b(s2.x, h2_pow2_neg(e0)) : s2.x;
       const uint32_t sm1 = e1 ? hmul2_b(s2.y, h2_pow2_neg(e1)) : s2.y;
       const uint32_t h0 = hmul2_b(q4.x, sm0), h1 = hmul2_b(q4.z, sm1);
-      const uint32_t b0 = hfma2_b(q4.y, sm0, hfma2_negc_b(q4.x, sm0, hmul2_b(h0, f1)));
-      const uint32_t b1 = hfma2_b(q4.w, sm1, hfma2_negc_b(q4.z, sm1, hmul2_b(h1, f1)));
+      const uint32_t b0 = hfma2_b(q4.y, sm0, hfma2_negc_b(q4.x, sm0, h0));
+      const uint32_t b1 = hfma2_b(q4.w, sm1, hfma2_negc_b(q4.z, sm1, h1));
       mma16816(zacc, q4.x, q4.y, q4.z, q4.w, z2.x, z2.y);
       mma16816(oacc, kH2Neg1024, kH2Neg1024, kH2Neg1024, kH2Neg1024, b0, b1);
       static_for<NM>([&](auto mt_) {
@@ -787,15 +701,15 @@ __device__ __forceinline__ void tail_chunk_pk(WarpState<D, KB, VB, G, true>& st,
   using C = DecCfg<D, KB, VB, G>;
   using TS = TailStage<D>;
   const int g8 = lane >> 2, i4 = lane & 3;
-  const uint32_t nf = g8 >= 4 ? 0u : 0x3C003C00u;   // (1, 1) on high lanes
-  // S^T = K q^T: rows 16 tokens, columns q_hi (n < 4) / q_lo (n >= 4)
+  // S^T = K q^T: rows 16 tokens, columns q_hi (n < 4) / q_lo (n >= 4): the
+  // lanes' x words
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const unsigned char* k0 = buf + g8 * TS::KROW + 4 * i4;
   const unsigned char* k1 = k0 + 8 * TS::KROW;
 #pragma unroll
   for (int kt = 0; kt < C::KT; ++kt) {
     const uint4 q4 = qsm[kt * 32 + lane];
-    const uint32_t b0 = hfma2_b(q4.x, nf, q4.y), b1 = hfma2_b(q4.z, nf, q4.w);
+    const uint32_t b0 = q4.y, b1 = q4.w;
     mma16816(acc, *reinterpret_cast<const uint32_t*>(k0 + 32 * kt),
              *reinterpret_cast<const uint32_t*>(k1 + 32 * kt),
              *reinterpret_cast<const uint32_t*>(k0 + 32 * kt + 16),

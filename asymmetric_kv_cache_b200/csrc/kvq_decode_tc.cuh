@@ -735,19 +735,18 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int h = 2 * hp + hh;
-          qh[hh][u] = qw[(kt * 32 + 4 * h + ii) * 4 + 2 * half];
+          qh[hh][u] = qw[(kt * 32 + 4 * (h + 4) + ii) * 4 + 2 * half];
           ql[hh][u] = qw[(kt * 32 + 4 * (h + 4) + ii) * 4 + 2 * half + 1];
         }
       }
       // bias fragments: columns 0-3 the heads' high parts, 4-7 their low parts
       uint32_t qb[C::KT][2];
       {
-        const uint32_t nf1 = g8 >= 4 ? 0u : 0x3C003C00u;
 #pragma unroll
-        for (int kt = 0; kt < C::KT; ++kt) {
+        for (int kt = 0; kt < C::KT; ++kt) {   // the lanes' x words
           const uint4 q4 = qsm[kt * 32 + lane];
-          qb[kt][0] = hfma2_b(q4.x, nf1, q4.y);
-          qb[kt][1] = hfma2_b(q4.z, nf1, q4.w);
+          qb[kt][0] = q4.y;
+          qb[kt][1] = q4.w;
         }
       }
       for (int i = 0; i < ntiles; ++i) {
