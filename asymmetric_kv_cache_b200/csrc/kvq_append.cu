@@ -39,14 +39,10 @@ namespace {
 template <int D, int G, int KB, int VB>
 struct AppCfg {
   static constexpr int J = D / G;
-  static constexpr int QK = (1 << KB) - 1;
   static constexpr int QV = (1 << VB) - 1;
-  static constexpr int FK = 16 / KB;           // code pairs per 32-bit word
-  static constexpr int FV = 16 / VB;
-  static constexpr int KWORDS_PER_LANE = D * KB / 128;   // per 8-token tile
-  static constexpr int VWORDS_PER_LANE = D * VB / 64;    // per 16-token tile
-  static constexpr int KWORDS = G * D * KB / 32;
-  static constexpr int VWORDS = G * D * VB / 32;
+  static constexpr int FV = 16 / VB;                  // value-code pairs per 32-bit word
+  static constexpr int VWORDS_PER_LANE = D * VB / 64;  // per 16-token tile
+  static constexpr int VWORDS = G * D * VB / 32;       // (key words: key_codes)
   // dynamic shared memory: fp16 K and V of the group (token rows padded by
   // 16 bytes, so that rows fall 4 banks apart), the fp16 metadata in slot
   // order, and per key channel / per (token, value group) the fp32

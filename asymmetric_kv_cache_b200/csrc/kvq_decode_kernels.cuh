@@ -227,7 +227,7 @@ __device__ __forceinline__ void process_group(WarpState<D, KB, VB, G>& st,
   constexpr int WCH = (NT * C::LWK <= 8) ? C::LWK : (C::LWK >= 2 ? 2 : 1);
   constexpr int KT_PER_CH = WCH * C::FK / 2;   // k-steps covered by a chunk
   static_assert(C::KT % KT_PER_CH == 0, "k-steps split evenly into code chunks");
-  const int g8 = lane >> 2, i4 = lane & 3;
+  const int i4 = lane & 3;
 
   const uint32_t* kcw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KCODES);
   const uint32_t* ksw = reinterpret_cast<const uint32_t*>(sp + C::SEC_KSCALE) + i4 * (D / 8);

@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(TcCfg<KB>::THREADS, 1)
   using T = TcCfg<KB>;
   using C = typename T::C;
   constexpr int D = 128, G = 32, VB = 2;
-  extern __shared__ __align__(1024) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char tc_smem[];
+  unsigned char* const smem = tc_smem;
   __shared__ int32_t wsum[T::NWARP];
   __shared__ int32_t ticket_flag[3];
   __shared__ uint32_t tmem_base_s;
