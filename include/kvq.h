@@ -247,7 +247,11 @@ KVQ_API kvq_status kvq_reset(kvq_cache* cache, void* stream);
  * counts, read before the call returns.
  * Performs prefill quantization (whole groups straight from the input),
  * per-step appends into the fp16 tail and the flush of a tail that reaches
- * R + G tokens (its oldest G become a group), all in one launch.  The kernel
+ * R + G tokens (its oldest G become a group), all in one launch.  The launch
+ * is a programmatic dependent of the previous kernel on the stream: its
+ * CTAs may become resident while that kernel runs, and they wait for it to
+ * complete before they read or write any memory (inputs included), so
+ * stream order holds as for a plain launch.  The kernel
  * takes the current lengths from the device copy and advances it, so an
  * append captured in a CUDA graph may be replayed provided every n_new[b] <
  * G (the launch shape then does not depend on the lengths); after replays,
