@@ -411,6 +411,25 @@ def run_fp16_baseline(wl, ks, vs, q, stream, device, iters=200):
             "achieved_gbs": round(byts / us / 1e3, 1), "launches": iters, "copies": copies}
 
 
+def decode_bytes_one_seq(n, G, d, kb, vb, hkv, hq, window=0, sink=0, akvq_delta=0):
+    """Algorithmic bytes of one decode over one sequence of n tokens: every
+    quantized group's block (codes + fp16 scale/min pairs; with adaptive key
+    widths the 2-bit groups' smaller block), 4d bytes per fp16 token (tail
+    and sink), and the fp16 queries.  Returns (bytes, quantized tokens)."""
+    blk = G * d * (kb + vb) // 8 + 8 * d
+    after = n - min(n, sink)                                  # tokens after the sink
+    nq = G * ((after - window) // G) if after > window else 0   # quantized tokens
+    if akvq_delta:
+        # groups wholly before Delta or ending after n - Delta keep 4-bit keys
+        blk2 = G * d * (2 + vb) // 8 + 8 * d
+        wide = sum(1 for g in range(nq // G)
+                   if (g + 1) * G <= akvq_delta or (g + 1) * G > n - akvq_delta)
+        qbytes = wide * blk + (nq // G - wide) * blk2
+    else:
+        qbytes = (nq // G) * blk
+    return hkv * (qbytes + (n - nq) * 4 * d) + hq * d * 2, nq
+
+
 def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akvq_delta=0,
                      rotate=0):
     """Decode alone on the 128k-token long-context workload (batch 1, 32 q /
@@ -435,18 +454,8 @@ def run_long_context(stream, device, iters=100, window=0, fp16=True, sink=0, akv
                          w.batch, n, window=window, sink=sink, akvq_delta=akvq_delta,
                          rotate=rotate)
     G, d = w.group, w.head_dim
-    blk = G * d * (kb + w.v_bits) // 8 + 8 * d
-    after = n - min(n, sink)                                  # tokens after the sink
-    nq = G * ((after - window) // G) if after > window else 0   # quantized tokens
-    if akvq_delta:
-        # groups wholly before Delta or ending after n - Delta keep 4-bit keys
-        blk2 = G * d * (2 + w.v_bits) // 8 + 8 * d
-        wide = sum(1 for g in range(nq // G)
-                   if (g + 1) * G <= akvq_delta or (g + 1) * G > n - akvq_delta)
-        qbytes = wide * blk + (nq // G - wide) * blk2
-    else:
-        qbytes = (nq // G) * blk
-    byts = w.n_kv_heads * (qbytes + (n - nq) * 4 * d) + w.n_q_heads * d * 2
+    byts, nq = decode_bytes_one_seq(n, G, d, kb, w.v_bits, w.n_kv_heads, w.n_q_heads,
+                                    window=window, sink=sink, akvq_delta=akvq_delta)
     copies = max(2, math.ceil(3 * L2_BYTES / byts))
     k = torch.from_numpy(np.concatenate(w.keys)).to(device)
     v = torch.from_numpy(np.concatenate(w.values)).to(device)
