@@ -10,7 +10,10 @@ dequantized keys.  Pinned here: hand-worked requantization examples, the
 widths after any append history against a closed form of the region sizes
 derived separately, the key bytes per sequence in closed form, decode equal
 to plain attention on keys exactly representable at both widths whatever
-the history, and the history dependence of the bytes (not of the widths).
+the history, the history dependence of the bytes (not of the widths), a
+prefill's blocks equal to the plain 4-bit and 2-bit caches' blocks group by
+group, and Delta beyond the length reducing to the plain 4-bit cache and
+its decode.
 """
 import dataclasses
 import json
@@ -154,3 +157,46 @@ def test_bytes_depend_on_the_history_widths_do_not():
     for g, bits in enumerate(a["bits"]):
         if bits == 4:
             assert np.array_equal(a["blocks"][:, g], b["blocks"][:, g])
+
+
+def test_prefill_image_selects_plain_k4_and_k2_blocks():
+    """One append (a prefill): every group is quantized from its fp16 keys at
+    its width, so its block is the plain 4-bit cache's block or the plain
+    2-bit cache's block (from the start of the slot), group by group."""
+    G, delta, d = 32, 96, 64
+    cfg = _cfg(G, delta, d)
+    rng = np.random.default_rng(21)
+    n = 20 * G + 11
+    k = (rng.standard_normal((n, 2, d)) * np.exp(rng.standard_normal((1, 2, d)))).astype(np.float16)
+    v = rng.standard_normal((n, 2, d)).astype(np.float16)
+    img = o.akvq_cache_image(cfg, k, v, [n])
+    c4 = o.cache_image(dataclasses.replace(cfg, akvq_delta=0), k, v)
+    c2 = o.cache_image(dataclasses.replace(cfg, k_bits=2, akvq_delta=0), k, v)
+    n2 = o.block_sections(dataclasses.replace(cfg, k_bits=2))["total"][1]
+    assert set(img["bits"]) == {2, 4}
+    for g, bits in enumerate(img["bits"]):
+        if bits == 4:
+            assert np.array_equal(img["blocks"][:, g], c4["blocks"][:, g])
+        else:
+            assert np.array_equal(img["blocks"][:, g, :n2], c2["blocks"][:, g])
+            assert not img["blocks"][:, g, n2:].any()
+
+
+@pytest.mark.parametrize("chunks", [[700], [1] * 700, [5, 300, 1, 1, 393]])
+def test_delta_beyond_the_length_is_the_plain_4bit_cache(chunks):
+    """Delta >= n: every group is early or recent, so the cache is the plain
+    4-bit cache whatever the history, and so is the decode."""
+    G, d = 32, 64
+    n = sum(chunks)
+    cfg = _cfg(G, 1024, d)
+    rng = np.random.default_rng(22)
+    k = rng.standard_normal((n, 1, d)).astype(np.float16)
+    v = rng.standard_normal((n, 1, d)).astype(np.float16)
+    q = rng.standard_normal((1, d))
+    img = o.akvq_cache_image(cfg, k, v, chunks)
+    plain = dataclasses.replace(cfg, akvq_delta=0)
+    c4 = o.cache_image(plain, k, v)
+    assert img["bits"] == [4] * (n // G)
+    assert np.array_equal(img["blocks"], c4["blocks"])
+    assert np.allclose(o.akvq_decode(cfg, k, v, q, chunks), o.decode(plain, k, v, q), rtol=0,
+                       atol=1e-12)
